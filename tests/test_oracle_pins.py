@@ -1,0 +1,623 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Every check compares the oracle with something other than itself: the worked
+example printed on the Ultralytics "FP4" page, the E2M1 value set listed
+there, independent codec libraries (ml_dtypes, torch), scipy's Hadamard
+matrix, Triton's CPU-interpreted Philox, closed-form invariants and brute
+force over every scale code.  CPU only.
+"""
+import itertools
+import os
+import subprocess
+import sys
+
+import ml_dtypes as md
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+from mxfp4_block_scaled_fos_b200 import workloads
+
+E2M1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+
+
+def _read_golden(path):
+    rows = []
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def _f4_codes(v):
+    """ml_dtypes' E2M1 conversion (RNE, saturating) as 4-bit codes."""
+    return np.asarray(v, np.float32).astype(md.float4_e2m1fn).view(np.uint8) & 0xF
+
+
+def _e4m3_sat_codes(v):
+    v = np.clip(np.asarray(v, np.float32), -448.0, 448.0)
+    return v.astype(md.float8_e4m3fn).view(np.uint8)
+
+
+def _e4m3_val(code):
+    return np.asarray(code, np.uint8).view(md.float8_e4m3fn).astype(np.float64)
+
+
+def _e2m1_val(code):
+    return (np.asarray(code, np.uint8) & 0xF).view(md.float4_e2m1fn).astype(np.float64)
+
+
+# ------------------------------------------------------------------ page pins
+def test_page_example_mae(golden_dir):
+    """FP4 page, "Como funciona FP4" worked example: 0.7238 / 0.0901 / 0.0747."""
+    x = workloads.page_example_input().numpy()
+    for block, expect in _read_golden(os.path.join(golden_dir, "page_example_mae.txt")):
+        mae = oracle.page_example_mae(x, int(block))
+        assert abs(mae - float(expect)) < 5e-5, (block, mae, expect)
+
+
+def test_page_example_mae_matches_torch_recomputation():
+    """The same MAEs via torch ops run as a separate program (argmin tie rule)."""
+    x = workloads.page_example_input()
+    grid = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    for block in (4096, 32, 16):
+        blocks = x.reshape(-1, block)
+        scale = blocks.abs().amax(dim=1, keepdim=True) / 6.0
+        nearest = ((blocks.abs() / scale).unsqueeze(-1) - grid).abs().argmin(dim=-1)
+        deq = grid[nearest] * blocks.sign() * scale
+        err = (deq.flatten() - x).abs().double().mean().item()
+        assert abs(err - oracle.page_example_mae(x.numpy(), block)) < 1e-6
+
+
+def test_e2m1_value_set(golden_dir):
+    """FP4 page intro: E2M1 represents exactly 0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6."""
+    vals = [float(v) for v in _read_golden(os.path.join(golden_dir, "e2m1_values.txt"))[0]]
+    decoded = sorted({oracle.e2m1_decode(c) for c in range(16)})
+    expect = sorted(set(vals) | {-v for v in vals})
+    assert decoded == expect
+    # magnitudes are monotone in the code and the sign is bit 3
+    for c in range(8):
+        assert oracle.e2m1_decode(c) == vals[c]
+        assert oracle.e2m1_decode(c | 8) == -vals[c] or (c == 0)
+
+
+# ------------------------------------------------------------------ codecs
+def _structured_f32(rng, n_random=1 << 20):
+    hi = np.arange(1 << 16, dtype=np.uint32) << 16
+    lows = np.array([0, 1, 0x7FFF, 0x8000, 0x8001, 0xFFFF], np.uint32)
+    pats = (hi[:, None] | lows[None, :]).ravel()
+    rnd = rng.integers(0, 1 << 32, n_random, dtype=np.uint64).astype(np.uint32)
+    pats = np.concatenate([pats, rnd])
+    f = pats.view(np.float32)
+    return f[np.isfinite(f)]
+
+
+def test_e2m1_encode_vs_ml_dtypes():
+    rng = np.random.default_rng(1)
+    f = _structured_f32(rng)
+    # exact ties and their neighbours
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0], np.float32)
+    nb = np.concatenate([ties, np.nextafter(ties, 0), np.nextafter(ties, 10)])
+    f = np.concatenate([f, nb, -nb, [0.0, -0.0, np.inf, -np.inf]]).astype(np.float32)
+    got = oracle.e2m1_encode(f)
+    want = _f4_codes(f)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (f[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_e2m1_exhaustive_bf16_patterns():
+    pats = (np.arange(1 << 16, dtype=np.uint32) << 16).view(np.float32)
+    pats = pats[np.isfinite(pats)]
+    assert np.array_equal(oracle.e2m1_encode(pats), _f4_codes(pats))
+
+
+def test_e4m3_decode_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    want = codes.view(md.float8_e4m3fn).astype(np.float32)
+    got = np.array([oracle.e4m3_decode(int(c)) for c in codes], np.float32)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), want[~nan].view(np.uint32))
+    assert oracle.e4m3_decode(0x7E) == 448.0
+
+
+def test_e4m3_encode_vs_ml_dtypes_saturating():
+    rng = np.random.default_rng(2)
+    f = _structured_f32(rng, 1 << 18)
+    f = f[np.abs(f) < 1e6]
+    # every midpoint between neighbouring E4M3 values and its neighbours
+    vals = np.arange(0, 0x7F, dtype=np.uint8).view(md.float8_e4m3fn).astype(np.float64)
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)
+    extra = np.concatenate([mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9),
+                            vals.astype(np.float32), [448.0, 464.0, 470.0, 480.0, 1e30]])
+    f = np.concatenate([f, extra, -extra]).astype(np.float32)
+    got = oracle.e4m3_encode(f)
+    want = _e4m3_sat_codes(f)
+    # ml_dtypes keeps -0 for tiny negatives; so does the oracle (sign bit)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (f[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_e8m0_decode_and_exponent():
+    codes = np.arange(255, dtype=np.uint8)
+    want = codes.view(md.float8_e8m0fnu).astype(np.float64)
+    got = np.array([lib_e8m0(int(c)) for c in codes])
+    assert np.array_equal(got, want)
+    rng = np.random.default_rng(3)
+    exps = np.arange(-149, 128)
+    mant = rng.random((exps.size, 8)) + 1.0
+    a = (mant * np.exp2(exps)[:, None]).astype(np.float32).ravel()
+    pw = np.exp2(exps).astype(np.float32)
+    a = np.concatenate([a, pw, np.nextafter(pw, 0), np.nextafter(pw, np.inf),
+                        [np.float32(3.4e38)]]).astype(np.float32)
+    a = a[(a > 0) & np.isfinite(a)]
+    want = np.clip(np.floor(np.log2(a.astype(np.float64))) - 2, -127, 127).astype(np.int32)
+    assert np.array_equal(oracle.e8m0_exponent(a), want)
+    assert oracle.e8m0_exponent(np.zeros(1, np.float32))[0] == -127
+
+
+def lib_e8m0(c):
+    return oracle.lib().or_e8m0_decode(c)
+
+
+def test_bf16_rne_vs_torch():
+    rng = np.random.default_rng(4)
+    f = _structured_f32(rng, 1 << 18)
+    f = f[np.abs(f) < 3e38]
+    got = oracle.f32_to_bf16(f)
+    want = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+
+
+# ------------------------------------------------------------------ Philox / RHT
+_TRITON_PROG = r"""
+import os, sys, json
+os.environ["TRITON_INTERPRET"] = "1"
+import numpy as np, torch, triton, triton.language as tl
+
+@triton.jit
+def k(out_ptr, seed, c0_ptr, c1_ptr, c2_ptr, c3_ptr, N: tl.constexpr):
+    i = tl.arange(0, N)
+    c0 = tl.load(c0_ptr + i); c1 = tl.load(c1_ptr + i)
+    c2 = tl.load(c2_ptr + i); c3 = tl.load(c3_ptr + i)
+    a, b, c, d = tl.philox(seed, c0, c1, c2, c3)
+    tl.store(out_ptr + i * 4 + 0, a)
+    tl.store(out_ptr + i * 4 + 1, b)
+    tl.store(out_ptr + i * 4 + 2, c)
+    tl.store(out_ptr + i * 4 + 3, d)
+
+cases = json.loads(sys.stdin.read())
+res = []
+for seed, ctrs in cases:
+    n = len(ctrs)
+    cols = [torch.tensor([c[j] for c in ctrs], dtype=torch.int64).to(torch.uint32) for j in range(4)]
+    out = torch.zeros(4 * n, dtype=torch.uint32)
+    k[(1,)](out, seed, *cols, N=n)
+    res.append([int(v) for v in out.tolist()])
+print(json.dumps(res))
+"""
+
+
+def test_philox_vs_triton_interpreter():
+    """Philox4x32-10 against Triton's own implementation run on the CPU."""
+    rng = np.random.default_rng(5)
+    seeds = [0, 1, 0x9E3779B97F4A7C15 & ((1 << 63) - 1), (123 << 32) | 77]
+    cases = []
+    for s in seeds:
+        ctr = rng.integers(0, 1 << 32, (16, 4), dtype=np.uint64)
+        ctr[0] = 0
+        ctr[1] = [0, 0, 1, 0]
+        ctr[2] = [0xFFFFFFFF] * 4
+        cases.append([int(s), ctr.tolist()])
+    import json
+    p = subprocess.run([sys.executable, "-c", _TRITON_PROG], input=json.dumps(cases),
+                       capture_output=True, text=True, timeout=600)
+    if p.returncode != 0:
+        pytest.skip("triton interpreter unavailable: " + p.stderr[-300:])
+    res = json.loads(p.stdout.strip().splitlines()[-1])
+    for (s, ctr), got_t in zip(cases, res):
+        key = np.array([[s & 0xFFFFFFFF, s >> 32]] * len(ctr), np.uint32)
+        got = oracle.philox(np.array(ctr, np.uint32), key).ravel()
+        assert np.array_equal(got, np.array(got_t, np.uint32)), s
+    # the RHT sign mask is word 0 of Philox(counter (0,0,1,0), key seed), low 16 bits
+    for (s, _), got_t in zip(cases, res):
+        assert oracle.rht16_signs(s) == (got_t[4] & 0xFFFF)
+
+
+@pytest.mark.parametrize("seed", [0, 7, 2 ** 40 + 3])
+def test_rht16_matrix_is_scaled_sylvester_hadamard(seed):
+    H = scipy.linalg.hadamard(16).astype(np.float64)
+    mask = oracle.rht16_signs(seed)
+    D = np.diag([-1.0 if (mask >> i) & 1 else 1.0 for i in range(16)])
+    M = 0.25 * H @ D
+    cols = oracle.rht16(np.eye(16, dtype=np.float32), seed).reshape(16, 16)
+    # row i of the output is the transform of unit vector e_i = column i of M
+    assert np.array_equal(cols.T.astype(np.float64), M)
+    assert np.allclose(M @ M.T, np.eye(16))
+    x = np.random.default_rng(seed % 97).standard_normal((64, 16)).astype(np.float32)
+    y = oracle.rht16(x, seed).reshape(64, 16).astype(np.float64)
+    ref = x.astype(np.float64) @ M.T
+    assert np.allclose(y, ref, rtol=0, atol=1e-5 * np.abs(x).max())
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-5)
+
+
+# ------------------------------------------------------------------ 4/6 invariants
+def _bf16_bits(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _blocks_fp64(x_bits):
+    return (x_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _nibbles(codes):
+    lo = codes & 0xF
+    hi = codes >> 4
+    return np.stack([lo, hi], axis=-1).reshape(*codes.shape[:-1], codes.shape[-1] * 2)
+
+
+def _random_tensor(rng, rows, cols, kind="normal"):
+    if kind == "normal":
+        x = rng.standard_normal((rows, cols))
+    elif kind == "heavy":
+        x = rng.standard_t(3, (rows, cols))
+    elif kind == "outliers":
+        x = rng.standard_normal((rows, cols))
+        x.ravel()[::97] *= 40
+    else:
+        x = rng.uniform(-1, 1, (rows, cols)) * np.exp2(rng.integers(-20, 20, (rows, 1)))
+    return _bf16_bits(x.astype(np.float32)).reshape(1, rows, cols)
+
+
+@pytest.mark.parametrize("kind", ["normal", "heavy", "outliers", "scaled"])
+def test_46_choice_is_the_better_candidate_fp64(kind):
+    """Per block the kept candidate has fp64 squared error <= the other one.
+
+    The two candidates are rebuilt independently of the oracle: scale codes
+    from E4M3(RN(RN(a/S_t)/k)) and element codes from ml_dtypes' E2M1
+    conversion; errors are computed in fp64 from ml_dtypes' decoders.
+    """
+    rng = np.random.default_rng(10)
+    x = _random_tensor(rng, 64, 256, kind)
+    q = oracle.quantize(x)
+    w = _blocks_fp64(x[0]).reshape(-1, 16)
+    A = np.float32(np.abs(w).max())
+    S_t = np.float32(A / np.float32(1792.0))
+    assert q["tensor_scale"][0] == S_t
+    a = np.abs(w).max(axis=1).astype(np.float32)
+    r = (a / S_t).astype(np.float32)
+    s6 = _e4m3_sat_codes((r / np.float32(6.0)).astype(np.float32))
+    s4 = _e4m3_sat_codes((r / np.float32(4.0)).astype(np.float32))
+    scales = q["r_scales"].reshape(-1)
+    choice = np.unpackbits(q["r_choice"], bitorder="little")[: w.shape[0]]
+    assert np.array_equal(scales, np.where(choice == 1, s4, s6))
+
+    def cand_err(s):
+        e = (_e4m3_val(s).astype(np.float32) * S_t).astype(np.float32)
+        inv = np.where(e > 0, (np.float32(1) / np.where(e > 0, e, 1)).astype(np.float32), 0)
+        v = (np.abs(w).astype(np.float32) * inv[:, None]).astype(np.float32)
+        qq = _e2m1_val(_f4_codes(v)) * np.sign(w)
+        return ((w - qq * e[:, None].astype(np.float64)) ** 2).sum(axis=1)
+
+    e6, e4 = cand_err(s6), cand_err(s4)
+    chosen = np.where(choice == 1, e4, e6)
+    other = np.where(choice == 1, e6, e4)
+    tol = 1e-5 * np.maximum(chosen, other) + 1e-30
+    assert np.all(chosen <= other + tol)
+    # 4/6 is never worse than the 6-candidate, block by block
+    assert np.all(chosen <= e6 + tol)
+    # and the codes are the RNE codes of the kept candidate
+    codes = _nibbles(q["r_codes"][0]).reshape(-1, 16)
+    s = np.where(choice == 1, s4, s6)
+    e = (_e4m3_val(s).astype(np.float32) * S_t).astype(np.float32)
+    inv = np.where(e > 0, (np.float32(1) / np.where(e > 0, e, 1)).astype(np.float32), 0)
+    v = (np.abs(w).astype(np.float32) * inv[:, None]).astype(np.float32)
+    want = _f4_codes(v * np.where(np.signbit(w), -1, 1).astype(np.float32))
+    assert np.array_equal(codes, want)
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_NVFP4_46, oracle.FMT_NVFP4_6])
+def test_block_max_lands_on_4_or_6(fmt):
+    """With a normal scale the block max dequantizes to exactly 4*s*S_t or 6*s*S_t."""
+    rng = np.random.default_rng(11)
+    x = _random_tensor(rng, 128, 256, "heavy")
+    q = oracle.quantize(x, fmt=fmt)
+    w = _blocks_fp64(x[0]).reshape(-1, 16)
+    codes = _nibbles(q["r_codes"][0]).reshape(-1, 16) & 7
+    scales = q["r_scales"].reshape(-1)
+    choice = np.unpackbits(q["r_choice"], bitorder="little")[: w.shape[0]]
+    normal = _e4m3_val(scales) >= 2.0 ** -6
+    imax = np.abs(w).argmax(axis=1)
+    top = codes[np.arange(w.shape[0]), imax]
+    want = np.where(choice == 1, 6, 7)
+    assert normal.sum() > 0.9 * w.shape[0]
+    assert np.array_equal(top[normal], want[normal])
+    if fmt == oracle.FMT_NVFP4_6:
+        assert not choice.any()
+        assert q["tensor_scale"][0] == np.float32(np.float32(np.abs(w).max()) / np.float32(2688.0))
+
+
+def test_tensor_max_block_uses_full_e4m3_range():
+    """S_t = amax/(4*448): the block holding the tensor max gets s4 = 448, s6 = 288."""
+    rng = np.random.default_rng(12)
+    x = _random_tensor(rng, 32, 128, "outliers")
+    q = oracle.quantize(x)
+    w = _blocks_fp64(x[0]).reshape(-1, 16)
+    b = np.abs(w).max(axis=1).argmax()
+    choice = np.unpackbits(q["r_choice"], bitorder="little")[: w.shape[0]]
+    s = q["r_scales"].reshape(-1)[b]
+    assert _e4m3_val(s) == (448.0 if choice[b] else 288.0)
+    assert q["r_scales"].max() <= 0x7E
+
+
+def test_brute_force_every_scale_code_tiny_blocks():
+    """For every E4M3 code, RNE per element is error-optimal (3 live values,
+    all 8^3 magnitude codes enumerated), and the 4/6 pick is the better of
+    the two candidate codes; the gap to the best code over all 126 is recorded."""
+    rng = np.random.default_rng(13)
+    gaps = []
+    for trial in range(40):
+        w16 = np.zeros(16, np.float32)
+        pos = rng.choice(16, 3, replace=False)
+        w16[pos] = rng.standard_normal(3) * np.exp2(rng.integers(-4, 5))
+        # a second row with a larger max fixes S_t independently of this block
+        big = np.zeros(16, np.float32)
+        big[0] = 8 * np.abs(w16).max()
+        x = _bf16_bits(np.stack([w16, big])).reshape(1, 2, 16)
+        q = oracle.quantize(x)
+        w = _blocks_fp64(x[0, 0])
+        S_t = q["tensor_scale"][0]
+        codes = _nibbles(q["r_codes"][0, 0:1])[0]
+        s_kept = q["r_scales"][0, 0, 0]
+        live = np.nonzero(w)[0]
+
+        def err_with(s, mags):
+            e = np.float64(np.float32(_e4m3_val(s) * S_t))
+            qq = E2M1[mags] * np.sign(w[live])
+            return ((w[live] - qq * e) ** 2).sum()
+
+        best = min(err_with(s_kept, np.array(m))
+                   for m in itertools.product(range(8), repeat=live.size))
+        got = err_with(s_kept, codes[live] & 7)
+        assert got <= best * (1 + 1e-6) + 1e-300, (trial, got, best)
+        per_code = [err_with(c, _f4_codes(np.abs(w[live]) / np.float32(_e4m3_val(c) * S_t)) & 7)
+                    for c in range(1, 127) if np.float32(_e4m3_val(c) * S_t) > 0]
+        a = np.float32(np.abs(w).max())
+        r = np.float32(a / S_t)
+        s6 = _e4m3_sat_codes(np.float32(r / np.float32(6)))
+        s4 = _e4m3_sat_codes(np.float32(r / np.float32(4)))
+        assert s_kept in (s4, s6)
+        e6 = err_with(s6, _f4_codes(np.abs(w[live]) / np.float32(_e4m3_val(s6) * S_t)) & 7)
+        e4 = err_with(s4, _f4_codes(np.abs(w[live]) / np.float32(_e4m3_val(s4) * S_t)) & 7)
+        assert err_with(s_kept, codes[live] & 7) <= min(e4, e6) * (1 + 1e-5) + 1e-300
+        gaps.append(min(e4, e6) - min(per_code))
+    assert min(gaps) >= -1e-12  # no code beats the global optimum
+
+
+@pytest.mark.parametrize("second,want_scale,want_pick4,want_codes", [
+    # S_t = 1792/1792 = 1; block max 24: s6 = E4M3(24/6) = 4, s4 = E4M3(24/4) = 6.
+    (12.0, 4.0, 0, (7, 5)),   # 12/4 = 3 and 12/6 = 2 are both exact: tie -> 6
+    (9.0, 6.0, 1, (6, 3)),    # 9/4 = 2.25 -> 2 (err 1); 9/6 = 1.5 exact (err 0) -> 4
+    (15.0, 4.0, 0, (7, 6)),   # 15/4 = 3.75 -> 4 (err 1); 15/6 = 2.5 -> 2 (err 9) -> 6
+])
+def test_46_choice_closed_form(second, want_scale, want_pick4, want_codes):
+    """Hand-computed blocks pin the comparison direction and the tie rule."""
+    row0 = np.zeros(16, np.float32)
+    row0[0] = 1792.0  # tensor amax -> S_t = 1 exactly
+    row1 = np.zeros(16, np.float32)
+    row1[0], row1[1] = 24.0, second
+    x = _bf16_bits(np.stack([row0, row1])).reshape(1, 2, 16)
+    q = oracle.quantize(x)
+    assert q["tensor_scale"][0] == 1.0
+    assert _e4m3_val(q["r_scales"][0, 1, 0]) == want_scale
+    assert np.unpackbits(q["r_choice"], bitorder="little")[1] == want_pick4
+    codes = _nibbles(q["r_codes"][0, 1:2])[0]
+    assert tuple(codes[:2]) == want_codes and not codes[2:].any()
+
+
+def test_zero_tensor_and_zero_blocks():
+    x = np.zeros((1, 16, 32), np.uint16)
+    x[0, 3, 5] = 0x8000  # -0.0
+    q = oracle.quantize(x, colwise=True)
+    assert q["tensor_scale"][0] == 0
+    assert not q["r_scales"].any() and not q["r_choice"].any()
+    codes = _nibbles(q["r_codes"][0])
+    assert codes[3, 5] == 8 and (codes.sum() == 8)
+    # non-zero tensor with an all-zero block: scale 0, choice 6, signed zeros
+    y = _random_tensor(np.random.default_rng(14), 16, 64)
+    y[0, 2, 16:32] = 0
+    q = oracle.quantize(y)
+    assert q["r_scales"][0, 2, 1] == 0
+    assert not (np.unpackbits(q["r_choice"], bitorder="little")[2 * 4 + 1])
+
+
+def test_nonfinite_input_is_refused():
+    x = _random_tensor(np.random.default_rng(15), 16, 32)
+    x[0, 1, 1] = 0x7FC0
+    with pytest.raises(ValueError):
+        oracle.quantize(x)
+    x[0, 1, 1] = 0xFF80
+    with pytest.raises(ValueError):
+        oracle.amax(x)
+
+
+# ------------------------------------------------------------------ options
+def test_2d_single_row_tile_reduces_to_1x16():
+    """A 16x16 tile with one non-zero row quantizes exactly like that 1x16 row."""
+    rng = np.random.default_rng(16)
+    x = np.zeros((1, 16, 64), np.uint16)
+    x[0, 5] = _random_tensor(rng, 1, 64)[0, 0]
+    q2 = oracle.quantize(x, blk=oracle.BLK_16X16, colwise=True)
+    q1 = oracle.quantize(x)
+    assert np.array_equal(q2["r_codes"], q1["r_codes"])
+    assert np.array_equal(q2["r_scales"][0, 5], q1["r_scales"][0, 5])
+    c1 = np.unpackbits(q1["r_choice"], bitorder="little")[5 * 4: 5 * 4 + 4]
+    c2 = np.unpackbits(q2["r_choice"], bitorder="little")[:4]
+    assert np.array_equal(c1, c2)
+
+
+def test_2d_transposed_copy_is_exact_transpose():
+    rng = np.random.default_rng(17)
+    x = _random_tensor(rng, 48, 64, "heavy")
+    q = oracle.quantize(x, blk=oracle.BLK_16X16, colwise=True)
+    rc = _nibbles(q["r_codes"][0])
+    cc = _nibbles(q["c_codes"][0])
+    assert np.array_equal(rc.T, cc)
+    rs = q["r_scales"][0]           # [48, 4]
+    cs = q["c_scales"][0]           # [64, 3]
+    assert np.array_equal(rs[::16], cs[::16].T)
+    assert np.array_equal(rs, np.repeat(rs[::16], 16, axis=0))
+    assert np.array_equal(cs, np.repeat(cs[::16], 16, axis=0))
+    d_r = oracle.dequantize(q["r_codes"], q["r_scales"], q["tensor_scale"])
+    d_c = oracle.dequantize(q["c_codes"], q["c_scales"], q["tensor_scale"])
+    assert np.array_equal(d_r[0].T, d_c[0])
+
+
+def test_colwise_is_rowwise_of_transpose():
+    rng = np.random.default_rng(18)
+    x = _random_tensor(rng, 64, 48, "outliers")
+    q = oracle.quantize(x, colwise=True)
+    qt = oracle.quantize(np.ascontiguousarray(x[0].T)[None])
+    assert np.array_equal(q["c_codes"], qt["r_codes"])
+    assert np.array_equal(q["c_scales"], qt["r_scales"])
+    assert np.array_equal(q["c_choice"], qt["r_choice"])
+
+
+def test_rht_quantizes_the_transformed_blocks():
+    """RHT mode equals plain 4/6 of the (fp32) transformed blocks, whose amax it uses."""
+    rng = np.random.default_rng(19)
+    x = _random_tensor(rng, 16, 64, "outliers")
+    q = oracle.quantize(x, rht=True, seed=3)
+    y = oracle.rht16(_blocks_fp64(x).astype(np.float32).reshape(-1), 3)
+    A = np.float32(np.abs(y).max())
+    assert oracle.amax(x, rht=True, seed=3)[0] == A
+    assert q["tensor_scale"][0] == np.float32(A / np.float32(1792))
+    # every transformed block's max lands on 4 or 6 with a normal scale
+    codes = _nibbles(q["r_codes"][0]).reshape(-1, 16) & 7
+    yb = y.reshape(-1, 16)
+    choice = np.unpackbits(q["r_choice"], bitorder="little")[: yb.shape[0]]
+    top = codes[np.arange(yb.shape[0]), np.abs(yb).argmax(axis=1)]
+    normal = _e4m3_val(q["r_scales"].reshape(-1)) >= 2.0 ** -6
+    assert np.array_equal(top[normal], np.where(choice == 1, 6, 7)[normal])
+
+
+def test_stochastic_rounding_properties():
+    """SR keeps grid values, returns a neighbour of v, and is unbiased to 1/512."""
+    rng = np.random.default_rng(20)
+    v = rng.uniform(0, 6.5, 4096).astype(np.float32)
+    v[:8] = E2M1
+    lo_hi = []
+    for b in range(256):
+        m = oracle.e2m1_sr(v, np.full(v.size, b, np.uint8))
+        lo_hi.append(E2M1[m])
+    q = np.array(lo_hi)  # [256, n]
+    grid = np.append(E2M1, np.inf)
+    lo = E2M1[np.searchsorted(grid, v, side="right") - 1]
+    hi = np.where(v >= 6, 6.0, grid[np.minimum(np.searchsorted(grid, v, side="right"), 7)])
+    assert np.all((q == lo) | (q == hi))
+    assert np.all(q[:, :8] == E2M1)
+    mean = q.mean(axis=0)
+    vv = np.minimum(v.astype(np.float64), 6.0)
+    step = np.where(hi > lo, hi - lo, 1)
+    assert np.all(np.abs(mean - vv) <= step / 512 + 1e-12)
+
+
+def test_sr_tensor_unbiased_and_deterministic():
+    rng = np.random.default_rng(21)
+    x = _random_tensor(rng, 16, 64, "normal")
+    w = _blocks_fp64(x[0])
+    acc = np.zeros_like(w)
+    n = 200
+    q0 = None
+    for s in range(n):
+        q = oracle.quantize(x, rnd=oracle.RND_SR, seed=s)
+        if s == 0:
+            q0 = q
+        acc += _blocks_fp64(oracle.dequantize(q["r_codes"], q["r_scales"], q["tensor_scale"])[0])
+    again = oracle.quantize(x, rnd=oracle.RND_SR, seed=0)
+    assert all(np.array_equal(q0[k], again[k]) for k in q0)
+    mean = acc / n
+    # expected spread: each element has variance <= step^2/4 with step <= 2*e
+    e = _e4m3_val(q0["r_scales"][0]).repeat(16, axis=1) * q0["tensor_scale"][0]
+    assert np.all(np.abs(mean - w) <= 2 * e * (5 / np.sqrt(n) + 1 / 512) + 1e-3 * np.abs(w))
+    rel = np.abs(mean - w).mean() / np.abs(w).mean()
+    assert rel < 0.05
+
+
+def test_sr_shard_invariance_by_element_offset():
+    rng = np.random.default_rng(22)
+    x = _random_tensor(rng, 64, 32, "heavy")
+    full = oracle.quantize(x, rnd=oracle.RND_SR, seed=9, colwise=True)
+    A = oracle.amax(x)
+    parts = [oracle.quantize(x[:, r:r + 32], rnd=oracle.RND_SR, seed=9, colwise=True,
+                             elem_offset=r * 32, amax_in=A) for r in (0, 32)]
+    assert np.array_equal(np.concatenate([p["r_codes"] for p in parts], axis=1), full["r_codes"])
+    assert np.array_equal(np.concatenate([p["c_codes"] for p in parts], axis=2), full["c_codes"])
+
+
+def test_sr_bytes_follow_the_counter_layout():
+    """One Philox call per 16 consecutive elements; byte j of the 128-bit output."""
+    g = np.arange(0, 64, dtype=np.int64) + (5 << 36)
+    b = oracle.sr_bytes(11, g)
+    ctr = np.array([[(int(gi) >> 4) & 0xFFFFFFFF, int(gi) >> 36, 0, 0] for gi in g[::16]], np.uint32)
+    words = oracle.philox(ctr, np.array([[11, 0]] * len(ctr), np.uint32))
+    assert np.array_equal(b, words.view(np.uint8).ravel())
+
+
+# ------------------------------------------------------------------ dequantize / MX
+@pytest.mark.parametrize("fmt", [oracle.FMT_NVFP4_46, oracle.FMT_NVFP4_6])
+def test_dequantize_vs_independent_decoders(fmt):
+    rng = np.random.default_rng(23)
+    x = _random_tensor(rng, 32, 64, "heavy")
+    q = oracle.quantize(x, fmt=fmt)
+    y = oracle.dequantize(q["r_codes"], q["r_scales"], q["tensor_scale"])
+    codes = _nibbles(q["r_codes"][0])
+    qv = _e2m1_val(codes).astype(np.float32)
+    sv = np.repeat(_e4m3_val(q["r_scales"][0]).astype(np.float32), 16, axis=1)
+    prod = (qv * sv).astype(np.float32)
+    assert np.array_equal(prod.astype(np.float64), _e2m1_val(codes) * np.repeat(_e4m3_val(q["r_scales"][0]), 16, axis=1))
+    out = (prod * q["tensor_scale"][0]).astype(np.float32)
+    want = torch.from_numpy(out).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(y[0], want)
+
+
+def test_mxfp4_block_scale_and_codes():
+    rng = np.random.default_rng(24)
+    x = _random_tensor(rng, 32, 128, "scaled")
+    q = oracle.quantize(x, fmt=oracle.FMT_MXFP4, blk=oracle.BLK_1X32)
+    w = _blocks_fp64(x[0]).reshape(-1, 32)
+    a = np.abs(w).max(axis=1)
+    E = np.clip(np.floor(np.log2(np.where(a > 0, a, 1))) - 2, -127, 127)
+    E = np.where(a > 0, E, -127)
+    assert np.array_equal(q["r_scales"].reshape(-1).astype(np.int64), (E + 127).astype(np.int64))
+    v = (np.abs(w) * np.exp2(-E)[:, None]).astype(np.float32)
+    want = _f4_codes(v * np.where(np.signbit(w), -1, 1).astype(np.float32))
+    assert np.array_equal(_nibbles(q["r_codes"][0]).reshape(-1, 32), want)
+    top = (want & 7)[np.arange(w.shape[0]), np.abs(w).argmax(axis=1)]
+    assert np.all((top == 6) | (top == 7))
+    y = oracle.dequantize(q["r_codes"], q["r_scales"], None, fmt=oracle.FMT_MXFP4)
+    scale = np.repeat(q["r_scales"][0].view(md.float8_e8m0fnu).astype(np.float64), 32, axis=1)
+    ref = (_e2m1_val(_nibbles(q["r_codes"][0])) * scale).astype(np.float32)
+    assert np.array_equal(y[0], torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
+# ------------------------------------------------------------------ swizzle
+def test_swizzle_is_a_permutation_with_128x4_tiles():
+    rows, sfc = 256, 12
+    lin = np.arange(rows * sfc, dtype=np.int64)
+    offs = np.array([oracle.swizzle_offset(r, c, sfc) for r in range(rows) for c in range(sfc)])
+    assert len(set(offs.tolist())) == offs.size
+    assert offs.max() < oracle.swizzled_size(rows, sfc)
+    # 4 consecutive scales of one row are 4 consecutive bytes
+    o = offs.reshape(rows, sfc)
+    assert np.all(np.diff(o[:, :4], axis=1) == 1)
+    # rows r and r+32 of a 128-row tile are 4 bytes apart, r and r+1 16 bytes
+    assert np.all(o[32:64, 0] - o[0:32, 0] == 4)
+    assert np.all(o[1:32, 0] - o[0:31, 0] == 16)
+    # one 128x4 tile spans exactly 512 contiguous bytes
+    assert sorted(o[:128, :4].ravel().tolist()) == list(range(512))
+    del lin
