@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark: NVFP4 4/6 quantize GB/s and fraction of B200 HBM bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fos|reference]
+
+One step = one pass of the quantizer over the MoE expert workload
+(128 x 2880 x 2880 bf16, per-expert N(0, 0.02^2) times U(0.5, 2)): the
+per-expert amax pass and the 4/6 quantize to packed E2M1 codes + E4M3 scales +
+FP32 per-expert scales.  value = bytes / time with bytes = 2 (bf16 in) + 0.5
+(codes) + 1/16 (scales) per element, summed over ranks (weak scaling: every
+rank quantizes its own 128 experts).  Under torchrun one process per GPU;
+rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+BYTES_PER_ELEM = 2 + 0.5 + 1 / 16           # one orientation, NVFP4
+BYTES_PER_ELEM_DUAL = 2 + 2 * (0.5 + 1 / 16)  # two orientations from one read
+BYTES_PER_ELEM_MX = 2 + 0.5 + 1 / 32
+BYTES_PER_ELEM_DEQ = 0.5 + 1 / 16 + 2
+WORKLOAD = "moe_experts_128x2880x2880_nvfp4_46_1x16_rne"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", 6650.0)), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ dist
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index=0):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.cmd = ["nvidia-smi", "-i", ident, "--query-gpu=timestamp," + self.FIELDS,
+                        "--format=csv,noheader,nounits", "-lms", "50"]
+        except Exception:
+            self.cmd = None
+
+    def start(self):
+        if self.cmd is None:
+            return
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self, busy_from=0):
+        rows = []
+        for l in self.lines[busy_from:]:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for name, v in zip(names[1:], r[3][1:]):
+                if v.lower() in ("active", "1", "yes"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+# ------------------------------------------------------------------ timing
+def time_loop(fn, steps, warmup, world, stream):
+    """Device time of `steps` calls of fn (CUDA events on `stream`), ms total."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
+# ------------------------------------------------------------------ CPU baseline
+def cpu_baseline(x_cpu_bits, budget_s=12.0):
+    """Time the oracle (single thread) on whole experts until ~budget_s."""
+    import numpy as np
+    import oracle
+    done = 0
+    t0 = time.perf_counter()
+    per = x_cpu_bits.shape[1] * x_cpu_bits.shape[2]
+    while True:
+        e = done % x_cpu_bits.shape[0]
+        oracle.quantize(np.ascontiguousarray(x_cpu_bits[e:e + 1]))
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    elems = done * per
+    return {"value": round(elems * BYTES_PER_ELEM / dt / 1e9, 6), "unit": "GB/s",
+            "elems_per_s": round(elems / dt, 1), "cores": 1, "kind": "oracle",
+            "sample": "%d expert(s) of 2880x2880 (%d elements), amax pass + 4/6 quantize, "
+                      "single-threaded C oracle" % (done, elems)}
+
+
+# ------------------------------------------------------------------ main arms
+def run_fos(args, world, rank):
+    import mxfp4_block_scaled_fos_b200 as F
+    from mxfp4_block_scaled_fos_b200 import workloads
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    E, R, C = 128, 2880, 2880
+    x = workloads.moe_experts(E, R, C, device=dev, seed=rank)
+    elems = x.numel()
+    flags = 0
+    row = F.quantize(x)[0]  # allocate outputs once
+    ws = torch.empty(F.workspace_size(E, R, C), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    launches_per_step = 2  # amax pass + quantize
+
+    def step():
+        F.quantize(x, out_row=row, workspace=ws, status=status)
+
+    clk = ClockSampler(torch.cuda.current_device())
+    clk.start()
+    time.sleep(0.15)
+    t_ms = time_loop(step, args.steps, args.warmup, world, stream)
+    clk.stop()
+
+    # roofline of the dominant kernel: the quantize kernel alone (amax given)
+    amax = F.amax(x)
+
+    def q_only():
+        F.quantize(x, out_row=row, amax=amax, status=status)
+
+    k_steps = max(args.steps, 20)
+    tq_ms = time_loop(q_only, k_steps, 3, world, stream) / k_steps
+    ta_ms = time_loop(lambda: F.amax(x, out=amax), k_steps, 3, world, stream) / k_steps
+    peak, peak_kind = measured_peaks()
+    achieved = elems * BYTES_PER_ELEM / (tq_ms * 1e-3) / 1e9
+
+    extra = {}
+    if not args.no_modes:
+        extra = measure_modes(args, world, x, dev, stream, peak)
+
+    # end to end through the public API with host buffers
+    e2e = measure_e2e(args, world, x, row, ws, status, stream)
+    assert int(status.item()) == 0, "non-finite input reported"
+
+    ms_per_step = t_ms / args.steps
+    value = world * elems * BYTES_PER_ELEM / (ms_per_step * 1e-3) / 1e9
+    clocks = clk.summary()
+    out = {
+        "metric": "NVFP4 4/6 quantize GB/s and % of B200 HBM peak (bf16 in, FP4+E4M3 out)",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->e2m1+e4m3 (f32 arithmetic)", "data": "synthetic",
+        "frac_of_hbm": round(value / world / peak, 4),
+        "config": {"workload": WORKLOAD, "batch": E, "rows": R, "cols": C,
+                   "elements_per_gpu": elems, "bytes_per_elem": BYTES_PER_ELEM,
+                   "amax": "computed in-step (per expert)", "parallelism": "dp%d" % world,
+                   "l2": "input %.2f GB > 126 MB L2; no flush needed" % (2 * elems / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "k_q1x16 (4/6, RNE, amax supplied)",
+                     "kernel_ms": round(tq_ms, 4), "amax_kernel_ms": round(ta_ms, 4),
+                     "peak_source": "%s hbm_gbs (burst copy)" % peak_kind},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "clocks": clocks,
+        "modes": extra,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        xs = workloads.bits(x[:4])
+        out["cpu_baseline"] = cpu_baseline(xs, budget_s=args.cpu_seconds)
+    return out
+
+
+def measure_modes(args, world, x, dev, stream, peak):
+    """Other modes of the hot path at their workloads (context, not the headline)."""
+    import mxfp4_block_scaled_fos_b200 as F
+    from mxfp4_block_scaled_fos_b200 import workloads
+    res = {}
+    n = max(5, min(args.steps, 20))
+    elems = x.numel()
+
+    def rec(name, ms, bpe, n_elems, note=""):
+        gbs = n_elems * bpe / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "GB_s": round(gbs, 1), "frac": round(gbs / peak, 4),
+                     "bytes_per_elem": bpe, "elements": n_elems}
+        if note:
+            res[name]["note"] = note
+
+    try:
+        r6 = F.quantize(x, fmt="nvfp4_6")[0]
+        a6 = F.amax(x)
+        ms = time_loop(lambda: F.quantize(x, fmt="nvfp4_6", out_row=r6, amax=a6), n, 3, world, stream) / n
+        rec("moe_nvfp4_6only_quant", ms, BYTES_PER_ELEM, elems, "amax supplied")
+        rm = F.quantize(x, fmt="mxfp4")[0]
+        ms = time_loop(lambda: F.quantize(x, fmt="mxfp4", out_row=rm), n, 3, world, stream) / n
+        rec("moe_mxfp4_quant", ms, BYTES_PER_ELEM_MX, elems)
+        r46 = F.quantize(x)[0]
+        y = torch.empty_like(x)
+        ms = time_loop(lambda: F.dequantize(r46, out=y), n, 3, world, stream) / n
+        rec("moe_nvfp4_dequant", ms, BYTES_PER_ELEM_DEQ, elems)
+        ms = time_loop(lambda: F.dequantize(rm, out=y), n, 3, world, stream) / n
+        rec("moe_mxfp4_dequant", ms, 0.5 + 1 / 32 + 2, elems)
+        del y, r6, rm, r46
+    except Exception as e:  # report, do not hide
+        res["moe_error"] = repr(e)
+    # activation-like 8192x4096 with RHT16: rotate 4 copies (256 MiB > L2)
+    try:
+        xs = [workloads.activation_outliers(8192, 4096, device=dev, seed=s) for s in range(4)]
+        outs = [F.quantize(t, rht=True)[0] for t in xs]
+        am = [F.amax(t, rht=True) for t in xs]
+        it = [0]
+
+        def f():
+            i = it[0] % 4
+            it[0] += 1
+            F.quantize(xs[i], rht=True, out_row=outs[i], amax=am[i])
+        ms = time_loop(f, 4 * n, 4, world, stream) / (4 * n)
+        rec("activation_rht16_quant", ms, BYTES_PER_ELEM, xs[0].numel(), "amax supplied; 4 rotating copies")
+        del xs, outs
+    except Exception as e:
+        res["activation_error"] = repr(e)
+    return res
+
+
+def measure_e2e(args, world, x, row, ws, status, stream):
+    """Same metric through the public API with pinned host buffers: H2D of the
+    input, quantize (amax + 4/6), D2H of codes, scales and S_t, every step."""
+    import mxfp4_block_scaled_fos_b200 as F
+    h_in = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    h_in.copy_(x)
+    h_codes = torch.empty(row.codes.shape, dtype=torch.uint8, pin_memory=True)
+    h_scales = torch.empty(row.scales.shape, dtype=torch.uint8, pin_memory=True)
+    h_ts = torch.empty(row.tensor_scale.shape, dtype=torch.float32, pin_memory=True)
+    d_in = torch.empty_like(x)
+
+    def step():
+        d_in.copy_(h_in, non_blocking=True)
+        F.quantize(d_in, out_row=row, workspace=ws, status=status)
+        h_codes.copy_(row.codes, non_blocking=True)
+        h_scales.copy_(row.scales, non_blocking=True)
+        h_ts.copy_(row.tensor_scale, non_blocking=True)
+
+    n = max(3, min(args.steps, 5))
+    ms = time_loop(step, n, 1, world, stream) / n
+    elems = x.numel()
+    h2d = x.numel() * 2
+    d2h = row.codes.numel() + row.scales.numel() + 4 * row.tensor_scale.numel()
+    return {"value": round(world * elems * BYTES_PER_ELEM / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_reference(args, world, rank):
+    """The oracle (CPU, single thread) on a bounded sample per step."""
+    import numpy as np
+    import oracle
+    from mxfp4_block_scaled_fos_b200 import workloads
+    if rank != 0:
+        return None
+    x = workloads.moe_experts(1, 2880, 2880, device="cpu", seed=0)
+    xb = workloads.bits(x)
+    oracle.lib()
+    for _ in range(args.warmup):
+        oracle.quantize(xb)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.quantize(xb)
+    dt = time.perf_counter() - t0
+    elems = xb.size * args.steps
+    v = elems * BYTES_PER_ELEM / dt / 1e9
+    sample = "one 2880x2880 expert per step (amax pass + 4/6 quantize), single-threaded C oracle"
+    return {"impl": "reference", "metric": "NVFP4 4/6 quantize GB/s and % of B200 HBM peak "
+            "(bf16 in, FP4+E4M3 out)", "value": round(v, 6), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (CPU)", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": "1 of 128 experts per step"},
+            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "kind": "oracle", "cores": 1,
+                             "sample": sample},
+            "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fos", "reference"], default="fos")
+    ap.add_argument("--no-modes", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, _ = dist_setup(args.gpus)
+    from mxfp4_block_scaled_fos_b200 import build as fbuild
+    if rank == 0:
+        fbuild.build()
+    barrier(world)
+    out = run_fos(args, world, rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,10 @@
+"""Four Over Six (4/6) NVFP4 block quantization for B200 (sm_100a).
+
+The kernels live in libfos.so (C ABI in include/fos.h); ``fos`` is the thin
+ctypes binding that passes torch device buffers and the current stream to it.
+"""
+from .fos import (  # noqa: F401
+    FLAG_RHT16, FLAG_SCALE_SWIZZLED, STATUS_NONFINITE, STATUS_TIMEOUT, FosError, Options,
+    QTensor, amax, dequantize, lib, quantize, scales_size, status_string, version,
+    workspace_size,
+)

@@ -1,0 +1,287 @@
+// fos_api.cu -- the C ABI of libfos.so (argument checks, workspace layout,
+// launch sequence).  Declarations and semantics: include/fos.h.
+#include <string.h>
+
+#include "fos.h"
+#include "fos_internal.h"
+
+namespace fos {
+
+FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  f.s = s;
+  // m = floor(2^32 * (2^s - d) / d) + 1
+  f.m = (uint32_t)((((1ull << s) - d) << 32) / d + 1ull);
+  return f;
+}
+
+namespace {
+
+constexpr uint32_t kUnitsQuant = 256 * 4;   // block pairs per CTA (1x16 quantizer)
+constexpr uint32_t kUnitsAmax = 256 * 8;    // block pairs per CTA (amax pass)
+constexpr uint32_t kUnitsMx = 256 * 4;      // 1x32 blocks per CTA
+constexpr uint32_t kUnitsDeq = 256 * 4;     // blocks per CTA (dequantize)
+
+inline bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
+
+long long round_up(long long v, long long m) { return (v + m - 1) / m * m; }
+
+size_t ws_bytes(int64_t batch) { return (size_t)(8 * round_up(batch, 64) + 256); }
+
+// Validate one output descriptor for a tensor of R rows and C columns.
+fos_status check_out(const fos_qtensor* q, int64_t R, int64_t C, int64_t bs, bool nvfp4,
+                     uint32_t flags) {
+  if (!q->codes || !q->scales) return FOS_ERR_NULL;
+  if (nvfp4 && !q->tensor_scale) return FOS_ERR_NULL;
+  if (!aligned(q->codes, 16) || q->codes_ld % 8 != 0) return FOS_ERR_ALIGN;
+  if (q->codes_ld < C / 2) return FOS_ERR_SHAPE;
+  if (!(flags & FOS_FLAG_SCALE_SWIZZLED) && q->scales_ld < C / bs) return FOS_ERR_SHAPE;
+  if (q->choice_bits && !aligned(q->choice_bits, 8)) return FOS_ERR_ALIGN;
+  if (q->tensor_scale && !aligned(q->tensor_scale, 4)) return FOS_ERR_ALIGN;
+  (void)R;
+  return FOS_OK;
+}
+
+OutDesc make_out(const fos_qtensor* q, int64_t R, int64_t C, int64_t bs, uint32_t flags,
+                 int64_t nblk_per_batch) {
+  OutDesc o;
+  o.codes = q->codes;
+  o.codes_ld = q->codes_ld;
+  o.codes_bs = q->codes_ld * R;
+  o.scales = q->scales;
+  const int64_t sfc = C / bs;
+  if (flags & FOS_FLAG_SCALE_SWIZZLED) {
+    o.col_tiles = (sfc + 3) / 4;
+    o.scales_bs = round_up(R, 128) * o.col_tiles * 4;
+  } else {
+    o.scales_ld = q->scales_ld;
+    o.scales_bs = q->scales_ld * R;
+  }
+  o.choice = q->choice_bits;
+  o.choice_aligned = (nblk_per_batch % 64) == 0;
+  o.tensor_scale = q->tensor_scale;
+  return o;
+}
+
+size_t choice_bytes(int64_t nblocks) { return (size_t)(8 * ((nblocks + 63) / 64)); }
+
+}  // namespace
+}  // namespace fos
+
+using namespace fos;
+
+extern "C" {
+
+int32_t fos_version(void) { return FOS_VERSION; }
+
+const char* fos_status_string(int32_t s) {
+  switch (s) {
+    case FOS_OK: return "ok";
+    case FOS_ERR_NULL: return "a required pointer is NULL";
+    case FOS_ERR_ALIGN: return "a pointer or leading dimension is misaligned";
+    case FOS_ERR_SHAPE: return "shape not divisible by the block, or out of range";
+    case FOS_ERR_UNSUPPORTED: return "option combination not supported";
+    case FOS_ERR_WORKSPACE: return "workspace missing or too small";
+    case FOS_ERR_CUDA: return "CUDA launch or memset failed";
+    case FOS_ERR_ARG: return "invalid enum value, flag or offset";
+    default: return "unknown status";
+  }
+}
+
+size_t fos_workspace_size(int64_t batch, int64_t rows, int64_t cols, const fos_options* opt) {
+  (void)rows;
+  (void)cols;
+  (void)opt;
+  return ws_bytes(batch < 1 ? 1 : batch);
+}
+
+size_t fos_scales_size(int64_t R, int64_t sf_cols, uint32_t flags) {
+  if (R < 0 || sf_cols < 0) return 0;
+  if (flags & FOS_FLAG_SCALE_SWIZZLED)
+    return (size_t)(round_up(R, 128) * round_up(sf_cols, 4));
+  return (size_t)(R * sf_cols);
+}
+
+fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
+                        const fos_options* opt, const float* amax_in,
+                        const fos_qtensor* rowwise, const fos_qtensor* colwise,
+                        void* workspace, size_t workspace_bytes, uint32_t* status,
+                        void* stream) {
+  if (!opt || !x) return FOS_ERR_NULL;
+  if (!rowwise && !colwise) return FOS_ERR_NULL;
+  if (opt->fmt < 0 || opt->fmt > 2 || opt->blk < 0 || opt->blk > 2 || opt->rnd < 0 ||
+      opt->rnd > 1 || (opt->flags & ~(FOS_FLAG_RHT16 | FOS_FLAG_SCALE_SWIZZLED)))
+    return FOS_ERR_ARG;
+  if (batch < 0 || rows < 0 || cols < 0) return FOS_ERR_SHAPE;
+  const bool mx = opt->fmt == FOS_FMT_MXFP4;
+  const bool rht = (opt->flags & FOS_FLAG_RHT16) != 0;
+  const bool swz = (opt->flags & FOS_FLAG_SCALE_SWIZZLED) != 0;
+  const bool sr = opt->rnd == FOS_ROUND_SR;
+  if (mx != (opt->blk == FOS_BLOCK_1X32)) return FOS_ERR_UNSUPPORTED;
+  if (mx && (sr || rht || colwise)) return FOS_ERR_UNSUPPORTED;
+  if (rht && (opt->blk != FOS_BLOCK_1X16 || colwise)) return FOS_ERR_UNSUPPORTED;
+  if (opt->blk == FOS_BLOCK_16X16 && !rowwise) return FOS_ERR_UNSUPPORTED;
+  const int64_t bs = mx ? 32 : 16;
+  if (cols % bs) return FOS_ERR_SHAPE;
+  if ((colwise || opt->blk == FOS_BLOCK_16X16) && rows % 16) return FOS_ERR_SHAPE;
+  if (sr && (opt->elem_offset < 0 || opt->elem_offset % 16)) return FOS_ERR_ARG;
+  if (!aligned(x, 16) || ld % 8 != 0) return FOS_ERR_ALIGN;
+  if (ld < cols) return FOS_ERR_SHAPE;
+  if (batch > 65535) return FOS_ERR_SHAPE;
+  // per-batch block counts must stay below 2^31 (32-bit block indices)
+  if (rows > 0 && cols > 0 && (rows * (cols / 16)) >= (1ll << 31)) return FOS_ERR_SHAPE;
+  if (colwise && rows > 0 && cols > 0 && (cols * (rows / 16)) >= (1ll << 31)) return FOS_ERR_SHAPE;
+  fos_status e;
+  if (rowwise && (e = check_out(rowwise, rows, cols, bs, !mx, opt->flags)) != FOS_OK) return e;
+  if (colwise && (e = check_out(colwise, cols, rows, 16, !mx, opt->flags)) != FOS_OK) return e;
+  const bool need_ws = !mx && !amax_in;
+  if (need_ws) {
+    if (!workspace) return FOS_ERR_WORKSPACE;
+    if (workspace_bytes < ws_bytes(batch)) return FOS_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return FOS_ERR_ALIGN;
+  }
+  if (amax_in && !aligned(amax_in, 4)) return FOS_ERR_ALIGN;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  if (batch == 0) return FOS_OK;
+  if (rows == 0 || cols == 0) {  // empty entries: S_t = 0, nothing else to write
+    if (!mx) {
+      if (rowwise && cudaMemsetAsync(rowwise->tensor_scale, 0, 4 * batch, st) != cudaSuccess)
+        return FOS_ERR_CUDA;
+      if (colwise && cudaMemsetAsync(colwise->tensor_scale, 0, 4 * batch, st) != cudaSuccess)
+        return FOS_ERR_CUDA;
+    }
+    return FOS_OK;
+  }
+
+  QuantArgs a;
+  a.x = (const uint16_t*)x;
+  a.ld = ld;
+  a.x_bs = rows * ld;
+  a.rows = (int)rows;
+  a.cols = (int)cols;
+  a.nblk = (uint32_t)(rows * (cols / bs));
+  a.bpr = make_fastdiv((uint32_t)(cols / bs));
+  a.amax_in = amax_in;
+  a.status = status;
+  a.seed = opt->seed;
+  a.elem_offset = opt->elem_offset;
+  if (rowwise) {
+    const int64_t nb = opt->blk == FOS_BLOCK_16X16 ? (rows / 16) * (cols / 16) : rows * (cols / bs);
+    a.row = make_out(rowwise, rows, cols, bs, opt->flags, nb);
+  }
+  if (colwise) {
+    const int64_t nb = opt->blk == FOS_BLOCK_16X16 ? (rows / 16) * (cols / 16) : cols * (rows / 16);
+    a.col = make_out(colwise, cols, rows, 16, opt->flags, nb);
+  }
+
+  if (mx) {
+    a.units_per_cta = kUnitsMx;
+    return launch_mxfp4(a, (int)batch, swz, st) == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;
+  }
+
+  // per-tensor amax pass, unless the caller supplies the amaxes
+  uint32_t* amax_ws = (uint32_t*)workspace;
+  if (!amax_in) {
+    if (cudaMemsetAsync(amax_ws, 0, 4 * batch, st) != cudaSuccess) return FOS_ERR_CUDA;
+    a.units_per_cta = kUnitsAmax;
+    if (launch_amax(a, (int)batch, rht, amax_ws, st) != cudaSuccess) return FOS_ERR_CUDA;
+  }
+  a.amax_ws = amax_ws;
+
+  // choice bitmaps that are shared between CTAs are built with atomics
+  const int64_t nb_row = opt->blk == FOS_BLOCK_16X16 ? batch * (rows / 16) * (cols / 16)
+                                                     : batch * rows * (cols / 16);
+  const int64_t nb_col = opt->blk == FOS_BLOCK_16X16 ? nb_row : batch * cols * (rows / 16);
+  if (rowwise && rowwise->choice_bits && !a.row.choice_aligned)
+    if (cudaMemsetAsync(rowwise->choice_bits, 0, choice_bytes(nb_row), st) != cudaSuccess)
+      return FOS_ERR_CUDA;
+  if (colwise && colwise->choice_bits && !a.col.choice_aligned)
+    if (cudaMemsetAsync(colwise->choice_bits, 0, choice_bytes(nb_col), st) != cudaSuccess)
+      return FOS_ERR_CUDA;
+
+  cudaError_t ce;
+  a.units_per_cta = kUnitsQuant;
+  if (opt->blk == FOS_BLOCK_16X16) {
+    ce = launch_q16x16(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr, st);
+  } else if (colwise) {
+    ce = launch_q1x16_dual(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, st);
+  } else {
+    ce = launch_q1x16_rowwise(a, (int)batch, opt->fmt, sr, rht, swz, st);
+  }
+  if (ce == cudaErrorNotSupported) return FOS_ERR_UNSUPPORTED;
+  return ce == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;
+}
+
+fos_status fos_amax(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
+                    const fos_options* opt, float* amax_out, uint32_t* status, void* stream) {
+  if (!x || !opt || !amax_out) return FOS_ERR_NULL;
+  if (opt->flags & ~(FOS_FLAG_RHT16 | FOS_FLAG_SCALE_SWIZZLED)) return FOS_ERR_ARG;
+  if (batch < 0 || rows < 0 || cols < 0 || batch > 65535) return FOS_ERR_SHAPE;
+  if (cols % 16) return FOS_ERR_SHAPE;
+  if (!aligned(x, 16) || ld % 8 != 0 || !aligned(amax_out, 4)) return FOS_ERR_ALIGN;
+  if (ld < cols) return FOS_ERR_SHAPE;
+  if (rows > 0 && cols > 0 && rows * (cols / 16) >= (1ll << 31)) return FOS_ERR_SHAPE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (batch == 0) return FOS_OK;
+  if (cudaMemsetAsync(amax_out, 0, 4 * batch, st) != cudaSuccess) return FOS_ERR_CUDA;
+  if (rows == 0 || cols == 0) return FOS_OK;
+  QuantArgs a;
+  a.x = (const uint16_t*)x;
+  a.ld = ld;
+  a.x_bs = rows * ld;
+  a.rows = (int)rows;
+  a.cols = (int)cols;
+  a.nblk = (uint32_t)(rows * (cols / 16));
+  a.bpr = make_fastdiv((uint32_t)(cols / 16));
+  a.status = status;
+  a.seed = opt->seed;
+  a.units_per_cta = kUnitsAmax;
+  return launch_amax(a, (int)batch, (opt->flags & FOS_FLAG_RHT16) != 0, (uint32_t*)amax_out, st) ==
+                 cudaSuccess
+             ? FOS_OK
+             : FOS_ERR_CUDA;
+}
+
+fos_status fos_dequantize(const fos_qtensor* q, int32_t fmt, int64_t batch, int64_t rows,
+                          int64_t cols, uint32_t flags, void* y, int64_t ldy, void* stream) {
+  if (!q || !y) return FOS_ERR_NULL;
+  if (fmt < 0 || fmt > 2 || (flags & ~(FOS_FLAG_RHT16 | FOS_FLAG_SCALE_SWIZZLED))) return FOS_ERR_ARG;
+  if (batch < 0 || rows < 0 || cols < 0 || batch > 65535) return FOS_ERR_SHAPE;
+  const bool mx = fmt == FOS_FMT_MXFP4;
+  const int64_t bs = mx ? 32 : 16;
+  if (cols % bs) return FOS_ERR_SHAPE;
+  fos_status e = check_out(q, rows, cols, bs, !mx, flags);
+  if (e != FOS_OK) return e;
+  if (!aligned(y, 16) || ldy % 8 != 0) return FOS_ERR_ALIGN;
+  if (ldy < cols) return FOS_ERR_SHAPE;
+  if (rows > 0 && cols > 0 && rows * (cols / bs) >= (1ll << 31)) return FOS_ERR_SHAPE;
+  if (batch == 0 || rows == 0 || cols == 0) return FOS_OK;
+  const OutDesc o = make_out(q, rows, cols, bs, flags, rows * (cols / bs));
+  DequantArgs a;
+  a.codes = o.codes;
+  a.codes_ld = o.codes_ld;
+  a.codes_bs = o.codes_bs;
+  a.scales = o.scales;
+  a.scales_ld = o.scales_ld;
+  a.scales_bs = o.scales_bs;
+  a.col_tiles = o.col_tiles;
+  a.tensor_scale = q->tensor_scale;
+  a.y = (uint16_t*)y;
+  a.ldy = ldy;
+  a.y_bs = ldy * rows;
+  a.rows = (int)rows;
+  a.cols = (int)cols;
+  a.nblk = (uint32_t)(rows * (cols / bs));
+  a.bpr = make_fastdiv((uint32_t)(cols / bs));
+  a.units_per_cta = kUnitsDeq;
+  return launch_dequant(a, (int)batch, mx, (flags & FOS_FLAG_SCALE_SWIZZLED) != 0,
+                        (cudaStream_t)stream) == cudaSuccess
+             ? FOS_OK
+             : FOS_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,163 @@
+// fos_device.cuh -- device-side building blocks of the sm_100a quantizers.
+//
+// Element and scale codecs use the Blackwell conversion instructions
+// (cvt.rn.satfinite.e2m1x2.f32, cvt.rn.satfinite.e4m3x2.f32 and the
+// e2m1x2 -> f16x2 decode); binary32 arithmetic that the quantizer's
+// definition fixes uses explicitly rounded intrinsics (no contraction), and
+// element pairs are processed with the packed f32x2 FMA/MUL/ADD of sm_100.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fos {
+
+constexpr float kE4M3Max = 448.0f;
+constexpr float kFltMax = 3.402823466e38f;
+
+// ---------------------------------------------------------------- bf16
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ---------------------------------------------------------------- f32x2
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// a - b with one rounding: b * (-1) is exact, the sum rounds once.
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
+// ---------------------------------------------------------------- E2M1
+// Eight binary32 values -> eight E2M1 nibbles (RNE, saturating at +-6);
+// element 2k goes to the low nibble of byte k.
+__device__ __forceinline__ uint32_t e2m1x8(float e0, float e1, float e2, float e3, float e4,
+                                           float e5, float e6, float e7) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(e0), "f"(e1), "f"(e2), "f"(e3), "f"(e4), "f"(e5), "f"(e6), "f"(e7));
+  return out;
+}
+
+// Eight E2M1 nibbles -> four f16x2 words (h[k] holds elements 2k, 2k+1),
+// exact.
+__device__ __forceinline__ void e2m1x8_to_h2(uint32_t codes, uint32_t h[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(codes));
+}
+
+__device__ __forceinline__ float h_lo(uint32_t h) {
+  return __half2float(__ushort_as_half((unsigned short)(h & 0xffffu)));
+}
+__device__ __forceinline__ float h_hi(uint32_t h) {
+  return __half2float(__ushort_as_half((unsigned short)(h >> 16)));
+}
+
+// ---------------------------------------------------------------- E4M3
+// Two binary32 values -> (E4M3(hi) << 8) | E4M3(lo), RNE, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3x2(float hi, float lo) {
+  unsigned short out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+  return out;
+}
+
+// E4M3 code (0..255) -> binary32, exact (via the f16x2 decode).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  uint32_t h;
+  unsigned short c = (unsigned short)(code & 0xffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c));
+  return h_lo(h);
+}
+
+// ---------------------------------------------------------------- Philox
+// Philox4x32-10 as published by Salmon et al. (SC'11).
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    if (i) {
+      k.x += 0x9E3779B9u;
+      k.y += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint2 seed_key(unsigned long long seed) {
+  return make_uint2((uint32_t)(seed & 0xffffffffull), (uint32_t)(seed >> 32));
+}
+
+// Philox output for the 16 consecutive source elements starting at g0
+// (g0 % 16 == 0): byte j belongs to element g0 + j.
+__device__ __forceinline__ uint4 sr_bytes16(unsigned long long seed, long long g0) {
+  const unsigned long long u = (unsigned long long)g0;
+  return philox4x32_10(make_uint4((uint32_t)((u >> 4) & 0xffffffffull), (uint32_t)(u >> 36), 0u, 0u),
+                       seed_key(seed));
+}
+
+__device__ __forceinline__ uint32_t byte_of(uint4 r, int j) {
+  const uint32_t w = (j < 4) ? r.x : (j < 8) ? r.y : (j < 12) ? r.z : r.w;
+  return (w >> (8 * (j & 3))) & 0xffu;
+}
+
+// 16-bit mask of the random Hadamard signs: bit i set -> element i negated.
+__device__ __forceinline__ uint32_t rht_sign_mask(unsigned long long seed) {
+  return philox4x32_10(make_uint4(0u, 0u, 1u, 0u), seed_key(seed)).x & 0xffffu;
+}
+
+// ---------------------------------------------------------------- SR
+// Stochastic rounding of v >= 0 on the E2M1 magnitude grid: with lo <= v < hi
+// the neighbouring grid values, round up iff 2*byte+1 < 512*(v-lo)/(hi-lo).
+// Every step below is exact in binary32.
+__device__ __forceinline__ float sr_e2m1_mag(float v, uint32_t byte) {
+  if (v >= 6.0f) return 6.0f;
+  const float step = v < 2.0f ? 0.5f : (v < 4.0f ? 1.0f : 2.0f);
+  const float inv_step = v < 2.0f ? 2.0f : (v < 4.0f ? 1.0f : 0.5f);
+  const float t = __fmul_rn(v, inv_step);
+  const float fl = floorf(t);
+  const float p = __fsub_rn(t, fl);
+  const float lo = __fmul_rn(fl, step);
+  const float thr = (float)(2u * byte + 1u);
+  return (thr < __fmul_rn(512.0f, p)) ? __fadd_rn(lo, step) : lo;
+}
+
+// ---------------------------------------------------------------- indexing
+// Division by a runtime constant d >= 1 for numerators n < 2^31:
+// n / d = (umulhi(n, m) + n) >> s.
+struct FastDiv {
+  uint32_t d, m, s;
+};
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.m) + n) >> f.s;
+}
+
+// Byte offset of scale (r, c) of an [R][sf_cols] matrix in the tensor-core
+// block-scaled layout: 512-byte tiles of 128 rows x 4 scales, tiles ordered
+// row-major; inside a tile (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.
+__device__ __forceinline__ long long swz_offset(long long r, long long c, long long col_tiles) {
+  return ((r >> 7) * col_tiles + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+// Non-negative binary32 values compare like their bit patterns.
+__device__ __forceinline__ void atomic_max_pos(uint32_t* addr, float v) {
+  atomicMax(addr, __float_as_uint(v));
+}
+
+}  // namespace fos

@@ -1,0 +1,71 @@
+// fos_internal.h -- launch descriptors shared by the C ABI layer and the
+// kernel files of libfos.so (host side; no device code).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fos_device.cuh"
+
+namespace fos {
+
+// One output orientation as the kernels see it.
+struct OutDesc {
+  uint8_t* codes = nullptr;
+  long long codes_ld = 0;   // bytes per row
+  long long codes_bs = 0;   // bytes per batch entry
+  uint8_t* scales = nullptr;
+  long long scales_ld = 0;  // bytes per row (linear layout)
+  long long scales_bs = 0;  // bytes per batch entry
+  long long col_tiles = 0;  // swizzled layout: ceil(sf_cols / 4)
+  uint8_t* choice = nullptr;
+  int choice_aligned = 0;   // blocks per batch entry % 64 == 0
+  float* tensor_scale = nullptr;
+};
+
+struct QuantArgs {
+  const uint16_t* x = nullptr;
+  long long ld = 0;          // elements per row of x
+  long long x_bs = 0;        // elements per batch entry of x
+  int rows = 0, cols = 0;
+  uint32_t nblk = 0;         // 1x16 (or 1x32) blocks per batch entry
+  FastDiv bpr{};             // blocks per row
+  uint32_t units_per_cta = 0;
+  const float* amax_in = nullptr;   // nullable
+  const uint32_t* amax_ws = nullptr;
+  uint32_t* status = nullptr;       // nullable
+  unsigned long long seed = 0;
+  long long elem_offset = 0;
+  OutDesc row, col;
+};
+
+FastDiv make_fastdiv(uint32_t d);
+
+// Kernel launchers (return the launch's cudaError_t).
+cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_ws,
+                        cudaStream_t st);
+cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
+                                 bool swz, cudaStream_t st);
+cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
+                              bool want_row, cudaStream_t st);
+cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
+                          bool want_row, bool want_col, cudaStream_t st);
+cudaError_t launch_mxfp4(const QuantArgs& a, int batch, bool swz, cudaStream_t st);
+
+struct DequantArgs {
+  const uint8_t* codes = nullptr;
+  long long codes_ld = 0, codes_bs = 0;
+  const uint8_t* scales = nullptr;
+  long long scales_ld = 0, scales_bs = 0, col_tiles = 0;
+  const float* tensor_scale = nullptr;
+  uint16_t* y = nullptr;
+  long long ldy = 0, y_bs = 0;
+  int rows = 0, cols = 0;
+  uint32_t nblk = 0;   // blocks per batch entry
+  FastDiv bpr{};
+  uint32_t units_per_cta = 0;
+};
+
+cudaError_t launch_dequant(const DequantArgs& a, int batch, bool mx, bool swz, cudaStream_t st);
+
+}  // namespace fos

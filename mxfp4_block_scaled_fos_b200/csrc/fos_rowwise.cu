@@ -1,0 +1,523 @@
+// fos_rowwise.cu -- per-tensor amax pass and the rowwise 1x16 NVFP4 (4/6 and
+// 6-only) quantizer for sm_100a.
+//
+// Method: Hugging Face transformers doc "Four Over Six", introduction (each
+// NVFP4 block scaled so its max maps to 4 or to 6, the lower-error candidate
+// kept); Ultralytics glossary "FP4", "Como funciona FP4" (NVFP4: 16 values,
+// E4M3 block scale, FP32 per-tensor scale) and introduction (E2M1 values).
+// Options from the "Four Over Six" usage section: random Hadamard transform
+// and stochastic rounding.
+//
+// Design: each thread owns two neighbouring 16-element blocks and carries
+// them as 16 packed pairs (element i of block A, element i of block B), so
+// every binary32 step of both blocks -- scaling, the error fma, squaring and
+// the whole pairwise error tree -- is one sm_100 f32x2 instruction.  Loads are
+// 4 x 128-bit per thread with the next pair prefetched; codes leave as 8-byte
+// stores (a warp writes 512 contiguous bytes), the 4/6 choice bits as one
+// 64-bit word per warp.
+#include "fos.h"
+#include "fos_internal.h"
+
+namespace fos {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// Sign flips of the random Hadamard transform for the two bf16 halves of
+// word k (elements 2k and 2k+1).
+__device__ __forceinline__ uint32_t rht_word_mask(uint32_t mask16, int k) {
+  return (((mask16 >> (2 * k)) & 1u) << 15) | (((mask16 >> (2 * k + 1)) & 1u) << 31);
+}
+
+// In-place 16-point fast Walsh-Hadamard transform of the packed pairs with
+// butterflies (a, b) -> (a + b, a - b) at strides 1, 2, 4, 8, then * 0.25.
+__device__ __forceinline__ void fwht16_pairs(float2 (&P)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h *= 2) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2 * h) {
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float2 a = P[j], b = P[j + h];
+        P[j] = add2(a, b);
+        P[j + h] = sub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) P[i] = mul2(P[i], make_float2(0.25f, 0.25f));
+}
+
+// Unpack two blocks of 8 bf16x2 words into 16 packed (A_i, B_i) pairs.
+__device__ __forceinline__ void unpack_pairs(const uint4 (&wa)[2], const uint4 (&wb)[2],
+                                             float2 (&P)[16]) {
+  const uint32_t A[8] = {wa[0].x, wa[0].y, wa[0].z, wa[0].w, wa[1].x, wa[1].y, wa[1].z, wa[1].w};
+  const uint32_t B[8] = {wb[0].x, wb[0].y, wb[0].z, wb[0].w, wb[1].x, wb[1].y, wb[1].z, wb[1].w};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    P[2 * k] = make_float2(bf_lo(A[k]), bf_lo(B[k]));
+    P[2 * k + 1] = make_float2(bf_hi(A[k]), bf_hi(B[k]));
+  }
+}
+
+// max |x| of 8 bf16x2 words, as binary32 bits (NaN/Inf give >= 0x7f800000).
+__device__ __forceinline__ uint32_t amax_bits_bf16(const uint4 (&w)[2]) {
+  uint32_t m = __vmaxu2(w[0].x & 0x7fff7fffu, w[0].y & 0x7fff7fffu);
+  m = __vmaxu2(m, w[0].z & 0x7fff7fffu);
+  m = __vmaxu2(m, w[0].w & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].x & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].y & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].z & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].w & 0x7fff7fffu);
+  return max(m & 0xffffu, m >> 16) << 16;
+}
+
+// max |P[i].x| and max |P[i].y| as binary32 bits.
+__device__ __forceinline__ void amax_bits_pairs(const float2 (&P)[16], uint32_t& ma, uint32_t& mb) {
+  ma = 0;
+  mb = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    ma = max(ma, __float_as_uint(P[i].x) & 0x7fffffffu);
+    mb = max(mb, __float_as_uint(P[i].y) & 0x7fffffffu);
+  }
+}
+
+// Candidate scale codes of a block with amax a: (s6, s4) as E4M3 bytes.
+template <bool F46>
+__device__ __forceinline__ void cand_scales(float a, float St, uint32_t& s6, uint32_t& s4) {
+  const float r = (St == 0.0f) ? 0.0f : __fdiv_rn(a, St);
+  // r >= 0 for valid input; the 0x7f mask keeps a caller-supplied negative
+  // amax from indexing past the 128-entry scale table
+  if (F46) {
+    const uint32_t both = e4m3x2(__fdiv_rn(r, 6.0f), __fmul_rn(r, 0.25f));
+    s6 = (both >> 8) & 0x7fu;
+    s4 = both & 0x7fu;
+  } else {
+    s6 = e4m3x2(0.0f, __fdiv_rn(r, 6.0f)) & 0x7fu;
+    s4 = 0;
+  }
+}
+
+struct Cand {
+  uint32_t ca[2], cb[2];  // codes of block A and block B (2 words each)
+  float2 err;             // (error A, error B)
+};
+
+// Round both blocks with one candidate scale per block and, when WANT_ERR,
+// form the binary32 squared error d = fma(-q, e, w), t = d*d, pairwise tree.
+template <bool WANT_ERR>
+__device__ __forceinline__ Cand candidate(const float2 (&P)[16], float2 inv, float2 nege) {
+  Cand c;
+  float2 v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = mul2(P[i], inv);
+  c.ca[0] = e2m1x8(v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x);
+  c.ca[1] = e2m1x8(v[8].x, v[9].x, v[10].x, v[11].x, v[12].x, v[13].x, v[14].x, v[15].x);
+  c.cb[0] = e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y);
+  c.cb[1] = e2m1x8(v[8].y, v[9].y, v[10].y, v[11].y, v[12].y, v[13].y, v[14].y, v[15].y);
+  c.err = make_float2(0.0f, 0.0f);
+  if (WANT_ERR) {
+    uint32_t ha[8], hb[8];
+    e2m1x8_to_h2(c.ca[0], ha);
+    e2m1x8_to_h2(c.ca[1], ha + 4);
+    e2m1x8_to_h2(c.cb[0], hb);
+    e2m1x8_to_h2(c.cb[1], hb + 4);
+    float2 l1[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 q0 = make_float2(h_lo(ha[k]), h_lo(hb[k]));
+      const float2 q1 = make_float2(h_hi(ha[k]), h_hi(hb[k]));
+      const float2 d0 = fma2(q0, nege, P[2 * k]);
+      const float2 d1 = fma2(q1, nege, P[2 * k + 1]);
+      l1[k] = add2(mul2(d0, d0), mul2(d1, d1));
+    }
+    const float2 l2a = add2(l1[0], l1[1]), l2b = add2(l1[2], l1[3]);
+    const float2 l2c = add2(l1[4], l1[5]), l2d = add2(l1[6], l1[7]);
+    c.err = add2(add2(l2a, l2b), add2(l2c, l2d));
+  }
+  return c;
+}
+
+// Stochastic rounding of the kept candidate of one block (A: which = 0,
+// B: which = 1) with 16 Philox bytes.
+__device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float inv, uint4 rnd,
+                                         uint32_t (&out)[2]) {
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float w = which ? P[i].y : P[i].x;
+    const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
+    q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
+  }
+  out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+  out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+}
+
+// Bit i of a -> bit 2i, bit i of b -> bit 2i+1.
+__device__ __forceinline__ unsigned long long interleave_bits(uint32_t a, uint32_t b) {
+  auto spread = [](unsigned long long x) {
+    x = (x | (x << 16)) & 0x0000FFFF0000FFFFull;
+    x = (x | (x << 8)) & 0x00FF00FF00FF00FFull;
+    x = (x | (x << 4)) & 0x0F0F0F0F0F0F0F0Full;
+    x = (x | (x << 2)) & 0x3333333333333333ull;
+    x = (x | (x << 1)) & 0x5555555555555555ull;
+    return x;
+  };
+  return spread(a) | (spread(b) << 1);
+}
+
+__device__ __forceinline__ void store_choice64(const OutDesc& o, unsigned long long gbit,
+                                               unsigned long long word) {
+  unsigned long long* base = reinterpret_cast<unsigned long long*>(o.choice);
+  if (o.choice_aligned) {
+    base[gbit >> 6] = word;
+  } else if (word) {
+    // only words that receive a set bit are touched, so nothing past the
+    // last block's word is accessed
+    const int sh = (int)(gbit & 63);
+    const unsigned long long lo = word << sh, hi = sh ? (word >> (64 - sh)) : 0ull;
+    if (lo) atomicOr(base + (gbit >> 6), lo);
+    if (hi) atomicOr(base + (gbit >> 6) + 1, hi);
+  }
+}
+
+__device__ __forceinline__ float tensor_scale_of(const QuantArgs& a, int b, bool f46) {
+  const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_ws[b]);
+  return __fdiv_rn(A, f46 ? 1792.0f : 2688.0f);
+}
+
+// (E(c), 1/E(c)) for every non-negative E4M3 code c, E(c) = float(c) * S_t;
+// a zero E gives a zero inverse, an overflowing inverse is clamped to
+// FLT_MAX.
+__device__ __forceinline__ void build_scale_table(float2* tab, float St) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float E = __fmul_rn(e4m3_to_f32((uint32_t)c), St);
+    const float inv = (E == 0.0f) ? 0.0f : fminf(__frcp_rn(E), kFltMax);
+    tab[c] = make_float2(E, inv);
+  }
+}
+
+__device__ __forceinline__ void load_block(const QuantArgs& a, int b, uint32_t j, uint4 (&w)[2]) {
+  const uint32_t row = fdiv(j, a.bpr);
+  const uint32_t cb = j - row * a.bpr.d;
+  const uint4* p = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs +
+                                                 (long long)row * a.ld + (long long)cb * 16);
+  w[0] = __ldg(p);
+  w[1] = __ldg(p + 1);
+}
+
+template <bool SWZ>
+__device__ __forceinline__ void store_block(const OutDesc& o, int b, uint32_t j, const FastDiv& bpr,
+                                            const uint32_t (&codes)[2], uint32_t scale) {
+  const uint32_t row = fdiv(j, bpr);
+  const uint32_t cb = j - row * bpr.d;
+  uint2* cp = reinterpret_cast<uint2*>(o.codes + (long long)b * o.codes_bs +
+                                       (long long)row * o.codes_ld + (long long)cb * 8);
+  *cp = make_uint2(codes[0], codes[1]);
+  long long so;
+  if (SWZ) so = (long long)b * o.scales_bs + swz_offset(row, cb, o.col_tiles);
+  else     so = (long long)b * o.scales_bs + (long long)row * o.scales_ld + cb;
+  o.scales[so] = (uint8_t)scale;
+}
+
+// --------------------------------------------------------------------------
+// K0: per-batch-entry amax of |x| (or of the RHT of x).
+// grid (chunks, batch); each thread handles pairs of blocks.
+template <bool RHT>
+__global__ void __launch_bounds__(kThreads) k_amax(const QuantArgs a, uint32_t* amax_ws) {
+  const int b = blockIdx.y;
+  const uint32_t nunit = (a.nblk + 1) / 2;
+  const uint32_t u0 = blockIdx.x * a.units_per_cta;
+  const uint32_t u1 = min(u0 + a.units_per_cta, nunit);
+  uint32_t mask16 = 0;
+  if (RHT) mask16 = rht_sign_mask(a.seed);
+  uint32_t m = 0;
+  for (uint32_t u = u0 + threadIdx.x; u < u1; u += kThreads) {
+    const uint32_t j0 = 2 * u;
+    const bool has1 = j0 + 1 < a.nblk;
+    uint4 wa[2], wb[2];
+    load_block(a, b, j0, wa);
+    if (has1) load_block(a, b, j0 + 1, wb);
+    else      { wb[0] = wa[0]; wb[1] = wa[1]; }
+    if (RHT) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t xa = rht_word_mask(mask16, k), xb = rht_word_mask(mask16, k + 4);
+        (&wa[0].x)[k] ^= xa; (&wb[0].x)[k] ^= xa;
+        (&wa[1].x)[k] ^= xb; (&wb[1].x)[k] ^= xb;
+      }
+      float2 P[16];
+      unpack_pairs(wa, wb, P);
+      fwht16_pairs(P);
+      uint32_t ma, mb;
+      amax_bits_pairs(P, ma, mb);
+      m = max(m, max(ma, mb));
+    } else {
+      m = max(m, max(amax_bits_bf16(wa), amax_bits_bf16(wb)));
+    }
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  __shared__ uint32_t s_m[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) s_m[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t v = threadIdx.x < kThreads / 32 ? s_m[threadIdx.x] : 0u;
+    v = __reduce_max_sync(0xffffffffu, v);
+    if (threadIdx.x == 0) {
+      if (v >= 0x7f800000u) {
+        if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+      } else {
+        atomicMax(amax_ws + b, v);
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// K1: rowwise 1x16 NVFP4 quantizer.  grid (chunks, batch).
+template <bool F46, bool SR, bool RHT, bool SWZ>
+__global__ void __launch_bounds__(kThreads, 2) k_q1x16(const QuantArgs a) {
+  __shared__ float2 s_tab[128];
+  const int b = blockIdx.y;
+  const float St = tensor_scale_of(a, b, F46);
+  build_scale_table(s_tab, St);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[b] = St;
+  uint32_t mask16 = 0;
+  if (RHT) mask16 = rht_sign_mask(a.seed);
+  __syncthreads();
+
+  const uint32_t nunit = (a.nblk + 1) / 2;
+  const uint32_t u0 = blockIdx.x * a.units_per_cta;
+  const uint32_t u1 = min(u0 + a.units_per_cta, nunit);
+  const int lane = threadIdx.x & 31;
+  uint32_t bad = 0;
+
+  // software pipeline: the next pair is loaded before this one is processed
+  uint32_t u = u0 + threadIdx.x;
+  uint4 na[2], nb[2];
+  if (u < u1) {
+    load_block(a, b, 2 * u, na);
+    if (2 * u + 1 < a.nblk) load_block(a, b, 2 * u + 1, nb);
+  }
+  for (uint32_t ubase = u0; ubase < u1; ubase += kThreads) {
+    const bool valid = u < u1;
+    const uint32_t j0 = 2 * u;
+    const bool has1 = valid && (j0 + 1 < a.nblk);
+    uint4 wa[2] = {na[0], na[1]}, wb[2] = {nb[0], nb[1]};
+    if (!has1) { wb[0] = wa[0]; wb[1] = wa[1]; }
+    const uint32_t un = u + kThreads;
+    if (un < u1) {
+      load_block(a, b, 2 * un, na);
+      if (2 * un + 1 < a.nblk) load_block(a, b, 2 * un + 1, nb);
+    }
+
+    uint32_t pick_a = 0, pick_b = 0;
+    if (valid) {
+      if (RHT) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t xa = rht_word_mask(mask16, k), xb = rht_word_mask(mask16, k + 4);
+          (&wa[0].x)[k] ^= xa; (&wb[0].x)[k] ^= xa;
+          (&wa[1].x)[k] ^= xb; (&wb[1].x)[k] ^= xb;
+        }
+      }
+      float2 P[16];
+      unpack_pairs(wa, wb, P);
+      uint32_t ma, mb;
+      if (RHT) {
+        fwht16_pairs(P);
+        amax_bits_pairs(P, ma, mb);
+      } else {
+        ma = amax_bits_bf16(wa);
+        mb = amax_bits_bf16(wb);
+      }
+      bad |= (max(ma, mb) >= 0x7f800000u);
+      uint32_t s6a, s4a, s6b, s4b;
+      cand_scales<F46>(__uint_as_float(ma), St, s6a, s4a);
+      cand_scales<F46>(__uint_as_float(mb), St, s6b, s4b);
+      const float2 t6a = s_tab[s6a], t6b = s_tab[s6b];
+      const Cand c6 = candidate<F46>(P, make_float2(t6a.y, t6b.y), make_float2(-t6a.x, -t6b.x));
+      uint32_t ca[2] = {c6.ca[0], c6.ca[1]}, cbk[2] = {c6.cb[0], c6.cb[1]};
+      uint32_t sa = s6a, sb = s6b;
+      float inva = t6a.y, invb = t6b.y;
+      if (F46) {
+        const float2 t4a = s_tab[s4a], t4b = s_tab[s4b];
+        const Cand c4 = candidate<true>(P, make_float2(t4a.y, t4b.y), make_float2(-t4a.x, -t4b.x));
+        pick_a = c4.err.x < c6.err.x;
+        pick_b = c4.err.y < c6.err.y;
+        if (pick_a) { ca[0] = c4.ca[0]; ca[1] = c4.ca[1]; sa = s4a; inva = t4a.y; }
+        if (pick_b) { cbk[0] = c4.cb[0]; cbk[1] = c4.cb[1]; sb = s4b; invb = t4b.y; }
+      }
+      if (SR) {
+        const long long g0 = a.elem_offset + (long long)b * a.rows * a.cols;
+        const uint32_t rowa = fdiv(j0, a.bpr), cba = j0 - rowa * a.bpr.d;
+        sr_block(P, 0, inva, sr_bytes16(a.seed, g0 + (long long)rowa * a.cols + cba * 16), ca);
+        if (has1) {
+          const uint32_t rowb = fdiv(j0 + 1, a.bpr), cbb = j0 + 1 - rowb * a.bpr.d;
+          sr_block(P, 1, invb, sr_bytes16(a.seed, g0 + (long long)rowb * a.cols + cbb * 16), cbk);
+        }
+      }
+      store_block<SWZ>(a.row, b, j0, a.bpr, ca, sa);
+      if (has1) store_block<SWZ>(a.row, b, j0 + 1, a.bpr, cbk, sb);
+    }
+    if (F46 && a.row.choice) {
+      const uint32_t ba = __ballot_sync(0xffffffffu, pick_a);
+      const uint32_t bb = __ballot_sync(0xffffffffu, pick_b);
+      const uint32_t uw = ubase + (threadIdx.x & ~31u);
+      if (lane == 0 && uw < u1) {
+        store_choice64(a.row, (unsigned long long)b * a.nblk + 2ull * uw, interleave_bits(ba, bb));
+      }
+    }
+    u = un;
+  }
+  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// --------------------------------------------------------------------------
+// MXFP4 1x32: E = floor(log2 amax) - 2 from the exponent bits, clamped to
+// [-127, 127]; codes = E2M1_rne(w * 2^-E) (the scaling is exact).
+template <bool SWZ>
+__global__ void __launch_bounds__(kThreads) k_mxfp4(const QuantArgs a) {
+  const int b = blockIdx.y;
+  const uint32_t u0 = blockIdx.x * a.units_per_cta;
+  const uint32_t u1 = min(u0 + a.units_per_cta, a.nblk);
+  uint32_t bad = 0;
+  for (uint32_t j = u0 + threadIdx.x; j < u1; j += kThreads) {
+    const uint32_t row = fdiv(j, a.bpr);
+    const uint32_t cb = j - row * a.bpr.d;
+    const uint4* p = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs +
+                                                   (long long)row * a.ld + (long long)cb * 32);
+    uint4 w4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w4[k] = __ldg(p + k);
+    const uint4 lo[2] = {w4[0], w4[1]}, hi[2] = {w4[2], w4[3]};
+    const uint32_t am = max(amax_bits_bf16(lo), amax_bits_bf16(hi));
+    bad |= am >= 0x7f800000u;
+    const uint32_t ex = max(am >> 23, 2u);          // biased exponent, >= 2
+    const uint32_t scale = ex - 2u;                 // E + 127 with E = ex - 129
+    const float inv = __uint_as_float((256u - ex) << 23);  // 2^-E
+    const float2 inv2 = make_float2(inv, inv);
+    const uint32_t* w = &w4[0].x;
+    float v[32];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float2 r = mul2(make_float2(bf_lo(w[k]), bf_hi(w[k])), inv2);
+      v[2 * k] = r.x;
+      v[2 * k + 1] = r.y;
+    }
+    uint4 c;
+    c.x = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+    c.y = e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+    c.z = e2m1x8(v[16], v[17], v[18], v[19], v[20], v[21], v[22], v[23]);
+    c.w = e2m1x8(v[24], v[25], v[26], v[27], v[28], v[29], v[30], v[31]);
+    uint2* cp = reinterpret_cast<uint2*>(a.row.codes + (long long)b * a.row.codes_bs +
+                                         (long long)row * a.row.codes_ld + (long long)cb * 16);
+    cp[0] = make_uint2(c.x, c.y);
+    cp[1] = make_uint2(c.z, c.w);
+    long long so;
+    if (SWZ) so = (long long)b * a.row.scales_bs + swz_offset(row, cb, a.row.col_tiles);
+    else     so = (long long)b * a.row.scales_bs + (long long)row * a.row.scales_ld + cb;
+    a.row.scales[so] = (uint8_t)scale;
+  }
+  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// --------------------------------------------------------------------------
+// Dequantize: NVFP4 y = bf16_rne((q * float(s)) * S_t); MXFP4 y = q * 2^(s-127).
+template <bool MX, bool SWZ>
+__global__ void __launch_bounds__(kThreads) k_dequant(const DequantArgs a) {
+  const int b = blockIdx.y;
+  const uint32_t u0 = blockIdx.x * a.units_per_cta;
+  const uint32_t u1 = min(u0 + a.units_per_cta, a.nblk);
+  const float St = MX ? 1.0f : a.tensor_scale[b];
+  constexpr int BS = MX ? 32 : 16;
+  for (uint32_t j = u0 + threadIdx.x; j < u1; j += kThreads) {
+    const uint32_t row = fdiv(j, a.bpr);
+    const uint32_t cb = j - row * a.bpr.d;
+    long long so;
+    if (SWZ) so = (long long)b * a.scales_bs + swz_offset(row, cb, a.col_tiles);
+    else     so = (long long)b * a.scales_bs + (long long)row * a.scales_ld + cb;
+    const uint32_t sc = a.scales[so];
+    const float s = MX ? __uint_as_float(sc == 0 ? 0x00400000u : (sc << 23)) : e4m3_to_f32(sc);
+    const uint2* cp = reinterpret_cast<const uint2*>(a.codes + (long long)b * a.codes_bs +
+                                                     (long long)row * a.codes_ld +
+                                                     (long long)cb * (BS / 2));
+    uint4* yp = reinterpret_cast<uint4*>(a.y + (long long)b * a.y_bs + (long long)row * a.ldy +
+                                         (long long)cb * BS);
+#pragma unroll
+    for (int part = 0; part < BS / 16; ++part) {
+      const uint2 cw = cp[part];
+      uint32_t h[8];
+      e2m1x8_to_h2(cw.x, h);
+      e2m1x8_to_h2(cw.y, h + 4);
+      uint32_t o[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float2 q = make_float2(h_lo(h[k]), h_hi(h[k]));
+        q = mul2(q, make_float2(s, s));
+        if (!MX) q = mul2(q, make_float2(St, St));
+        const __nv_bfloat162 r = __floats2bfloat162_rn(q.x, q.y);
+        o[k] = *reinterpret_cast<const uint32_t*>(&r);
+      }
+      yp[2 * part] = make_uint4(o[0], o[1], o[2], o[3]);
+      yp[2 * part + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+static dim3 grid_for(uint32_t units, uint32_t per_cta, int batch) {
+  return dim3((units + per_cta - 1) / per_cta, (unsigned)batch, 1);
+}
+
+cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_ws,
+                        cudaStream_t st) {
+  const uint32_t nunit = (a.nblk + 1) / 2;
+  const dim3 g = grid_for(nunit, a.units_per_cta, batch);
+  if (rht) k_amax<true><<<g, kThreads, 0, st>>>(a, amax_ws);
+  else     k_amax<false><<<g, kThreads, 0, st>>>(a, amax_ws);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
+                                 bool swz, cudaStream_t st) {
+  const uint32_t nunit = (a.nblk + 1) / 2;
+  const dim3 g = grid_for(nunit, a.units_per_cta, batch);
+  const bool f46 = fmt == 0;
+#define FOS_L(F, S, R, W) k_q1x16<F, S, R, W><<<g, kThreads, 0, st>>>(a)
+#define FOS_W(F, S, R) do { if (swz) FOS_L(F, S, R, true); else FOS_L(F, S, R, false); } while (0)
+#define FOS_R(F, S) do { if (rht) FOS_W(F, S, true); else FOS_W(F, S, false); } while (0)
+#define FOS_S(F) do { if (sr) FOS_R(F, true); else FOS_R(F, false); } while (0)
+  if (f46) FOS_S(true);
+  else     FOS_S(false);
+#undef FOS_S
+#undef FOS_R
+#undef FOS_W
+#undef FOS_L
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp4(const QuantArgs& a, int batch, bool swz, cudaStream_t st) {
+  const dim3 g = grid_for(a.nblk, a.units_per_cta, batch);
+  if (swz) k_mxfp4<true><<<g, kThreads, 0, st>>>(a);
+  else     k_mxfp4<false><<<g, kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const DequantArgs& a, int batch, bool mx, bool swz, cudaStream_t st) {
+  const dim3 g = grid_for(a.nblk, a.units_per_cta, batch);
+  if (mx) {
+    if (swz) k_dequant<true, true><<<g, kThreads, 0, st>>>(a);
+    else     k_dequant<true, false><<<g, kThreads, 0, st>>>(a);
+  } else {
+    if (swz) k_dequant<false, true><<<g, kThreads, 0, st>>>(a);
+    else     k_dequant<false, false><<<g, kThreads, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fos

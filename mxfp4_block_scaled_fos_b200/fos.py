@@ -1,0 +1,235 @@
+"""ctypes binding of libfos.so (include/fos.h) with torch tensors as buffers.
+
+This module only marshals arguments: it checks dtypes and devices, allocates
+output tensors with torch when the caller does not pass them, and hands raw
+device pointers and the current CUDA stream to the C ABI.  Every step of the
+quantizer runs in the library's sm_100a kernels; there is no CPU fallback.
+If libfos.so is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfos.so")
+
+FMT = {"nvfp4_46": 0, "nvfp4_6": 1, "mxfp4": 2}
+BLK = {"1x16": 0, "16x16": 1, "1x32": 2}
+RND = {"rne": 0, "sr": 1}
+FLAG_RHT16 = 0x1
+FLAG_SCALE_SWIZZLED = 0x2
+STATUS_NONFINITE = 0x1
+STATUS_TIMEOUT = 0x2
+
+ERRORS = {
+    1: "FOS_ERR_NULL", 2: "FOS_ERR_ALIGN", 3: "FOS_ERR_SHAPE", 4: "FOS_ERR_UNSUPPORTED",
+    5: "FOS_ERR_WORKSPACE", 6: "FOS_ERR_CUDA", 7: "FOS_ERR_ARG",
+}
+
+# every symbol include/fos.h declares
+EXPORTS = ("fos_quantize", "fos_amax", "fos_dequantize", "fos_workspace_size",
+           "fos_scales_size", "fos_status_string", "fos_version")
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("blk", ctypes.c_int32), ("rnd", ctypes.c_int32),
+                ("flags", ctypes.c_uint32), ("seed", ctypes.c_uint64),
+                ("elem_offset", ctypes.c_int64)]
+
+
+class QTensorC(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("choice_bits", ctypes.c_void_p),
+                ("codes_ld", ctypes.c_int64), ("scales_ld", ctypes.c_int64)]
+
+
+class FosError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (%d)" % (what, ERRORS.get(code, "?"), code))
+        self.code = code
+
+
+_lib = None
+
+
+def lib(path: str = LIB_PATH):
+    """Load libfos.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("libfos.so is missing at %s; build it with "
+                           "`python -m mxfp4_block_scaled_fos_b200.build`" % path)
+    L = ctypes.CDLL(path)
+    P, i64, i32, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32
+    L.fos_quantize.restype = i32
+    L.fos_quantize.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P,
+                               ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), P,
+                               ctypes.c_size_t, P, P]
+    L.fos_amax.restype = i32
+    L.fos_amax.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P, P, P]
+    L.fos_dequantize.restype = i32
+    L.fos_dequantize.argtypes = [ctypes.POINTER(QTensorC), i32, i64, i64, i64, u32, P, i64, P]
+    L.fos_workspace_size.restype = ctypes.c_size_t
+    L.fos_workspace_size.argtypes = [i64, i64, i64, ctypes.POINTER(Options)]
+    L.fos_scales_size.restype = ctypes.c_size_t
+    L.fos_scales_size.argtypes = [i64, i64, u32]
+    L.fos_status_string.restype = ctypes.c_char_p
+    L.fos_status_string.argtypes = [i32]
+    L.fos_version.restype = i32
+    L.fos_version.argtypes = []
+    _lib = L
+    return L
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass
+class QTensor:
+    """One quantized orientation of a [batch, R, C] tensor (device tensors)."""
+    codes: torch.Tensor              # uint8 [batch, R, C/2]
+    scales: torch.Tensor             # uint8 [batch, R, C/bs] or flat swizzled
+    tensor_scale: Optional[torch.Tensor]  # float32 [batch] (NVFP4)
+    choice: Optional[torch.Tensor]   # uint8 bitmap, 8 * ceil(nblocks/64) bytes
+    batch: int
+    rows: int
+    cols: int
+    fmt: str
+    block: str
+    flags: int
+
+    def c_struct(self) -> QTensorC:
+        sld = 0 if self.flags & FLAG_SCALE_SWIZZLED else self.scales.shape[-1]
+        return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(),
+                        self.tensor_scale.data_ptr() if self.tensor_scale is not None else None,
+                        self.choice.data_ptr() if self.choice is not None else None,
+                        self.codes.shape[-1], sld)
+
+
+def scales_size(R: int, sf_cols: int, flags: int = 0) -> int:
+    return int(lib().fos_scales_size(R, sf_cols, flags))
+
+
+def workspace_size(batch: int, rows: int, cols: int, opts: Optional[Options] = None) -> int:
+    return int(lib().fos_workspace_size(batch, rows, cols, ctypes.byref(opts or Options())))
+
+
+def _alloc_qtensor(batch, R, C, fmt, block, flags, device, with_choice, nblocks) -> QTensor:
+    bs = 32 if fmt == "mxfp4" else 16
+    codes = torch.empty(batch, R, C // 2, dtype=torch.uint8, device=device)
+    if flags & FLAG_SCALE_SWIZZLED:
+        scales = torch.empty(batch, scales_size(R, C // bs, flags), dtype=torch.uint8, device=device)
+    else:
+        scales = torch.empty(batch, R, C // bs, dtype=torch.uint8, device=device)
+    ts = torch.empty(batch, dtype=torch.float32, device=device) if fmt != "mxfp4" else None
+    ch = None
+    if with_choice and fmt == "nvfp4_46":
+        ch = torch.empty(8 * ((nblocks + 63) // 64), dtype=torch.uint8, device=device)
+    return QTensor(codes, scales, ts, ch, batch, R, C, fmt, block, flags)
+
+
+def _as3d(x: torch.Tensor) -> torch.Tensor:
+    if x.dim() == 2:
+        x = x.unsqueeze(0)
+    if x.dim() != 3:
+        raise ValueError("expected [rows, cols] or [batch, rows, cols]")
+    return x
+
+
+def quantize(x: torch.Tensor, fmt: str = "nvfp4_46", block: Optional[str] = None,
+             rounding: str = "rne", rht: bool = False, swizzle: bool = False, seed: int = 0,
+             elem_offset: int = 0, rowwise: bool = True, colwise: bool = False,
+             choice: bool = True, amax: Optional[torch.Tensor] = None,
+             status: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+             out_row: Optional[QTensor] = None, out_col: Optional[QTensor] = None,
+             stream=None):
+    """Quantize a CUDA bf16 tensor [batch, rows, cols] (or [rows, cols]).
+
+    Returns (rowwise QTensor or None, colwise QTensor or None).
+    """
+    x = _as3d(x)
+    if x.dtype != torch.bfloat16 or not x.is_cuda:
+        raise TypeError("x must be a CUDA bfloat16 tensor")
+    if x.stride(-1) != 1 or x.stride(0) != x.shape[1] * x.stride(1):
+        raise ValueError("x rows must be contiguous with batch stride rows * ld")
+    batch, rows, cols = x.shape
+    ld = x.stride(1)
+    block = block or ("1x32" if fmt == "mxfp4" else "1x16")
+    flags = (FLAG_RHT16 if rht else 0) | (FLAG_SCALE_SWIZZLED if swizzle else 0)
+    opts = Options(FMT[fmt], BLK[block], RND[rounding], flags, seed, elem_offset)
+    bs = 32 if fmt == "mxfp4" else 16
+    if block == "16x16":
+        nb_row = nb_col = batch * (rows // 16) * (cols // 16)
+    else:
+        nb_row = batch * rows * (cols // bs)
+        nb_col = batch * cols * (rows // 16)
+    if rowwise and out_row is None:
+        out_row = _alloc_qtensor(batch, rows, cols, fmt, block, flags, x.device, choice, nb_row)
+    if colwise and out_col is None:
+        out_col = _alloc_qtensor(batch, cols, rows, fmt, block, flags, x.device, choice, nb_col)
+    if not rowwise:
+        out_row = None
+    if not colwise:
+        out_col = None
+    wsz = workspace_size(batch, rows, cols, opts)
+    if workspace is None and amax is None and fmt != "mxfp4":
+        workspace = torch.empty(wsz, dtype=torch.uint8, device=x.device)
+    r = out_row.c_struct() if out_row is not None else None
+    c = out_col.c_struct() if out_col is not None else None
+    st = lib().fos_quantize(
+        ctypes.c_void_p(x.data_ptr()), batch, rows, cols, ld, ctypes.byref(opts), _ptr(amax),
+        ctypes.byref(r) if r is not None else None, ctypes.byref(c) if c is not None else None,
+        _ptr(workspace), workspace.numel() if workspace is not None else 0, _ptr(status),
+        _stream(stream))
+    if st != 0:
+        raise FosError(st, "fos_quantize")
+    return out_row, out_col
+
+
+def amax(x: torch.Tensor, rht: bool = False, seed: int = 0, out: Optional[torch.Tensor] = None,
+         status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per-batch-entry amax of |x| (of the 16-wide RHT of x when rht)."""
+    x = _as3d(x)
+    batch, rows, cols = x.shape
+    if out is None:
+        out = torch.empty(batch, dtype=torch.float32, device=x.device)
+    opts = Options(0, 0, 0, FLAG_RHT16 if rht else 0, seed, 0)
+    st = lib().fos_amax(ctypes.c_void_p(x.data_ptr()), batch, rows, cols, x.stride(1),
+                        ctypes.byref(opts), _ptr(out), _ptr(status), _stream(stream))
+    if st != 0:
+        raise FosError(st, "fos_amax")
+    return out
+
+
+def dequantize(q: QTensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Codes + scales (+ S_t) of one orientation back to bf16 [batch, R, C]."""
+    if out is None:
+        out = torch.empty(q.batch, q.rows, q.cols, dtype=torch.bfloat16, device=q.codes.device)
+    qc = q.c_struct()
+    st = lib().fos_dequantize(ctypes.byref(qc), FMT[q.fmt], q.batch, q.rows, q.cols,
+                              q.flags & FLAG_SCALE_SWIZZLED, ctypes.c_void_p(out.data_ptr()),
+                              out.stride(-2), _stream(stream))
+    if st != 0:
+        raise FosError(st, "fos_dequantize")
+    return out
+
+
+def status_string(code: int) -> str:
+    return lib().fos_status_string(code).decode()
+
+
+def version() -> int:
+    return int(lib().fos_version())

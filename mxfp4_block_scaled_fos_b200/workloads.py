@@ -1,7 +1,7 @@
 """Seeded synthetic inputs for the quantizer (no quantization arithmetic here).
 
-This module only draws random tensors.  Both the CUDA path's tests and the
-CPU oracle receive the same bf16 bytes from it, so it holds none of the
+This module only draws random tensors.  The CUDA path and the CPU reference
+used by the tests receive the same bf16 bytes from it, so it holds none of the
 method's arithmetic.  Every recipe follows the workload descriptions of the
 Four Over Six / FP4 pages' use cases (activations with outlier channels,
 weights, gradients, MoE expert weights) and the worked example of the

@@ -1,0 +1,94 @@
+"""Host-side checks of libfos.so (no GPU needed): the library loads, exports
+every symbol include/fos.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mxfp4_block_scaled_fos_b200 as F
+from mxfp4_block_scaled_fos_b200 import build as fbuild
+from mxfp4_block_scaled_fos_b200.fos import EXPORTS, Options, QTensorC
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return F.lib()
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"^\s*(?:fos_status|size_t|int32_t|const char\*)\s+(fos_\w+)\s*\(",
+                                    txt, re.M))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert declared, "no declarations found"
+    assert declared <= set(EXPORTS) | {"fos_quantize_static"}
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_version_and_strings(L):
+    assert F.version() == 1
+    assert F.status_string(0) == "ok"
+    for code in range(1, 8):
+        assert F.status_string(code) != "unknown status"
+
+
+def test_sizes(L):
+    assert F.scales_size(2880, 180, 0) == 2880 * 180
+    assert F.scales_size(2880, 180, F.FLAG_SCALE_SWIZZLED) == 2944 * 180
+    assert F.scales_size(1, 1, F.FLAG_SCALE_SWIZZLED) == 512
+    assert F.workspace_size(128, 2880, 2880) >= 4 * 128
+
+
+def _call(L, x=16, batch=1, rows=16, cols=32, ld=32, opts=None, row=True, col=False,
+          ws=16, wsb=1 << 16, amax=None):
+    o = opts or Options(0, 0, 0, 0, 0, 0)
+    q = QTensorC(64, 128, 256, None, cols // 2, cols // 16)
+    qc = QTensorC(64, 128, 256, None, rows // 2, rows // 16)
+    return L.fos_quantize(ctypes.c_void_p(x), batch, rows, cols, ld, ctypes.byref(o),
+                          ctypes.c_void_p(amax) if amax else None,
+                          ctypes.byref(q) if row else None, ctypes.byref(qc) if col else None,
+                          ctypes.c_void_p(ws) if ws else None, wsb, None, None)
+
+
+def test_argument_errors(L):
+    assert _call(L, x=0) == 1                                   # NULL input
+    assert _call(L, row=False, col=False) == 1                  # no output
+    assert _call(L, opts=Options(3, 0, 0, 0, 0, 0)) == 7        # bad format
+    assert _call(L, opts=Options(0, 0, 0, 0x80, 0, 0)) == 7     # unknown flag
+    assert _call(L, x=8) == 2                                   # misaligned x
+    assert _call(L, ld=36) == 2                                 # ld % 8
+    assert _call(L, cols=24, ld=24) == 3                        # cols % 16
+    assert _call(L, rows=15, col=True) == 3                     # colwise needs rows % 16
+    assert _call(L, opts=Options(2, 0, 0, 0, 0, 0)) == 4        # MXFP4 with 1x16
+    assert _call(L, opts=Options(0, 2, 0, 0, 0, 0)) == 4        # NVFP4 with 1x32
+    assert _call(L, opts=Options(2, 2, 1, 0, 0, 0)) == 4        # MXFP4 + SR
+    assert _call(L, opts=Options(0, 0, 0, 1, 0, 0), col=True) == 4  # RHT + colwise
+    assert _call(L, opts=Options(0, 1, 0, 1, 0, 0)) == 4        # RHT + 16x16
+    assert _call(L, opts=Options(0, 0, 1, 0, 0, 8)) == 7        # SR offset % 16
+    assert _call(L, ws=0) == 5                                  # no workspace
+    assert _call(L, wsb=16) == 5                                # workspace too small
+    assert _call(L, ld=16) == 3                                 # ld < cols
+    assert _call(L, rows=-1) == 3
+
+
+def test_library_has_no_oracle_dependency():
+    """The product library must not link or name the CPU oracle."""
+    src_dir = os.path.join(ROOT, "mxfp4_block_scaled_fos_b200")
+    for dirpath, _, files in os.walk(src_dir):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, fn)).read()
+                assert "oracle" not in txt.lower(), fn
