@@ -123,7 +123,6 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
   if (mx != (opt->blk == FOS_BLOCK_1X32)) return FOS_ERR_UNSUPPORTED;
   if (mx && (sr || rht || colwise)) return FOS_ERR_UNSUPPORTED;
   if (rht && (opt->blk != FOS_BLOCK_1X16 || colwise)) return FOS_ERR_UNSUPPORTED;
-  if (opt->blk == FOS_BLOCK_16X16 && !rowwise) return FOS_ERR_UNSUPPORTED;
   const int64_t bs = mx ? 32 : 16;
   if (cols % bs) return FOS_ERR_SHAPE;
   if ((colwise || opt->blk == FOS_BLOCK_16X16) && rows % 16) return FOS_ERR_SHAPE;
@@ -192,7 +191,16 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
   }
   a.amax_ws = amax_ws;
 
-  // choice bitmaps that are shared between CTAs are built with atomics
+  // Which choice-bit words a CTA owns outright depends on the kernel's tiling;
+  // bitmaps whose words are shared between CTAs are built with atomics on a
+  // zeroed buffer.
+  if (opt->blk == FOS_BLOCK_16X16) {
+    a.row.choice_aligned = a.col.choice_aligned = (cols / 16) % 8 == 0;
+  } else if (colwise) {
+    a.row.choice_aligned = (cols / 16) % 8 == 0;
+    a.col.choice_aligned = (rows / 16) % 32 == 0;
+  }
+
   const int64_t nb_row = opt->blk == FOS_BLOCK_16X16 ? batch * (rows / 16) * (cols / 16)
                                                      : batch * rows * (cols / 16);
   const int64_t nb_col = opt->blk == FOS_BLOCK_16X16 ? nb_row : batch * cols * (rows / 16);

@@ -1,0 +1,203 @@
+// fos_core.cuh -- the per-block 4/6 arithmetic shared by every NVFP4
+// quantizer kernel (rowwise, colwise, 16x16).
+//
+// Method: Hugging Face transformers doc "Four Over Six", introduction: both
+// candidates (block max mapped to 6 and to 4) are rounded to E2M1 and the
+// one with the lower block squared error is kept, ties keeping 6.
+// Ultralytics glossary "FP4", "Como funciona FP4": NVFP4 blocks of 16 values
+// with an E4M3 block scale and an FP32 per-tensor scale.
+//
+// Two blocks A and B are carried as 16 packed pairs (A_i, B_i) so that all
+// binary32 steps of both blocks run as sm_100 f32x2 instructions.  For a
+// 1x16 block the 16 elements are consecutive along its row (rowwise) or its
+// column (colwise); for a 16x16 tile, A and B are two of its rows.
+#pragma once
+
+#include "fos.h"
+#include "fos_internal.h"
+
+namespace fos {
+
+// Sign flips of the random Hadamard transform for the two bf16 halves of
+// word k (elements 2k and 2k+1).
+__device__ __forceinline__ uint32_t rht_word_mask(uint32_t mask16, int k) {
+  return (((mask16 >> (2 * k)) & 1u) << 15) | (((mask16 >> (2 * k + 1)) & 1u) << 31);
+}
+
+// In-place 16-point fast Walsh-Hadamard transform of the packed pairs with
+// butterflies (a, b) -> (a + b, a - b) at strides 1, 2, 4, 8, then * 0.25.
+__device__ __forceinline__ void fwht16_pairs(float2 (&P)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h *= 2) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2 * h) {
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float2 a = P[j], b = P[j + h];
+        P[j] = add2(a, b);
+        P[j + h] = sub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) P[i] = mul2(P[i], make_float2(0.25f, 0.25f));
+}
+
+// Unpack two blocks of 8 bf16x2 words into 16 packed (A_i, B_i) pairs.
+__device__ __forceinline__ void unpack_pairs(const uint4 (&wa)[2], const uint4 (&wb)[2],
+                                             float2 (&P)[16]) {
+  const uint32_t A[8] = {wa[0].x, wa[0].y, wa[0].z, wa[0].w, wa[1].x, wa[1].y, wa[1].z, wa[1].w};
+  const uint32_t B[8] = {wb[0].x, wb[0].y, wb[0].z, wb[0].w, wb[1].x, wb[1].y, wb[1].z, wb[1].w};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    P[2 * k] = make_float2(bf_lo(A[k]), bf_lo(B[k]));
+    P[2 * k + 1] = make_float2(bf_hi(A[k]), bf_hi(B[k]));
+  }
+}
+
+// max |x| of 8 bf16x2 words, as binary32 bits (NaN/Inf give >= 0x7f800000).
+__device__ __forceinline__ uint32_t amax_bits_bf16(const uint4 (&w)[2]) {
+  uint32_t m = __vmaxu2(w[0].x & 0x7fff7fffu, w[0].y & 0x7fff7fffu);
+  m = __vmaxu2(m, w[0].z & 0x7fff7fffu);
+  m = __vmaxu2(m, w[0].w & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].x & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].y & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].z & 0x7fff7fffu);
+  m = __vmaxu2(m, w[1].w & 0x7fff7fffu);
+  return max(m & 0xffffu, m >> 16) << 16;
+}
+
+// max |P[i].x| and max |P[i].y| as binary32 bits.
+__device__ __forceinline__ void amax_bits_pairs(const float2 (&P)[16], uint32_t& ma, uint32_t& mb) {
+  ma = 0;
+  mb = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    ma = max(ma, __float_as_uint(P[i].x) & 0x7fffffffu);
+    mb = max(mb, __float_as_uint(P[i].y) & 0x7fffffffu);
+  }
+}
+
+// Candidate scale codes of a block with amax a: (s6, s4) as E4M3 bytes.
+template <bool F46>
+__device__ __forceinline__ void cand_scales(float a, float St, uint32_t& s6, uint32_t& s4) {
+  const float r = (St == 0.0f) ? 0.0f : __fdiv_rn(a, St);
+  // r >= 0 for valid input; the 0x7f mask keeps a caller-supplied negative
+  // amax from indexing past the 128-entry scale table
+  if (F46) {
+    const uint32_t both = e4m3x2(__fdiv_rn(r, 6.0f), __fmul_rn(r, 0.25f));
+    s6 = (both >> 8) & 0x7fu;
+    s4 = both & 0x7fu;
+  } else {
+    s6 = e4m3x2(0.0f, __fdiv_rn(r, 6.0f)) & 0x7fu;
+    s4 = 0;
+  }
+}
+
+struct Cand {
+  uint32_t ca[2], cb[2];  // codes of block A and block B (2 words each)
+  float2 err;             // (error A, error B)
+};
+
+// Round both blocks with one candidate scale per block and, when WANT_ERR,
+// form the binary32 squared error d = fma(-q, e, w), t = d*d, pairwise tree.
+template <bool WANT_ERR>
+__device__ __forceinline__ Cand candidate(const float2 (&P)[16], float2 inv, float2 nege, float nz) {
+  Cand c;
+  float2 v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = mul2(P[i], inv);
+  c.ca[0] = e2m1x8(v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x);
+  c.ca[1] = e2m1x8(v[8].x, v[9].x, v[10].x, v[11].x, v[12].x, v[13].x, v[14].x, v[15].x);
+  c.cb[0] = e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y);
+  c.cb[1] = e2m1x8(v[8].y, v[9].y, v[10].y, v[11].y, v[12].y, v[13].y, v[14].y, v[15].y);
+  c.err = make_float2(0.0f, 0.0f);
+  if (WANT_ERR) {
+    uint32_t ha[8], hb[8];
+    e2m1x8_to_h2(c.ca[0], ha);
+    e2m1x8_to_h2(c.ca[1], ha + 4);
+    e2m1x8_to_h2(c.cb[0], hb);
+    e2m1x8_to_h2(c.cb[1], hb + 4);
+    float2 l1[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 q0 = make_float2(h_lo(ha[k]), h_lo(hb[k]));
+      const float2 q1 = make_float2(h_hi(ha[k]), h_hi(hb[k]));
+      const float2 d0 = fma2(q0, nege, P[2 * k]);
+      const float2 d1 = fma2(q1, nege, P[2 * k + 1]);
+      // squares as fma(d, d, nz) with nz = -0 known only at run time: equal to
+      // RN(d*d), and not fusable into the following add (a packed mul, or an
+      // fma with a literal -0 addend, feeding a packed add was contracted
+      // into one fma by the code generator, even as .rn PTX)
+      const float2 z2 = make_float2(nz, nz);
+      const float2 t0 = fma2(d0, d0, z2);
+      const float2 t1 = fma2(d1, d1, z2);
+      l1[k] = add2(t0, t1);
+    }
+    const float2 l2a = add2(l1[0], l1[1]), l2b = add2(l1[2], l1[3]);
+    const float2 l2c = add2(l1[4], l1[5]), l2d = add2(l1[6], l1[7]);
+    c.err = add2(add2(l2a, l2b), add2(l2c, l2d));
+  }
+  return c;
+}
+
+// Stochastic rounding of the kept candidate of one block (A: which = 0,
+// B: which = 1) with 16 Philox bytes.
+__device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float inv, uint4 rnd,
+                                         uint32_t (&out)[2]) {
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float w = which ? P[i].y : P[i].x;
+    const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
+    q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
+  }
+  out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+  out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+}
+
+// Bit i of a -> bit 2i, bit i of b -> bit 2i+1.
+__device__ __forceinline__ unsigned long long interleave_bits(uint32_t a, uint32_t b) {
+  auto spread = [](unsigned long long x) {
+    x = (x | (x << 16)) & 0x0000FFFF0000FFFFull;
+    x = (x | (x << 8)) & 0x00FF00FF00FF00FFull;
+    x = (x | (x << 4)) & 0x0F0F0F0F0F0F0F0Full;
+    x = (x | (x << 2)) & 0x3333333333333333ull;
+    x = (x | (x << 1)) & 0x5555555555555555ull;
+    return x;
+  };
+  return spread(a) | (spread(b) << 1);
+}
+
+__device__ __forceinline__ void store_choice64(const OutDesc& o, unsigned long long gbit,
+                                               unsigned long long word) {
+  unsigned long long* base = reinterpret_cast<unsigned long long*>(o.choice);
+  if (o.choice_aligned) {
+    base[gbit >> 6] = word;
+  } else if (word) {
+    // only words that receive a set bit are touched, so nothing past the
+    // last block's word is accessed
+    const int sh = (int)(gbit & 63);
+    const unsigned long long lo = word << sh, hi = sh ? (word >> (64 - sh)) : 0ull;
+    if (lo) atomicOr(base + (gbit >> 6), lo);
+    if (hi) atomicOr(base + (gbit >> 6) + 1, hi);
+  }
+}
+
+__device__ __forceinline__ float tensor_scale_of(const QuantArgs& a, int b, bool f46) {
+  const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_ws[b]);
+  return __fdiv_rn(A, f46 ? 1792.0f : 2688.0f);
+}
+
+// (E(c), 1/E(c)) for every non-negative E4M3 code c, E(c) = float(c) * S_t;
+// a zero E gives a zero inverse, an overflowing inverse is clamped to
+// FLT_MAX.
+__device__ __forceinline__ void build_scale_table(float2* tab, float St) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float E = __fmul_rn(e4m3_to_f32((uint32_t)c), St);
+    const float inv = (E == 0.0f) ? 0.0f : fminf(__frcp_rn(E), kFltMax);
+    tab[c] = make_float2(E, inv);
+  }
+}
+
+}  // namespace fos

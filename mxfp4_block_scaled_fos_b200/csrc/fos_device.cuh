@@ -22,12 +22,58 @@ __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w <<
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // ---------------------------------------------------------------- f32x2
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-// a - b with one rounding: b * (-1) is exact, the sum rounds once.
+// Packed binary32 pairs, as inline PTX with an explicit .rn.  Measured on
+// sm_100a with CUDA 12.9: a packed mul whose result feeds a packed add is
+// still contracted into one fused instruction (both with the
+// __fmul2_rn/__fadd2_rn intrinsics and with mul.rn/add.rn PTX), which drops
+// a rounding.  Wherever the definition needs RN(a*b) followed by an add, the
+// product is formed as fma(a, b, -0) instead (see the error tree).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+// a * b + c with one rounding per component.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+// a - b with one rounding per component.
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
 }
 
 // ---------------------------------------------------------------- E2M1
@@ -47,17 +93,27 @@ __device__ __forceinline__ uint32_t e2m1x8(float e0, float e1, float e2, float e
   return out;
 }
 
-// Eight E2M1 nibbles -> four f16x2 words (h[k] holds elements 2k, 2k+1),
-// exact.
+// Two E2M1 nibbles (the low byte of `byte`) -> f16x2 (low nibble in the low
+// half), exact.  The byte travels in a 16-bit register and is split with
+// mov.b16: unpacking a 32-bit register into four .b8 registers straight
+// after the packing cvt lost bytes 2 and 3 in measurement.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+  uint32_t out;
+  const unsigned short t = (unsigned short)(byte & 0xffu);
+  asm("{\n\t.reg .b8 lo, hi;\n\t"
+      "mov.b16 {lo, hi}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, lo;\n\t}"
+      : "=r"(out)
+      : "h"(t));
+  return out;
+}
+
+// Eight E2M1 nibbles -> four f16x2 words (h[k] holds elements 2k, 2k+1).
 __device__ __forceinline__ void e2m1x8_to_h2(uint32_t codes, uint32_t h[4]) {
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(codes));
+  h[0] = e2m1x2_to_h2(codes);
+  h[1] = e2m1x2_to_h2(codes >> 8);
+  h[2] = e2m1x2_to_h2(codes >> 16);
+  h[3] = e2m1x2_to_h2(codes >> 24);
 }
 
 __device__ __forceinline__ float h_lo(uint32_t h) {

@@ -36,6 +36,10 @@ struct QuantArgs {
   uint32_t* status = nullptr;       // nullable
   unsigned long long seed = 0;
   long long elem_offset = 0;
+  // -0.0f, passed at run time: the addend of the squares in the error sums,
+  // opaque to the code generator so that a square is never seen as a plain
+  // product and fused into the following add
+  float neg_zero = -0.0f;
   OutDesc row, col;
 };
 

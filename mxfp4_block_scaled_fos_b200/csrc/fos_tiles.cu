@@ -1,16 +1,496 @@
-// fos_tiles.cu -- quantizers that need both orientations of a tile:
-// rowwise + colwise 1x16 and 16x16 2D block scaling.
-#include "fos.h"
-#include "fos_internal.h"
+// fos_tiles.cu -- NVFP4 quantizers that need both orientations of a tile:
+//   * 1x16 rowwise + colwise ("transposed inputs" option of the Hugging Face
+//     transformers doc "Four Over Six", usage section): x and x^T are each
+//     quantized with 16-element blocks along their rows, one read of x;
+//   * 16x16 2D block scaling (same section): one scale and one 4/6 choice per
+//     16x16 tile, written row-major and as its exact transpose.
+//
+// A CTA of 256 threads walks a strip of up to 8 sub-tiles of 64 rows x 128
+// columns (16 KB of bf16) down the tensor.  Each sub-tile is staged in shared
+// memory with 16-byte chunks XOR-swizzled by row so that the row-major reads,
+// the column reads and the 16x16 reads are all free of bank conflicts; the
+// next sub-tile's global loads are issued before the current one is
+// processed.  Stochastic-rounding bytes are drawn once per 16 source elements
+// (one Philox call per rowwise block) and shared by both orientations
+// through shared memory.
+#include "fos_core.cuh"
 
 namespace fos {
 
-cudaError_t launch_q1x16_dual(const QuantArgs&, int, int, bool, bool, bool, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kSubRows = 64;
+constexpr int kSubCols = 128;
+constexpr int kStrip = 8;  // sub-tiles per CTA strip (512 rows)
+
+struct TileGeom {
+  int rows, cols;     // tensor
+  int r_strip0, c0;   // strip origin
+};
+
+// smem byte offset of the 16-byte chunk c16 of row r under swizzle f(r).
+template <int SHIFT>
+__device__ __forceinline__ uint32_t chunk_off(int r, int c16) {
+  return (uint32_t)(r * 256 + ((c16 ^ ((r >> SHIFT) & 7)) << 4));
 }
 
-cudaError_t launch_q16x16(const QuantArgs&, int, int, bool, bool, bool, bool, cudaStream_t) {
-  return cudaErrorNotSupported;
+// Global -> registers: 4 16-byte chunks per thread of the sub-tile whose
+// first row is r0 (zero beyond the tensor).
+__device__ __forceinline__ void load_sub(const QuantArgs& a, int b, int r0, int c0, uint4 (&reg)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int q = k * kThreads + threadIdx.x;
+    const int row = q >> 4, c16 = q & 15;
+    const int gr = r0 + row, gc = c0 + c16 * 8;
+    if (gr < a.rows && gc < a.cols) {
+      reg[k] = __ldg(reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs +
+                                                    (long long)gr * a.ld + gc));
+    } else {
+      reg[k] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
+template <int SHIFT>
+__device__ __forceinline__ void store_sub(uint8_t* tile, const uint4 (&reg)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int q = k * kThreads + threadIdx.x;
+    *reinterpret_cast<uint4*>(tile + chunk_off<SHIFT>(q >> 4, q & 15)) = reg[k];
+  }
+}
+
+template <bool SWZ>
+__device__ __forceinline__ long long scale_off(const OutDesc& o, int b, long long R, long long c) {
+  if (SWZ) return (long long)b * o.scales_bs + swz_offset(R, c, o.col_tiles);
+  return (long long)b * o.scales_bs + R * o.scales_ld + c;
+}
+
+__device__ __forceinline__ void store_codes8(const OutDesc& o, int b, long long R, long long byte_col,
+                                             uint32_t w0, uint32_t w1) {
+  *reinterpret_cast<uint2*>(o.codes + (long long)b * o.codes_bs + R * o.codes_ld + byte_col) =
+      make_uint2(w0, w1);
+}
+
+// Stochastic rounding of one block of a pair with explicit per-element bytes.
+__device__ __forceinline__ void sr_block_bytes(const float2 (&P)[16], int which, float inv,
+                                               const uint32_t (&bytes)[16], uint32_t (&out)[2]) {
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float w = which ? P[i].y : P[i].x;
+    const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), bytes[i]);
+    q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
+  }
+  out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+  out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+}
+
+// Quantize the pair P (blocks A, B) with per-block amax bits (ma, mb):
+// returns codes, scale bytes and picks (SR re-rounding done by the caller).
+template <bool F46>
+struct PairResult {
+  uint32_t ca[2], cb[2];
+  uint32_t sa, sb;
+  float inva, invb;
+  uint32_t pa, pb;
+};
+
+template <bool F46>
+__device__ __forceinline__ PairResult<F46> quant_pair(const float2 (&P)[16], uint32_t ma, uint32_t mb,
+                                                      float St, const float2* tab, float nz) {
+  PairResult<F46> r;
+  uint32_t s6a, s4a, s6b, s4b;
+  cand_scales<F46>(__uint_as_float(ma), St, s6a, s4a);
+  cand_scales<F46>(__uint_as_float(mb), St, s6b, s4b);
+  const float2 t6a = tab[s6a], t6b = tab[s6b];
+  const Cand c6 = candidate<F46>(P, make_float2(t6a.y, t6b.y), make_float2(-t6a.x, -t6b.x), nz);
+  r.ca[0] = c6.ca[0]; r.ca[1] = c6.ca[1]; r.cb[0] = c6.cb[0]; r.cb[1] = c6.cb[1];
+  r.sa = s6a; r.sb = s6b; r.inva = t6a.y; r.invb = t6b.y; r.pa = 0; r.pb = 0;
+  if (F46) {
+    const float2 t4a = tab[s4a], t4b = tab[s4b];
+    const Cand c4 = candidate<true>(P, make_float2(t4a.y, t4b.y), make_float2(-t4a.x, -t4b.x), nz);
+    r.pa = c4.err.x < c6.err.x;
+    r.pb = c4.err.y < c6.err.y;
+    if (r.pa) { r.ca[0] = c4.ca[0]; r.ca[1] = c4.ca[1]; r.sa = s4a; r.inva = t4a.y; }
+    if (r.pb) { r.cb[0] = c4.cb[0]; r.cb[1] = c4.cb[1]; r.sb = s4b; r.invb = t4b.y; }
+  }
+  return r;
+}
+
+// --------------------------------------------------------------------------
+// 1x16 rowwise + colwise.  grid (ceil(cols/128), ceil(rows/512), batch).
+template <bool F46, bool SR, bool SWZ, bool ROW>
+__global__ void __launch_bounds__(kThreads, 2) k_dual1x16(const QuantArgs a) {
+  __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
+  __shared__ __align__(16) uint4 s_rnd[SR ? kSubRows * 8 : 1];
+  __shared__ float2 s_tab[128];
+  __shared__ uint32_t s_rbits[kSubRows];
+  __shared__ uint32_t s_cbits[kSubCols];
+
+  const int b = blockIdx.z;
+  const int c0 = blockIdx.x * kSubCols;
+  const int rs0 = blockIdx.y * (kSubRows * kStrip);
+  const float St = tensor_scale_of(a, b, F46);
+  build_scale_table(s_tab, St);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
+    if (a.col.tensor_scale) a.col.tensor_scale[b] = St;
+  }
+  if (threadIdx.x < kSubCols) s_cbits[threadIdx.x] = 0;
+  if (threadIdx.x < kSubRows) s_rbits[threadIdx.x] = 0;
+
+  const int t = threadIdx.x;
+  // rowwise role: row rr, block pair pp (blocks 2pp, 2pp+1 of the 8 in a row)
+  const int rr = t & 63, pp = t >> 6;
+  // colwise role: column pair cq (cols 2cq, 2cq+1), row group gq (16 rows)
+  const int cq = t & 63, gq = t >> 6;
+  const long long nbc = a.cols / 16;   // rowwise blocks per row
+  const long long nrg = a.rows / 16;   // colwise blocks per column
+  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
+  uint32_t bad = 0;
+  uint32_t cbits_a = 0, cbits_b = 0;   // colwise picks of this thread's 2 columns
+
+  uint4 reg[4];
+  load_sub(a, b, rs0, c0, reg);
+  for (int k = 0; k < kStrip; ++k) {
+    const int r0 = rs0 + k * kSubRows;
+    if (r0 >= a.rows) break;
+    __syncthreads();
+    store_sub<0>(s_tile, reg);
+    __syncthreads();
+    if (k + 1 < kStrip && r0 + kSubRows < a.rows) load_sub(a, b, r0 + kSubRows, c0, reg);
+
+    // ---------------- rowwise pass (also draws the SR bytes) ----------------
+    {
+      const int gr = r0 + rr;
+      const int bc = c0 / 16 + 2 * pp;   // global block column of block A
+      const bool va = gr < a.rows && bc < nbc;
+      const bool vb = gr < a.rows && bc + 1 < nbc;
+      if (SR) {
+        uint4 ra = make_uint4(0, 0, 0, 0), rb = ra;
+        if (va) ra = sr_bytes16(a.seed, gbase + (long long)gr * a.cols + bc * 16);
+        if (vb) rb = sr_bytes16(a.seed, gbase + (long long)gr * a.cols + (bc + 1) * 16);
+        s_rnd[rr * 8 + 2 * pp] = ra;
+        s_rnd[rr * 8 + 2 * pp + 1] = rb;
+      }
+      if (ROW && va) {
+        uint4 wa[2], wb[2];
+        wa[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp));
+        wa[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp + 1));
+        wb[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp + 2));
+        wb[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp + 3));
+        float2 P[16];
+        unpack_pairs(wa, wb, P);
+        const uint32_t ma = amax_bits_bf16(wa), mb = amax_bits_bf16(wb);
+        bad |= max(ma, mb) >= 0x7f800000u;
+        PairResult<F46> q = quant_pair<F46>(P, ma, mb, St, s_tab, a.neg_zero);
+        if (SR) {
+          sr_block(P, 0, q.inva, s_rnd[rr * 8 + 2 * pp], q.ca);
+          sr_block(P, 1, q.invb, s_rnd[rr * 8 + 2 * pp + 1], q.cb);
+        }
+        store_codes8(a.row, b, gr, bc * 8, q.ca[0], q.ca[1]);
+        a.row.scales[scale_off<SWZ>(a.row, b, gr, bc)] = (uint8_t)q.sa;
+        if (vb) {
+          store_codes8(a.row, b, gr, (bc + 1) * 8, q.cb[0], q.cb[1]);
+          a.row.scales[scale_off<SWZ>(a.row, b, gr, bc + 1)] = (uint8_t)q.sb;
+        }
+        if (F46 && a.row.choice && (q.pa | q.pb))
+          atomicOr(&s_rbits[rr], (q.pa << (2 * pp)) | ((vb ? q.pb : 0u) << (2 * pp + 1)));
+      }
+    }
+    if (SR) __syncthreads();  // SR bytes visible to the colwise pass
+
+    // ---------------- colwise pass ----------------
+    {
+      const int gc = c0 + 2 * cq;
+      const int grow = r0 + 16 * gq;
+      if (gc < a.cols && grow < a.rows) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = 16 * gq + i;
+          w[i] = *reinterpret_cast<const uint32_t*>(s_tile + chunk_off<0>(r, cq >> 2) + (cq & 3) * 4);
+        }
+        float2 P[16];
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          P[i] = make_float2(bf_lo(w[i]), bf_hi(w[i]));
+          m = __vmaxu2(m, w[i] & 0x7fff7fffu);
+        }
+        const uint32_t ma = (m & 0xffffu) << 16, mb = m & 0xffff0000u;
+        bad |= max(ma, mb) >= 0x7f800000u;
+        PairResult<F46> q = quant_pair<F46>(P, ma, mb, St, s_tab, a.neg_zero);
+        if (SR) {
+          uint32_t ba[16], bb[16];
+          const uint8_t* rb = reinterpret_cast<const uint8_t*>(s_rnd);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int r = 16 * gq + i;
+            const uint32_t two = *reinterpret_cast<const uint16_t*>(rb + r * 128 + (cq >> 3) * 16 +
+                                                                    2 * (cq & 7));
+            ba[i] = two & 0xffu;
+            bb[i] = two >> 8;
+          }
+          sr_block_bytes(P, 0, q.inva, ba, q.ca);
+          sr_block_bytes(P, 1, q.invb, bb, q.cb);
+        }
+        const long long rg = grow / 16;
+        store_codes8(a.col, b, gc, rg * 8, q.ca[0], q.ca[1]);
+        store_codes8(a.col, b, gc + 1, rg * 8, q.cb[0], q.cb[1]);
+        a.col.scales[scale_off<SWZ>(a.col, b, gc, rg)] = (uint8_t)q.sa;
+        a.col.scales[scale_off<SWZ>(a.col, b, gc + 1, rg)] = (uint8_t)q.sb;
+        cbits_a |= q.pa << (4 * k + gq);
+        cbits_b |= q.pb << (4 * k + gq);
+      }
+    }
+
+    // rowwise choice bits of this sub-tile: 8 bits per row
+    if (ROW && F46 && a.row.choice) {
+      __syncthreads();
+      if (t < kSubRows) {
+        const uint32_t v = s_rbits[t];
+        s_rbits[t] = 0;
+        const int gr = r0 + t;
+        if (gr < a.rows) {
+          const unsigned long long bit = ((unsigned long long)b * a.rows + gr) * nbc + c0 / 16;
+          if (a.row.choice_aligned) {
+            a.row.choice[bit >> 3] = (uint8_t)v;
+          } else if (v) {
+            unsigned int* wp = reinterpret_cast<unsigned int*>(a.row.choice) + (bit >> 5);
+            const int sh = (int)(bit & 31);
+            const unsigned long long vv = (unsigned long long)v << sh;
+            if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
+            if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
+          }
+        }
+      }
+    }
+  }
+
+  // colwise choice bits of the strip: 32 row groups per column
+  if (F46 && a.col.choice) {
+    if (cbits_a) atomicOr(&s_cbits[2 * cq], cbits_a);
+    if (cbits_b) atomicOr(&s_cbits[2 * cq + 1], cbits_b);
+    __syncthreads();
+    if (t < kSubCols) {
+      const int gc = c0 + t;
+      if (gc < a.cols) {
+        const uint32_t v = s_cbits[t];
+        const unsigned long long bit = ((unsigned long long)b * a.cols + gc) * nrg + rs0 / 16;
+        unsigned int* base = reinterpret_cast<unsigned int*>(a.col.choice);
+        if (a.col.choice_aligned) {
+          base[bit >> 5] = v;
+        } else if (v) {
+          const int sh = (int)(bit & 31);
+          const unsigned long long vv = (unsigned long long)v << sh;
+          if ((uint32_t)vv) atomicOr(base + (bit >> 5), (uint32_t)vv);
+          if ((uint32_t)(vv >> 32)) atomicOr(base + (bit >> 5) + 1, (uint32_t)(vv >> 32));
+        }
+      }
+    }
+  }
+  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// Nibbles of a (8) into the low halves of 8 bytes, b into the high halves:
+// byte k = a_k | b_k << 4.
+__device__ __forceinline__ unsigned long long zip_nibbles(uint32_t a, uint32_t b) {
+  auto spread = [](unsigned long long x) {
+    x = (x | (x << 16)) & 0x0000FFFF0000FFFFull;
+    x = (x | (x << 8)) & 0x00FF00FF00FF00FFull;
+    x = (x | (x << 4)) & 0x0F0F0F0F0F0F0F0Full;
+    return x;
+  };
+  return spread(a) | (spread(b) << 4);
+}
+
+// --------------------------------------------------------------------------
+// 16x16 2D block scaling.  grid (ceil(cols/128), ceil(rows/512), batch).
+// In a sub-tile, 8 threads own one 16x16 tile; thread i holds rows 2i, 2i+1
+// as the pair (A, B), so the per-row error trees come out of the pair code
+// and the tree over the 16 row sums is a horizontal add plus three
+// xor-shuffles.
+template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
+__global__ void __launch_bounds__(kThreads, 2) k_2d16x16(const QuantArgs a) {
+  __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
+  __shared__ __align__(16) uint8_t s_tc[COL ? kSubCols * 32 : 16];
+  __shared__ float2 s_tab[128];
+  __shared__ uint32_t s_bits[kSubRows / 16];
+
+  const int b = blockIdx.z;
+  const int c0 = blockIdx.x * kSubCols;
+  const int rs0 = blockIdx.y * (kSubRows * kStrip);
+  const float St = tensor_scale_of(a, b, F46);
+  build_scale_table(s_tab, St);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
+    if (COL && a.col.tensor_scale) a.col.tensor_scale[b] = St;
+  }
+  if (threadIdx.x < kSubRows / 16) s_bits[threadIdx.x] = 0;
+
+  const int t = threadIdx.x;
+  const int tile = t >> 3, i = t & 7;
+  const int tr = tile >> 3, tc = tile & 7;   // tile row (0..3) and column (0..7)
+  const long long ntc = a.cols / 16, ntr = a.rows / 16;
+  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
+  uint32_t bad = 0;
+
+  uint4 reg[4];
+  load_sub(a, b, rs0, c0, reg);
+  for (int k = 0; k < kStrip; ++k) {
+    const int r0 = rs0 + k * kSubRows;
+    if (r0 >= a.rows) break;
+    __syncthreads();
+    store_sub<1>(s_tile, reg);
+    __syncthreads();
+    if (k + 1 < kStrip && r0 + kSubRows < a.rows) load_sub(a, b, r0 + kSubRows, c0, reg);
+
+    const long long gtr = (r0 >> 4) + tr;      // global tile row
+    const long long gtc = (c0 >> 4) + tc;      // global tile column
+    const bool valid = gtr < ntr && gtc < ntc; // uniform over the 8 threads of a tile
+    uint32_t pick = 0;
+    if (valid) {
+      const int ra = 16 * tr + 2 * i;
+      uint4 wa[2], wb[2];
+      wa[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra, 2 * tc));
+      wa[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra, 2 * tc + 1));
+      wb[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra + 1, 2 * tc));
+      wb[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra + 1, 2 * tc + 1));
+      float2 P[16];
+      unpack_pairs(wa, wb, P);
+      // the 8 lanes of one tile are all valid or all invalid: shuffle among them
+      const uint32_t gmask = 0xffu << (threadIdx.x & 24);
+      uint32_t m = max(amax_bits_bf16(wa), amax_bits_bf16(wb));
+      m = max(m, __shfl_xor_sync(gmask, m, 1));
+      m = max(m, __shfl_xor_sync(gmask, m, 2));
+      m = max(m, __shfl_xor_sync(gmask, m, 4));
+      bad |= m >= 0x7f800000u;
+      uint32_t s6, s4;
+      cand_scales<F46>(__uint_as_float(m), St, s6, s4);
+      const float2 t6 = s_tab[s6];
+      const Cand c6 = candidate<F46>(P, make_float2(t6.y, t6.y), make_float2(-t6.x, -t6.x), a.neg_zero);
+      uint32_t ca[2] = {c6.ca[0], c6.ca[1]}, cb[2] = {c6.cb[0], c6.cb[1]};
+      uint32_t s = s6;
+      float inv = t6.y;
+      if (F46) {
+        const float2 t4 = s_tab[s4];
+        const Cand c4 = candidate<true>(P, make_float2(t4.y, t4.y), make_float2(-t4.x, -t4.x), a.neg_zero);
+        // tree over the 16 row sums: (2i)+(2i+1), then across threads
+        float e6 = __fadd_rn(c6.err.x, c6.err.y), e4 = __fadd_rn(c4.err.x, c4.err.y);
+#pragma unroll
+        for (int sh = 1; sh < 8; sh *= 2) {
+          e6 = __fadd_rn(e6, __shfl_xor_sync(gmask, e6, sh));
+          e4 = __fadd_rn(e4, __shfl_xor_sync(gmask, e4, sh));
+        }
+        pick = e4 < e6;
+        if (pick) { ca[0] = c4.ca[0]; ca[1] = c4.ca[1]; cb[0] = c4.cb[0]; cb[1] = c4.cb[1]; s = s4; inv = t4.y; }
+      }
+      const long long grA = r0 + ra;
+      if (SR) {
+        sr_block(P, 0, inv, sr_bytes16(a.seed, gbase + grA * a.cols + gtc * 16), ca);
+        sr_block(P, 1, inv, sr_bytes16(a.seed, gbase + (grA + 1) * a.cols + gtc * 16), cb);
+      }
+      if (ROW) {
+        store_codes8(a.row, b, grA, gtc * 8, ca[0], ca[1]);
+        store_codes8(a.row, b, grA + 1, gtc * 8, cb[0], cb[1]);
+        a.row.scales[scale_off<SWZ>(a.row, b, grA, gtc)] = (uint8_t)s;
+        a.row.scales[scale_off<SWZ>(a.row, b, grA + 1, gtc)] = (uint8_t)s;
+      }
+      if (COL) {
+        // byte for rows (2i, 2i+1) of each of the tile's 16 columns
+        const unsigned long long lo = zip_nibbles(ca[0], cb[0]), hi = zip_nibbles(ca[1], cb[1]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          s_tc[(16 * tc + c) * 32 + 8 * tr + i] = (uint8_t)(lo >> (8 * c));
+          s_tc[(16 * tc + 8 + c) * 32 + 8 * tr + i] = (uint8_t)(hi >> (8 * c));
+        }
+        const long long gcA = (c0 + 16 * tc) + 2 * i;
+        a.col.scales[scale_off<SWZ>(a.col, b, gcA, gtr)] = (uint8_t)s;
+        a.col.scales[scale_off<SWZ>(a.col, b, gcA + 1, gtr)] = (uint8_t)s;
+      }
+      if (F46 && i == 0 && pick && (a.row.choice || a.col.choice)) atomicOr(&s_bits[tr], 1u << tc);
+    }
+    __syncthreads();
+    if (COL) {
+      // transposed codes: column col, 32 rows per half
+      const int col = t >> 1, h = t & 1;
+      const int gc = c0 + col;
+      const int grow = r0 + 32 * h;
+      if (gc < a.cols && grow < a.rows) {
+        const uint4 v = *reinterpret_cast<const uint4*>(s_tc + col * 32 + 16 * h);
+        const long long byte_col = grow / 2;
+        store_codes8(a.col, b, gc, byte_col, v.x, v.y);
+        if (grow + 16 < a.rows) store_codes8(a.col, b, gc, byte_col + 8, v.z, v.w);
+      }
+    }
+    if (F46 && t < kSubRows / 16) {
+      const uint32_t v = s_bits[t];
+      s_bits[t] = 0;
+      const long long gtr2 = (r0 >> 4) + t;
+      if (gtr2 < ntr) {
+        const unsigned long long bit = ((unsigned long long)b * ntr + gtr2) * ntc + (c0 >> 4);
+        uint8_t* ch[2] = {ROW ? a.row.choice : nullptr, COL ? a.col.choice : nullptr};
+        const int aligned[2] = {a.row.choice_aligned, a.col.choice_aligned};
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+          if (!ch[z]) continue;
+          if (aligned[z]) {
+            ch[z][bit >> 3] = (uint8_t)v;
+          } else if (v) {
+            unsigned int* wp = reinterpret_cast<unsigned int*>(ch[z]) + (bit >> 5);
+            const int sh = (int)(bit & 31);
+            const unsigned long long vv = (unsigned long long)v << sh;
+            if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
+            if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
+          }
+        }
+      }
+    }
+  }
+  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+}  // namespace
+
+cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
+                              bool want_row, cudaStream_t st) {
+  const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * kStrip - 1) / (kSubRows * kStrip),
+               (unsigned)batch);
+  const bool f46 = fmt == 0;
+#define FOS_L(F, S, W, R) k_dual1x16<F, S, W, R><<<g, kThreads, 0, st>>>(a)
+#define FOS_R(F, S, W) do { if (want_row) FOS_L(F, S, W, true); else FOS_L(F, S, W, false); } while (0)
+#define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)
+#define FOS_S(F) do { if (sr) FOS_W(F, true); else FOS_W(F, false); } while (0)
+  if (f46) FOS_S(true);
+  else     FOS_S(false);
+#undef FOS_S
+#undef FOS_W
+#undef FOS_R
+#undef FOS_L
+  return cudaGetLastError();
+}
+
+cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz, bool want_row,
+                          bool want_col, cudaStream_t st) {
+  const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * kStrip - 1) / (kSubRows * kStrip),
+               (unsigned)batch);
+  const bool f46 = fmt == 0;
+#define FOS_L(F, S, W, R, C) k_2d16x16<F, S, W, R, C><<<g, kThreads, 0, st>>>(a)
+#define FOS_C(F, S, W, R) do { if (want_col) FOS_L(F, S, W, R, true); else FOS_L(F, S, W, R, false); } while (0)
+#define FOS_R(F, S, W) do { if (want_row) FOS_C(F, S, W, true); else FOS_C(F, S, W, false); } while (0)
+#define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)
+#define FOS_S(F) do { if (sr) FOS_W(F, true); else FOS_W(F, false); } while (0)
+  if (f46) FOS_S(true);
+  else     FOS_S(false);
+#undef FOS_S
+#undef FOS_W
+#undef FOS_R
+#undef FOS_C
+#undef FOS_L
+  return cudaGetLastError();
 }
 
 }  // namespace fos

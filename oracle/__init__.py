@@ -251,7 +251,8 @@ def quantize(x_bits: np.ndarray, fmt: int = FMT_NVFP4_46, blk: int = BLK_1X16,
     if colwise:
         out["c_codes"] = np.zeros((b, c, r // 2), np.uint8)
         out["c_scales"] = np.zeros((b, c, r // 16), np.uint8)
-        out["c_choice"] = np.zeros((b * c * r // 16 + 7) // 8, np.uint8)
+        nblk_c = b * c * r // 16 if blk != BLK_16X16 else b * (r // 16) * (c // 16)
+        out["c_choice"] = np.zeros((nblk_c + 7) // 8, np.uint8)
     out["tensor_scale"] = np.zeros(b, np.float32)
     o = Opts(fmt, blk, rnd, int(rht), seed, elem_offset)
     ain = None

@@ -539,7 +539,9 @@ int or_quantize(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
               g[i * 16 + j] = base + r * cols + c;
             }
           uint8_t s = nvfp4_block(w, g, 256, S_t, o, codes, &p4);
+          /* R7: one bit per tile in tile row-major order, for both copies */
           set_bit(r_choice, (b * (rows / 16) + tr) * (cols / 16) + tc, p4);
+          set_bit(c_choice, (b * (rows / 16) + tr) * (cols / 16) + tc, p4);
           for (int i = 0; i < 16; i++) {
             int64_t r = tr * 16 + i;
             if (r_scales) r_scales[(b * rows + r) * (cols / 16) + tc] = s;

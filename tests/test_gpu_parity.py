@@ -193,8 +193,25 @@ def test_dequantize_oracle_codes(fmt, swizzle):
     assert_bytes_equal(np_bits(y), ref, "dequantized")
 
 
-def test_activation_outliers_rht_full_size():
-    """8192x4096 activations with 1% outlier channels, RHT16 (seed 0), 4/6 RNE."""
+# A block whose two candidate errors are exactly equal in binary32 (found in a
+# seeded Student-t tensor): the tie must keep 6.  Rows 0 and 1 carry the same
+# block in both halves of a pair, row 2 sets the tensor amax.
+TIE_BLOCK = [0.0002307891845703125, 0.00262451171875, 0.0006256103515625, -9.918212890625e-05,
+             -0.0089111328125, 0.00011682510375976562, -0.00115966796875, -6.4849853515625e-05,
+             -0.0004405975341796875, -0.00360107421875, 0.00201416015625, 0.00144195556640625,
+             0.000324249267578125, 0.0010528564453125, 0.000339508056640625, 0.0008544921875]
+
+
+def test_exact_tie_block_keeps_6():
     dev = require_gpu()
-    x = workloads.activation_outliers(8192, 4096, device=dev)
-    check_quantize(x, rht=True, seed=0)
+    rows = torch.zeros(16, 32)
+    rows[0, :16] = torch.tensor(TIE_BLOCK)
+    rows[0, 16:] = torch.tensor(TIE_BLOCK)
+    rows[1, 16:] = torch.tensor(TIE_BLOCK)
+    rows[2, 0] = 0.06787109375
+    x = rows.to(torch.bfloat16).to(dev)
+    r, _, ref = check_quantize(x)
+    # the oracle sees an exact tie here and keeps the 6-candidate
+    assert not (ref["r_choice"][0] & 0b1011)
+    check_quantize(x.t().contiguous(), colwise=True)
+    check_quantize(x, rounding="sr", seed=1)

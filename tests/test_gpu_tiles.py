@@ -1,0 +1,80 @@
+"""GPU parity of the two-orientation quantizers against the oracle:
+1x16 rowwise + colwise (x and x^T from one read) and 16x16 2D block scaling
+with its exact transposed copy.  Shapes cover whole and ragged 64x128
+sub-tiles, strips shorter and longer than 512 rows, batches, and the
+bitmap layouts whose words are owned by one CTA or shared."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import mxfp4_block_scaled_fos_b200 as F
+
+from helpers import check_quantize, np_bits, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 16, 16), (1, 64, 128), (2, 80, 272), (1, 512, 256), (1, 528, 400), (3, 1040, 128),
+          (1, 1024, 1024)]
+
+
+def _rand(shape, seed, dev, kind="heavy"):
+    g = torch.Generator().manual_seed(seed)
+    if kind == "heavy":
+        z = torch.randn(shape, generator=g)
+        c = sum(torch.randn(shape, generator=g) ** 2 for _ in range(3))
+        x = z / torch.sqrt(c / 3) * 1e-3
+    else:
+        x = torch.randn(shape, generator=g) * torch.exp2(
+            torch.randint(-12, 12, shape[:-1] + (1,), generator=g).float())
+    return x.to(torch.bfloat16).to(dev)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("rounding", ["rne", "sr"])
+@pytest.mark.parametrize("fmt", ["nvfp4_46", "nvfp4_6"])
+def test_dual_1x16(shape, rounding, fmt):
+    dev = require_gpu()
+    x = _rand(shape, shape[1] * 7 + shape[2], dev)
+    check_quantize(x, fmt=fmt, rounding=rounding, seed=99, rowwise=True, colwise=True)
+
+
+@pytest.mark.parametrize("shape", [(1, 64, 128), (2, 528, 400)])
+def test_colwise_only_and_swizzled(shape):
+    dev = require_gpu()
+    x = _rand(shape, 5, dev, "scaled")
+    check_quantize(x, rowwise=False, colwise=True)
+    check_quantize(x, rowwise=True, colwise=True, swizzle=True, rounding="sr", seed=3)
+
+
+def test_dual_sr_element_offset():
+    dev = require_gpu()
+    x = _rand((1, 96, 160), 8, dev)
+    check_quantize(x, rounding="sr", seed=17, elem_offset=16 * 12345, colwise=True)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("rounding", ["rne", "sr"])
+@pytest.mark.parametrize("fmt", ["nvfp4_46", "nvfp4_6"])
+def test_2d_16x16(shape, rounding, fmt):
+    dev = require_gpu()
+    x = _rand(shape, shape[1] + 3 * shape[2], dev, "scaled")
+    check_quantize(x, fmt=fmt, block="16x16", rounding=rounding, seed=5, rowwise=True, colwise=True)
+
+
+@pytest.mark.parametrize("row,col", [(True, False), (False, True)])
+def test_2d_one_orientation_and_swizzle(row, col):
+    dev = require_gpu()
+    x = _rand((2, 272, 400), 12, dev)
+    check_quantize(x, block="16x16", rowwise=row, colwise=col)
+    check_quantize(x, block="16x16", rowwise=row, colwise=col, swizzle=True)
+
+
+def test_2d_transposed_dequant_is_transpose():
+    dev = require_gpu()
+    x = _rand((1, 256, 384), 21, dev)
+    r, c = F.quantize(x, block="16x16", colwise=True)
+    yr = F.dequantize(r)
+    yc = F.dequantize(c)
+    torch.cuda.synchronize()
+    assert torch.equal(yr[0].t().contiguous().view(torch.int16), yc[0].contiguous().view(torch.int16))
