@@ -218,7 +218,11 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
   } else if (colwise) {
     ce = launch_q1x16_dual(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, st);
   } else {
-    ce = launch_q1x16_rowwise(a, (int)batch, opt->fmt, sr, rht, swz, st);
+    // contiguous rows, packed outputs, 32-byte aligned input: no index
+    // arithmetic per block and one 256-bit load per block
+    const bool dense = ld == cols && rowwise->codes_ld * 2 == cols && !swz &&
+                       rowwise->scales_ld * 16 == cols && aligned(x, 32);
+    ce = launch_q1x16_rowwise(a, (int)batch, opt->fmt, sr, rht, swz, dense, st);
   }
   if (ce == cudaErrorNotSupported) return FOS_ERR_UNSUPPORTED;
   return ce == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;

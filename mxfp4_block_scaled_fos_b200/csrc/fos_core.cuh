@@ -78,18 +78,19 @@ __device__ __forceinline__ void amax_bits_pairs(const float2 (&P)[16], uint32_t&
   }
 }
 
-// Candidate scale codes of a block with amax a: (s6, s4) as E4M3 bytes.
+// Candidate scale codes of a block with amax a: (s6, s4) as E4M3 bytes,
+// s6 = E4M3(RN(r/6)), s4 = E4M3(RN(r/4)), r = RN(a/S_t).
 template <bool F46>
 __device__ __forceinline__ void cand_scales(float a, float St, uint32_t& s6, uint32_t& s4) {
   const float r = (St == 0.0f) ? 0.0f : __fdiv_rn(a, St);
   // r >= 0 for valid input; the 0x7f mask keeps a caller-supplied negative
   // amax from indexing past the 128-entry scale table
   if (F46) {
-    const uint32_t both = e4m3x2(__fdiv_rn(r, 6.0f), __fmul_rn(r, 0.25f));
+    const uint32_t both = e4m3x2(div6_rn(r), __fmul_rn(r, 0.25f));
     s6 = (both >> 8) & 0x7fu;
     s4 = both & 0x7fu;
   } else {
-    s6 = e4m3x2(0.0f, __fdiv_rn(r, 6.0f)) & 0x7fu;
+    s6 = e4m3x2(0.0f, div6_rn(r)) & 0x7fu;
     s4 = 0;
   }
 }
@@ -100,44 +101,39 @@ struct Cand {
 };
 
 // Round both blocks with one candidate scale per block and, when WANT_ERR,
-// form the binary32 squared error d = fma(-q, e, w), t = d*d, pairwise tree.
+// form the binary32 squared error d = fma(-q, e, w), t = d*d, pairwise tree
+// over contiguous elements.  Eight elements at a time, to keep few values
+// live.  nz is -0 passed at run time (see the f32x2 helpers).
 template <bool WANT_ERR>
 __device__ __forceinline__ Cand candidate(const float2 (&P)[16], float2 inv, float2 nege, float nz) {
   Cand c;
-  float2 v[16];
+  float2 half_err[2];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = mul2(P[i], inv);
-  c.ca[0] = e2m1x8(v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x);
-  c.ca[1] = e2m1x8(v[8].x, v[9].x, v[10].x, v[11].x, v[12].x, v[13].x, v[14].x, v[15].x);
-  c.cb[0] = e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y);
-  c.cb[1] = e2m1x8(v[8].y, v[9].y, v[10].y, v[11].y, v[12].y, v[13].y, v[14].y, v[15].y);
-  c.err = make_float2(0.0f, 0.0f);
-  if (WANT_ERR) {
-    uint32_t ha[8], hb[8];
-    e2m1x8_to_h2(c.ca[0], ha);
-    e2m1x8_to_h2(c.ca[1], ha + 4);
-    e2m1x8_to_h2(c.cb[0], hb);
-    e2m1x8_to_h2(c.cb[1], hb + 4);
-    float2 l1[8];
+  for (int h = 0; h < 2; ++h) {
+    float2 v[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float2 q0 = make_float2(h_lo(ha[k]), h_lo(hb[k]));
-      const float2 q1 = make_float2(h_hi(ha[k]), h_hi(hb[k]));
-      const float2 d0 = fma2(q0, nege, P[2 * k]);
-      const float2 d1 = fma2(q1, nege, P[2 * k + 1]);
-      // squares as fma(d, d, nz) with nz = -0 known only at run time: equal to
-      // RN(d*d), and not fusable into the following add (a packed mul, or an
-      // fma with a literal -0 addend, feeding a packed add was contracted
-      // into one fma by the code generator, even as .rn PTX)
+    for (int i = 0; i < 8; ++i) v[i] = mul2(P[8 * h + i], inv);
+    c.ca[h] = e2m1x8(v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x);
+    c.cb[h] = e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y);
+    if (WANT_ERR) {
+      uint32_t ha[4], hb[4];
+      e2m1x8_to_h2(c.ca[h], ha);
+      e2m1x8_to_h2(c.cb[h], hb);
       const float2 z2 = make_float2(nz, nz);
-      const float2 t0 = fma2(d0, d0, z2);
-      const float2 t1 = fma2(d1, d1, z2);
-      l1[k] = add2(t0, t1);
+      float2 l1[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 q0 = make_float2(h_lo(ha[k]), h_lo(hb[k]));
+        const float2 q1 = make_float2(h_hi(ha[k]), h_hi(hb[k]));
+        const float2 d0 = fma2(q0, nege, P[8 * h + 2 * k]);
+        const float2 d1 = fma2(q1, nege, P[8 * h + 2 * k + 1]);
+        // squares as fma(d, d, -0): RN(d*d), never fused into the add below
+        l1[k] = add2(fma2(d0, d0, z2), fma2(d1, d1, z2));
+      }
+      half_err[h] = add2(add2(l1[0], l1[1]), add2(l1[2], l1[3]));
     }
-    const float2 l2a = add2(l1[0], l1[1]), l2b = add2(l1[2], l1[3]);
-    const float2 l2c = add2(l1[4], l1[5]), l2d = add2(l1[6], l1[7]);
-    c.err = add2(add2(l2a, l2b), add2(l2c, l2d));
   }
+  c.err = WANT_ERR ? add2(half_err[0], half_err[1]) : make_float2(0.0f, 0.0f);
   return c;
 }
 

@@ -22,58 +22,42 @@ __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w <<
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // ---------------------------------------------------------------- f32x2
-// Packed binary32 pairs, as inline PTX with an explicit .rn.  Measured on
-// sm_100a with CUDA 12.9: a packed mul whose result feeds a packed add is
-// still contracted into one fused instruction (both with the
-// __fmul2_rn/__fadd2_rn intrinsics and with mul.rn/add.rn PTX), which drops
-// a rounding.  Wherever the definition needs RN(a*b) followed by an add, the
-// product is formed as fma(a, b, -0) instead (see the error tree).
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  float2 r;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return r;
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  float2 r;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return r;
-}
-// a * b + c with one rounding per component.
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  float2 r;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return r;
-}
-// a - b with one rounding per component.
+// Packed binary32 pairs (sm_100 FMUL2/FADD2/FFMA2), each component rounded
+// like its scalar _rn counterpart.  Measured on sm_100a with CUDA 12.9: a
+// packed product that feeds a packed add may still be contracted into one
+// fused instruction (also when written as mul.rn/add.rn PTX, and when the
+// product is an fma with a literal -0 addend), which drops a rounding.  No
+// code here lets a product feed an add; where the definition needs RN(a*b)
+// followed by an add, the product is fma(a, b, z) with z = -0 passed at run
+// time.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// a - b with one rounding: b * (-1) is exact, the sum rounds once.
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  float2 r;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "sub.rn.f32x2 rd, ra, rb;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return r;
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
+// RN(r / 6) without a division: q0 = RN(r*y), y = RN(1/6); the remainder
+// r - 6*q0 is exact as an fma and one correction step q0 + rem*y gives the
+// correctly rounded quotient (P. Markstein, IBM J. Res. Dev. 34(1), 1990).
+// Checked against IEEE division for every binary32 r; it differs only for
+// r < 2^-125, where the quotient is subnormal, so those take a division.
+__device__ __forceinline__ float div6_rn(float r) {
+  if (!(r >= 2.35098870164457501594e-38f)) return __fdiv_rn(r, 6.0f);
+  const float y = 1.0f / 6.0f;
+  const float q0 = __fmul_rn(r, y);
+  const float rem = __fmaf_rn(-q0, 6.0f, r);
+  return __fmaf_rn(rem, y, q0);
+}
+
+// 32 bytes (one 16-element bf16 block) in one 256-bit load; p must be
+// 32-byte aligned.
+__device__ __forceinline__ void ld_block256(const void* p, uint4 (&w)[2]) {
+  asm("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(w[0].x), "=r"(w[0].y), "=r"(w[0].z), "=r"(w[0].w), "=r"(w[1].x), "=r"(w[1].y),
+        "=r"(w[1].z), "=r"(w[1].w)
+      : "l"(p));
 }
 
 // ---------------------------------------------------------------- E2M1
@@ -93,13 +77,13 @@ __device__ __forceinline__ uint32_t e2m1x8(float e0, float e1, float e2, float e
   return out;
 }
 
-// Two E2M1 nibbles (the low byte of `byte`) -> f16x2 (low nibble in the low
-// half), exact.  The byte travels in a 16-bit register and is split with
-// mov.b16: unpacking a 32-bit register into four .b8 registers straight
-// after the packing cvt lost bytes 2 and 3 in measurement.
+// Two E2M1 nibbles -> f16x2 (low nibble in the low half), exact.  `byte`
+// must be zero-extended (bits 8..31 clear): the conversion was measured to
+// give wrong results when the upper bits of its operand register are not
+// zero (bytes taken from a split 32-bit or 16-bit register).
 __device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
   uint32_t out;
-  const unsigned short t = (unsigned short)(byte & 0xffu);
+  const unsigned short t = (unsigned short)byte;
   asm("{\n\t.reg .b8 lo, hi;\n\t"
       "mov.b16 {lo, hi}, %1;\n\t"
       "cvt.rn.f16x2.e2m1x2 %0, lo;\n\t}"
@@ -108,12 +92,13 @@ __device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
   return out;
 }
 
-// Eight E2M1 nibbles -> four f16x2 words (h[k] holds elements 2k, 2k+1).
+// Eight E2M1 nibbles -> four f16x2 words (h[k] holds elements 2k, 2k+1);
+// each byte is extracted zero-extended with one byte permute.
 __device__ __forceinline__ void e2m1x8_to_h2(uint32_t codes, uint32_t h[4]) {
-  h[0] = e2m1x2_to_h2(codes);
-  h[1] = e2m1x2_to_h2(codes >> 8);
-  h[2] = e2m1x2_to_h2(codes >> 16);
-  h[3] = e2m1x2_to_h2(codes >> 24);
+  h[0] = e2m1x2_to_h2(__byte_perm(codes, 0u, 0x4440u));
+  h[1] = e2m1x2_to_h2(__byte_perm(codes, 0u, 0x4441u));
+  h[2] = e2m1x2_to_h2(__byte_perm(codes, 0u, 0x4442u));
+  h[3] = e2m1x2_to_h2(__byte_perm(codes, 0u, 0x4443u));
 }
 
 __device__ __forceinline__ float h_lo(uint32_t h) {

@@ -49,7 +49,7 @@ FastDiv make_fastdiv(uint32_t d);
 cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_ws,
                         cudaStream_t st);
 cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
-                                 bool swz, cudaStream_t st);
+                                 bool swz, bool dense, cudaStream_t st);
 cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
                               bool want_row, cudaStream_t st);
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,

@@ -101,7 +101,39 @@ __global__ void __launch_bounds__(kThreads) k_amax(const QuantArgs a, uint32_t* 
 
 // --------------------------------------------------------------------------
 // K1: rowwise 1x16 NVFP4 quantizer.  grid (chunks, batch).
-template <bool F46, bool SR, bool RHT, bool SWZ>
+// Warp w of a CTA takes groups of 64 consecutive blocks; lane l owns blocks
+// g + l (pair member A) and g + 32 + l (member B), so the two ballots of the
+// 4/6 picks are directly the two 32-bit halves of the group's bitmap word.
+// DENSE: rows are contiguous (ld == cols) and the outputs are packed
+// (codes_ld == cols/2, linear scales with scales_ld == cols/16), so block j
+// sits at element 16j, code byte 8j and scale byte j; x is 32-byte aligned
+// and each block is one 256-bit load.
+template <bool DENSE>
+__device__ __forceinline__ void k1_load(const QuantArgs& a, int b, uint32_t j, bool v, uint4 (&w)[2]) {
+  if (!v) {
+    w[0] = w[1] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  if (DENSE) {
+    ld_block256(a.x + (long long)b * a.x_bs + (long long)j * 16, w);
+  } else {
+    load_block(a, b, j, w);
+  }
+}
+
+template <bool SWZ, bool DENSE>
+__device__ __forceinline__ void k1_store(const QuantArgs& a, int b, uint32_t j, const uint32_t (&codes)[2],
+                                         uint32_t scale) {
+  if (DENSE) {
+    *reinterpret_cast<uint2*>(a.row.codes + (long long)b * a.row.codes_bs + (long long)j * 8) =
+        make_uint2(codes[0], codes[1]);
+    a.row.scales[(long long)b * a.row.scales_bs + j] = (uint8_t)scale;
+  } else {
+    store_block<SWZ>(a.row, b, j, a.bpr, codes, scale);
+  }
+}
+
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
 __global__ void __launch_bounds__(kThreads, 2) k_q1x16(const QuantArgs a) {
   __shared__ float2 s_tab[128];
   const int b = blockIdx.y;
@@ -112,33 +144,27 @@ __global__ void __launch_bounds__(kThreads, 2) k_q1x16(const QuantArgs a) {
   if (RHT) mask16 = rht_sign_mask(a.seed);
   __syncthreads();
 
-  const uint32_t nunit = (a.nblk + 1) / 2;
-  const uint32_t u0 = blockIdx.x * a.units_per_cta;
-  const uint32_t u1 = min(u0 + a.units_per_cta, nunit);
   const int lane = threadIdx.x & 31;
+  const uint32_t c0 = blockIdx.x * (2 * a.units_per_cta);
+  const uint32_t c1 = min(c0 + 2 * a.units_per_cta, a.nblk);
+  constexpr uint32_t kStep = 64 * (kThreads / 32);
   uint32_t bad = 0;
 
-  // software pipeline: the next pair is loaded before this one is processed
-  uint32_t u = u0 + threadIdx.x;
+  uint32_t g = c0 + 64 * (threadIdx.x >> 5);
   uint4 na[2], nb[2];
-  if (u < u1) {
-    load_block(a, b, 2 * u, na);
-    if (2 * u + 1 < a.nblk) load_block(a, b, 2 * u + 1, nb);
-  }
-  for (uint32_t ubase = u0; ubase < u1; ubase += kThreads) {
-    const bool valid = u < u1;
-    const uint32_t j0 = 2 * u;
-    const bool has1 = valid && (j0 + 1 < a.nblk);
+  k1_load<DENSE>(a, b, g + lane, g + lane < c1, na);
+  k1_load<DENSE>(a, b, g + 32 + lane, g + 32 + lane < c1, nb);
+  for (; g < c1; g += kStep) {   // uniform over the warp
+    const uint32_t ja = g + lane, jb = g + 32 + lane;
+    const bool va = ja < c1, vb = jb < c1;
     uint4 wa[2] = {na[0], na[1]}, wb[2] = {nb[0], nb[1]};
-    if (!has1) { wb[0] = wa[0]; wb[1] = wa[1]; }
-    const uint32_t un = u + kThreads;
-    if (un < u1) {
-      load_block(a, b, 2 * un, na);
-      if (2 * un + 1 < a.nblk) load_block(a, b, 2 * un + 1, nb);
+    const uint32_t gn = g + kStep;
+    if (gn < c1) {
+      k1_load<DENSE>(a, b, gn + lane, gn + lane < c1, na);
+      k1_load<DENSE>(a, b, gn + 32 + lane, gn + 32 + lane < c1, nb);
     }
-
     uint32_t pick_a = 0, pick_b = 0;
-    if (valid) {
+    if (va) {
       if (RHT) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -170,31 +196,34 @@ __global__ void __launch_bounds__(kThreads, 2) k_q1x16(const QuantArgs a) {
         const float2 t4a = s_tab[s4a], t4b = s_tab[s4b];
         const Cand c4 = candidate<true>(P, make_float2(t4a.y, t4b.y), make_float2(-t4a.x, -t4b.x), a.neg_zero);
         pick_a = c4.err.x < c6.err.x;
-        pick_b = has1 && (c4.err.y < c6.err.y);  // no bit for a missing second block
+        pick_b = vb && (c4.err.y < c6.err.y);  // no bit for a missing block
         if (pick_a) { ca[0] = c4.ca[0]; ca[1] = c4.ca[1]; sa = s4a; inva = t4a.y; }
         if (pick_b) { cbk[0] = c4.cb[0]; cbk[1] = c4.cb[1]; sb = s4b; invb = t4b.y; }
       }
       if (SR) {
         const long long g0 = a.elem_offset + (long long)b * a.rows * a.cols;
-        const uint32_t rowa = fdiv(j0, a.bpr), cba = j0 - rowa * a.bpr.d;
-        sr_block(P, 0, inva, sr_bytes16(a.seed, g0 + (long long)rowa * a.cols + cba * 16), ca);
-        if (has1) {
-          const uint32_t rowb = fdiv(j0 + 1, a.bpr), cbb = j0 + 1 - rowb * a.bpr.d;
-          sr_block(P, 1, invb, sr_bytes16(a.seed, g0 + (long long)rowb * a.cols + cbb * 16), cbk);
+        if (DENSE) {
+          sr_block(P, 0, inva, sr_bytes16(a.seed, g0 + (long long)ja * 16), ca);
+          if (vb) sr_block(P, 1, invb, sr_bytes16(a.seed, g0 + (long long)jb * 16), cbk);
+        } else {
+          const uint32_t rowa = fdiv(ja, a.bpr), cba = ja - rowa * a.bpr.d;
+          sr_block(P, 0, inva, sr_bytes16(a.seed, g0 + (long long)rowa * a.cols + cba * 16), ca);
+          if (vb) {
+            const uint32_t rowb = fdiv(jb, a.bpr), cbb = jb - rowb * a.bpr.d;
+            sr_block(P, 1, invb, sr_bytes16(a.seed, g0 + (long long)rowb * a.cols + cbb * 16), cbk);
+          }
         }
       }
-      store_block<SWZ>(a.row, b, j0, a.bpr, ca, sa);
-      if (has1) store_block<SWZ>(a.row, b, j0 + 1, a.bpr, cbk, sb);
+      k1_store<SWZ, DENSE>(a, b, ja, ca, sa);
+      if (vb) k1_store<SWZ, DENSE>(a, b, jb, cbk, sb);
     }
     if (F46 && a.row.choice) {
       const uint32_t ba = __ballot_sync(0xffffffffu, pick_a);
       const uint32_t bb = __ballot_sync(0xffffffffu, pick_b);
-      const uint32_t uw = ubase + (threadIdx.x & ~31u);
-      if (lane == 0 && uw < u1) {
-        store_choice64(a.row, (unsigned long long)b * a.nblk + 2ull * uw, interleave_bits(ba, bb));
-      }
+      if (lane == 0)
+        store_choice64(a.row, (unsigned long long)b * a.nblk + g,
+                       (unsigned long long)ba | ((unsigned long long)bb << 32));
     }
-    u = un;
   }
   if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
@@ -308,12 +337,14 @@ cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_
 }
 
 cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
-                                 bool swz, cudaStream_t st) {
+                                 bool swz, bool dense, cudaStream_t st) {
   const uint32_t nunit = (a.nblk + 1) / 2;
   const dim3 g = grid_for(nunit, a.units_per_cta, batch);
   const bool f46 = fmt == 0;
-#define FOS_L(F, S, R, W) k_q1x16<F, S, R, W><<<g, kThreads, 0, st>>>(a)
-#define FOS_W(F, S, R) do { if (swz) FOS_L(F, S, R, true); else FOS_L(F, S, R, false); } while (0)
+  if (dense) swz = false;
+#define FOS_L(F, S, R, W, D) k_q1x16<F, S, R, W, D><<<g, kThreads, 0, st>>>(a)
+#define FOS_D(F, S, R, W) do { if (dense) FOS_L(F, S, R, W, true); else FOS_L(F, S, R, W, false); } while (0)
+#define FOS_W(F, S, R) do { if (swz) FOS_D(F, S, R, true); else FOS_D(F, S, R, false); } while (0)
 #define FOS_R(F, S) do { if (rht) FOS_W(F, S, true); else FOS_W(F, S, false); } while (0)
 #define FOS_S(F) do { if (sr) FOS_R(F, true); else FOS_R(F, false); } while (0)
   if (f46) FOS_S(true);
@@ -321,6 +352,7 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 #undef FOS_S
 #undef FOS_R
 #undef FOS_W
+#undef FOS_D
 #undef FOS_L
   return cudaGetLastError();
 }
