@@ -47,14 +47,20 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True,
+          defines=(), out: str | None = None) -> str:
+    """Compile every csrc/*.cu and link libfos.so (or `out`, with extra -D
+    `defines`, e.g. tuning constants; objects then go to a separate folder)."""
+    lib = out or LIB
+    if not force and not defines and out is None and up_to_date():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    bdir = BUILD if not defines else os.path.join(BUILD, "variant_%d" % abs(hash(tuple(defines))))
+    os.makedirs(bdir, exist_ok=True)
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    extra += ["-D" + d for d in defines]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         p = subprocess.run(cmd, capture_output=True, text=True)
         if p.returncode != 0:
@@ -67,13 +73,13 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) 
         for _, err in results:
             sys.stderr.write(err)
     objs = [o for o, _ in results]
-    tmp = LIB + ".tmp%d" % os.getpid()
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     p = subprocess.run(cmd, capture_output=True, text=True)
     if p.returncode != 0:
         raise RuntimeError("nvcc link failed:\n" + p.stderr[-8000:])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main():

@@ -20,7 +20,8 @@ FastDiv make_fastdiv(uint32_t d) {
 
 namespace {
 
-constexpr uint32_t kUnitsQuant = 256 * 4;   // block pairs per CTA (1x16 quantizer)
+constexpr uint32_t kUnitsQuant = 256 * 4;   // work units per CTA (tile kernels)
+constexpr uint32_t kBlocksRowwise = 256 * 8; // 16-element blocks per CTA (rowwise 1x16)
 constexpr uint32_t kUnitsAmax = 256 * 8;    // block pairs per CTA (amax pass)
 constexpr uint32_t kUnitsMx = 256 * 4;      // 1x32 blocks per CTA
 constexpr uint32_t kUnitsDeq = 256 * 4;     // blocks per CTA (dequantize)
@@ -213,6 +214,7 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
 
   cudaError_t ce;
   a.units_per_cta = kUnitsQuant;
+  if (opt->blk == FOS_BLOCK_1X16 && !colwise) a.units_per_cta = kBlocksRowwise;
   if (opt->blk == FOS_BLOCK_16X16) {
     ce = launch_q16x16(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr, st);
   } else if (colwise) {

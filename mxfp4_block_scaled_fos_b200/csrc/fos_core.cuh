@@ -86,11 +86,11 @@ __device__ __forceinline__ void cand_scales(float a, float St, uint32_t& s6, uin
   // r >= 0 for valid input; the 0x7f mask keeps a caller-supplied negative
   // amax from indexing past the 128-entry scale table
   if (F46) {
-    const uint32_t both = e4m3x2(div6_rn(r), __fmul_rn(r, 0.25f));
+    const uint32_t both = e4m3x2(div6_for_e4m3(r), __fmul_rn(r, 0.25f));
     s6 = (both >> 8) & 0x7fu;
     s4 = both & 0x7fu;
   } else {
-    s6 = e4m3x2(0.0f, div6_rn(r)) & 0x7fu;
+    s6 = e4m3x2(0.0f, div6_for_e4m3(r)) & 0x7fu;
     s4 = 0;
   }
 }
@@ -137,6 +137,50 @@ __device__ __forceinline__ Cand candidate(const float2 (&P)[16], float2 inv, flo
   return c;
 }
 
+// One block as 8 natural pairs P[k] = (w_2k, w_2k+1): round with one
+// candidate scale (inv, e) and, when WANT_ERR, form the same binary32 error
+// as above (d = fma(-q, e, w), t = d*d, pairwise tree over contiguous
+// elements); the first tree level adds the two halves of each pair.
+struct Cand1 {
+  uint32_t c[2];  // codes of the block
+  float err;
+};
+
+template <bool WANT_ERR>
+__device__ __forceinline__ Cand1 candidate1(const float2 (&P)[8], float inv, float nege, float nz) {
+  Cand1 r;
+  const float2 inv2 = make_float2(inv, inv);
+  float s[8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float2 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = mul2(P[4 * h + k], inv2);
+    r.c[h] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
+    if (WANT_ERR) {
+      uint32_t hq[4];
+      e2m1x8_to_h2(r.c[h], hq);
+      const float2 ne2 = make_float2(nege, nege), z2 = make_float2(nz, nz);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 q = __half22float2(as_h2(hq[k]));
+        const float2 d = fma2(q, ne2, P[4 * h + k]);
+        const float2 t = fma2(d, d, z2);   // RN(d*d), never fused into the add
+        s[4 * h + k] = __fadd_rn(t.x, t.y);
+      }
+    }
+  }
+  if (WANT_ERR) {
+    const float2 l2a = add2(make_float2(s[0], s[2]), make_float2(s[1], s[3]));
+    const float2 l2b = add2(make_float2(s[4], s[6]), make_float2(s[5], s[7]));
+    const float2 l3 = add2(make_float2(l2a.x, l2b.x), make_float2(l2a.y, l2b.y));
+    r.err = __fadd_rn(l3.x, l3.y);
+  } else {
+    r.err = 0.0f;
+  }
+  return r;
+}
+
 // Stochastic rounding of the kept candidate of one block (A: which = 0,
 // B: which = 1) with 16 Philox bytes.
 __device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float inv, uint4 rnd,
@@ -150,6 +194,44 @@ __device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float
   }
   out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
   out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+}
+
+// Stochastic rounding of one block held as 8 natural pairs.
+__device__ __forceinline__ void sr_block1(const float2 (&P)[8], float inv, uint4 rnd, uint32_t (&out)[2]) {
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float w = (i & 1) ? P[i >> 1].y : P[i >> 1].x;
+    const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
+    q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
+  }
+  out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+  out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+}
+
+// 16-point fast Walsh-Hadamard transform of one block held as natural
+// pairs: butterflies (a, b) -> (a + b, a - b) at element strides 1 (inside a
+// pair), 2, 4, 8 (between pairs), then * 0.25.
+__device__ __forceinline__ void fwht16_natural(float2 (&P)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float a = P[k].x, b = P[k].y;
+    P[k] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+#pragma unroll
+  for (int h = 1; h < 8; h *= 2) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2 * h) {
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float2 a = P[j], b = P[j + h];
+        P[j] = add2(a, b);
+        P[j + h] = sub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) P[k] = mul2(P[k], make_float2(0.25f, 0.25f));
 }
 
 // Bit i of a -> bit 2i, bit i of b -> bit 2i+1.

@@ -11,6 +11,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace fos {
 
@@ -41,10 +42,11 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
 // RN(r / 6) without a division: q0 = RN(r*y), y = RN(1/6); the remainder
 // r - 6*q0 is exact as an fma and one correction step q0 + rem*y gives the
 // correctly rounded quotient (P. Markstein, IBM J. Res. Dev. 34(1), 1990).
-// Checked against IEEE division for every binary32 r; it differs only for
-// r < 2^-125, where the quotient is subnormal, so those take a division.
-__device__ __forceinline__ float div6_rn(float r) {
-  if (!(r >= 2.35098870164457501594e-38f)) return __fdiv_rn(r, 6.0f);
+// Checked against IEEE division for every binary32 r: equal for all
+// r >= 2^-125.  Below that both results are < 2^-127, far under the
+// smallest E4M3 subnormal (2^-9), so the E4M3 code of the quotient -- the
+// only use here -- is 0 either way and no fallback branch is needed.
+__device__ __forceinline__ float div6_for_e4m3(float r) {
   const float y = 1.0f / 6.0f;
   const float q0 = __fmul_rn(r, y);
   const float rem = __fmaf_rn(-q0, 6.0f, r);
@@ -101,12 +103,14 @@ __device__ __forceinline__ void e2m1x8_to_h2(uint32_t codes, uint32_t h[4]) {
   h[3] = e2m1x2_to_h2(__byte_perm(codes, 0u, 0x4443u));
 }
 
-__device__ __forceinline__ float h_lo(uint32_t h) {
-  return __half2float(__ushort_as_half((unsigned short)(h & 0xffffu)));
+__device__ __forceinline__ __half2 as_h2(uint32_t h) {
+  __half2 r;
+  memcpy(&r, &h, 4);
+  return r;
 }
-__device__ __forceinline__ float h_hi(uint32_t h) {
-  return __half2float(__ushort_as_half((unsigned short)(h >> 16)));
-}
+// exact f16 -> f32 of the low / high half (no masking or shifting)
+__device__ __forceinline__ float h_lo(uint32_t h) { return __low2float(as_h2(h)); }
+__device__ __forceinline__ float h_hi(uint32_t h) { return __high2float(as_h2(h)); }
 
 // ---------------------------------------------------------------- E4M3
 // Two binary32 values -> (E4M3(hi) << 8) | E4M3(lo), RNE, saturating at 448.

@@ -22,6 +22,10 @@ namespace fos {
 namespace {
 
 constexpr int kThreads = 256;
+// resident CTAs per SM the rowwise quantizer is compiled for (register cap)
+#ifndef FOS_K1_MIN_BLOCKS
+#define FOS_K1_MIN_BLOCKS 4
+#endif
 
 __device__ __forceinline__ void load_block(const QuantArgs& a, int b, uint32_t j, uint4 (&w)[2]) {
   const uint32_t row = fdiv(j, a.bpr);
@@ -101,9 +105,12 @@ __global__ void __launch_bounds__(kThreads) k_amax(const QuantArgs a, uint32_t* 
 
 // --------------------------------------------------------------------------
 // K1: rowwise 1x16 NVFP4 quantizer.  grid (chunks, batch).
-// Warp w of a CTA takes groups of 64 consecutive blocks; lane l owns blocks
-// g + l (pair member A) and g + 32 + l (member B), so the two ballots of the
-// 4/6 picks are directly the two 32-bit halves of the group's bitmap word.
+// One block per thread per step: lane l of warp w takes block g + l, so a
+// warp reads 1 KB of contiguous input per step, writes 256 contiguous code
+// bytes and 32 scale bytes, and its ballot of 4/6 picks is one 32-bit word
+// of the choice bitmap.  The block is carried as 8 natural pairs
+// (w_2k, w_2k+1), the layout in which bf16 words unpack, E2M1 bytes pack and
+// decode, so every packed f32x2 operand is formed without moves.
 // DENSE: rows are contiguous (ld == cols) and the outputs are packed
 // (codes_ld == cols/2, linear scales with scales_ld == cols/16), so block j
 // sits at element 16j, code byte 8j and scale byte j; x is 32-byte aligned
@@ -133,8 +140,21 @@ __device__ __forceinline__ void k1_store(const QuantArgs& a, int b, uint32_t j, 
   }
 }
 
+__device__ __forceinline__ void store_choice32(const OutDesc& o, unsigned long long gbit, uint32_t word) {
+  unsigned int* base = reinterpret_cast<unsigned int*>(o.choice);
+  if (o.choice_aligned) {
+    base[gbit >> 5] = word;
+  } else if (word) {
+    // only words that receive a set bit are touched
+    const int sh = (int)(gbit & 31);
+    const unsigned long long vv = (unsigned long long)word << sh;
+    if ((uint32_t)vv) atomicOr(base + (gbit >> 5), (uint32_t)vv);
+    if ((uint32_t)(vv >> 32)) atomicOr(base + (gbit >> 5) + 1, (uint32_t)(vv >> 32));
+  }
+}
+
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
-__global__ void __launch_bounds__(kThreads, 2) k_q1x16(const QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS) k_q1x16(const QuantArgs a) {
   __shared__ float2 s_tab[128];
   const int b = blockIdx.y;
   const float St = tensor_scale_of(a, b, F46);
@@ -145,84 +165,68 @@ __global__ void __launch_bounds__(kThreads, 2) k_q1x16(const QuantArgs a) {
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const uint32_t c0 = blockIdx.x * (2 * a.units_per_cta);
-  const uint32_t c1 = min(c0 + 2 * a.units_per_cta, a.nblk);
-  constexpr uint32_t kStep = 64 * (kThreads / 32);
+  const uint32_t c0 = blockIdx.x * a.units_per_cta;
+  const uint32_t c1 = min(c0 + a.units_per_cta, a.nblk);
   uint32_t bad = 0;
 
-  uint32_t g = c0 + 64 * (threadIdx.x >> 5);
-  uint4 na[2], nb[2];
-  k1_load<DENSE>(a, b, g + lane, g + lane < c1, na);
-  k1_load<DENSE>(a, b, g + 32 + lane, g + 32 + lane < c1, nb);
-  for (; g < c1; g += kStep) {   // uniform over the warp
-    const uint32_t ja = g + lane, jb = g + 32 + lane;
-    const bool va = ja < c1, vb = jb < c1;
-    uint4 wa[2] = {na[0], na[1]}, wb[2] = {nb[0], nb[1]};
-    const uint32_t gn = g + kStep;
-    if (gn < c1) {
-      k1_load<DENSE>(a, b, gn + lane, gn + lane < c1, na);
-      k1_load<DENSE>(a, b, gn + 32 + lane, gn + 32 + lane < c1, nb);
-    }
-    uint32_t pick_a = 0, pick_b = 0;
-    if (va) {
+  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += kThreads) {  // uniform per warp
+    const uint32_t j = g + lane;
+    const bool valid = j < c1;
+    uint4 w[2];
+    k1_load<DENSE>(a, b, j, valid, w);
+    uint32_t pick = 0;
+    if (valid) {
       if (RHT) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint32_t xa = rht_word_mask(mask16, k), xb = rht_word_mask(mask16, k + 4);
-          (&wa[0].x)[k] ^= xa; (&wb[0].x)[k] ^= xa;
-          (&wa[1].x)[k] ^= xb; (&wb[1].x)[k] ^= xb;
+          (&w[0].x)[k] ^= rht_word_mask(mask16, k);
+          (&w[1].x)[k] ^= rht_word_mask(mask16, k + 4);
         }
       }
-      float2 P[16];
-      unpack_pairs(wa, wb, P);
-      uint32_t ma, mb;
+      const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+      float2 P[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) P[k] = make_float2(bf_lo(W[k]), bf_hi(W[k]));
+      uint32_t m;
       if (RHT) {
-        fwht16_pairs(P);
-        amax_bits_pairs(P, ma, mb);
+        fwht16_natural(P);
+        m = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
       } else {
-        ma = amax_bits_bf16(wa);
-        mb = amax_bits_bf16(wb);
+        m = amax_bits_bf16(w);
       }
-      bad |= (max(ma, mb) >= 0x7f800000u);
-      uint32_t s6a, s4a, s6b, s4b;
-      cand_scales<F46>(__uint_as_float(ma), St, s6a, s4a);
-      cand_scales<F46>(__uint_as_float(mb), St, s6b, s4b);
-      const float2 t6a = s_tab[s6a], t6b = s_tab[s6b];
-      const Cand c6 = candidate<F46>(P, make_float2(t6a.y, t6b.y), make_float2(-t6a.x, -t6b.x), a.neg_zero);
-      uint32_t ca[2] = {c6.ca[0], c6.ca[1]}, cbk[2] = {c6.cb[0], c6.cb[1]};
-      uint32_t sa = s6a, sb = s6b;
-      float inva = t6a.y, invb = t6b.y;
+      bad |= (m >= 0x7f800000u);
+      uint32_t s6, s4;
+      cand_scales<F46>(__uint_as_float(m), St, s6, s4);
+      const float2 t6 = s_tab[s6];
+      const Cand1 c6 = candidate1<F46>(P, t6.y, -t6.x, a.neg_zero);
+      uint32_t codes[2] = {c6.c[0], c6.c[1]};
+      uint32_t sc = s6;
+      float inv = t6.y;
       if (F46) {
-        const float2 t4a = s_tab[s4a], t4b = s_tab[s4b];
-        const Cand c4 = candidate<true>(P, make_float2(t4a.y, t4b.y), make_float2(-t4a.x, -t4b.x), a.neg_zero);
-        pick_a = c4.err.x < c6.err.x;
-        pick_b = vb && (c4.err.y < c6.err.y);  // no bit for a missing block
-        if (pick_a) { ca[0] = c4.ca[0]; ca[1] = c4.ca[1]; sa = s4a; inva = t4a.y; }
-        if (pick_b) { cbk[0] = c4.cb[0]; cbk[1] = c4.cb[1]; sb = s4b; invb = t4b.y; }
+        const float2 t4 = s_tab[s4];
+        const Cand1 c4 = candidate1<true>(P, t4.y, -t4.x, a.neg_zero);
+        pick = c4.err < c6.err;   // strictly lower wins; ties keep 6
+        if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.y; }
       }
       if (SR) {
         const long long g0 = a.elem_offset + (long long)b * a.rows * a.cols;
+        long long e0;
         if (DENSE) {
-          sr_block(P, 0, inva, sr_bytes16(a.seed, g0 + (long long)ja * 16), ca);
-          if (vb) sr_block(P, 1, invb, sr_bytes16(a.seed, g0 + (long long)jb * 16), cbk);
+          e0 = g0 + (long long)j * 16;
         } else {
-          const uint32_t rowa = fdiv(ja, a.bpr), cba = ja - rowa * a.bpr.d;
-          sr_block(P, 0, inva, sr_bytes16(a.seed, g0 + (long long)rowa * a.cols + cba * 16), ca);
-          if (vb) {
-            const uint32_t rowb = fdiv(jb, a.bpr), cbb = jb - rowb * a.bpr.d;
-            sr_block(P, 1, invb, sr_bytes16(a.seed, g0 + (long long)rowb * a.cols + cbb * 16), cbk);
-          }
+          const uint32_t row = fdiv(j, a.bpr), cb = j - row * a.bpr.d;
+          e0 = g0 + (long long)row * a.cols + cb * 16;
         }
+        sr_block1(P, inv, sr_bytes16(a.seed, e0), codes);
       }
-      k1_store<SWZ, DENSE>(a, b, ja, ca, sa);
-      if (vb) k1_store<SWZ, DENSE>(a, b, jb, cbk, sb);
+      k1_store<SWZ, DENSE>(a, b, j, codes, sc);
     }
     if (F46 && a.row.choice) {
-      const uint32_t ba = __ballot_sync(0xffffffffu, pick_a);
-      const uint32_t bb = __ballot_sync(0xffffffffu, pick_b);
-      if (lane == 0)
-        store_choice64(a.row, (unsigned long long)b * a.nblk + g,
-                       (unsigned long long)ba | ((unsigned long long)bb << 32));
+      const uint32_t word = __ballot_sync(0xffffffffu, pick);
+      if (lane == 0) store_choice32(a.row, (unsigned long long)b * a.nblk + g, word);
     }
   }
   if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
@@ -338,8 +342,7 @@ cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_
 
 cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
                                  bool swz, bool dense, cudaStream_t st) {
-  const uint32_t nunit = (a.nblk + 1) / 2;
-  const dim3 g = grid_for(nunit, a.units_per_cta, batch);
+  const dim3 g = grid_for(a.nblk, a.units_per_cta, batch);
   const bool f46 = fmt == 0;
   if (dense) swz = false;
 #define FOS_L(F, S, R, W, D) k_q1x16<F, S, R, W, D><<<g, kThreads, 0, st>>>(a)

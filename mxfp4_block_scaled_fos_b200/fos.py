@@ -16,7 +16,9 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libfos.so")
+# FOS_LIBRARY may point at another build of the same library (e.g. one
+# compiled with different tuning constants); default: the in-tree build.
+LIB_PATH = os.environ.get("FOS_LIBRARY") or os.path.join(_PKG, "libfos.so")
 
 FMT = {"nvfp4_46": 0, "nvfp4_6": 1, "mxfp4": 2}
 BLK = {"1x16": 0, "16x16": 1, "1x32": 2}
