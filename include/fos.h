@@ -162,6 +162,34 @@ fos_status fos_amax(const void* x, int64_t batch, int64_t rows, int64_t cols, in
 fos_status fos_dequantize(const fos_qtensor* q, int32_t fmt, int64_t batch, int64_t rows,
                           int64_t cols, uint32_t flags, void* y, int64_t ldy, void* stream);
 
+/*
+ * fos_quantize_static -- fos_quantize without a workspace argument, for
+ * callers that cannot allocate device memory: code that runs inside a stream
+ * capture (cudaMalloc cannot be captured), serving paths that must not
+ * allocate because an allocation can synchronize the device, and hosts or
+ * plugins whose memory is owned by another allocator that hands out no
+ * scratch buffers.  The paper has no counterpart; this is a deployment aid.
+ *
+ * Arguments, outputs and errors are those of fos_quantize.  The scratch
+ * memory (the per-batch-entry amax words) lives in a fixed array inside the
+ * library, sized for FOS_STATIC_MAX_BATCH batch entries; every GPU that
+ * loads the library holds it (about 33 KB) until the process exits.
+ * batch > FOS_STATIC_MAX_BATCH returns FOS_ERR_WORKSPACE.  No device memory
+ * is allocated or freed.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and keeps it; make that first call before any stream
+ * capture.  All calls share the one array: calls that overlap on the GPU
+ * (other streams, other host threads, concurrent graph launches) race and
+ * give wrong results.  Each call clears the words it uses before reading
+ * them, so the contents left by an earlier call do not matter.
+ */
+#define FOS_STATIC_MAX_BATCH 4096
+fos_status fos_quantize_static(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                               int64_t ld, const fos_options* opt, const float* amax_in,
+                               const fos_qtensor* rowwise, const fos_qtensor* colwise,
+                               uint32_t* status, void* stream);
+
 /* Bytes of workspace fos_quantize needs for this call. */
 size_t fos_workspace_size(int64_t batch, int64_t rows, int64_t cols, const fos_options* opt);
 

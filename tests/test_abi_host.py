@@ -33,7 +33,7 @@ def _declared_functions():
 def test_exports_every_declared_symbol(L):
     declared = _declared_functions()
     assert declared, "no declarations found"
-    assert declared <= set(EXPORTS) | {"fos_quantize_static"}
+    assert declared <= set(EXPORTS)
     for name in declared:
         assert hasattr(L, name), name
 
