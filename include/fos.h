@@ -171,9 +171,9 @@ fos_status fos_dequantize(const fos_qtensor* q, int32_t fmt, int64_t batch, int6
  * scratch buffers.  The paper has no counterpart; this is a deployment aid.
  *
  * Arguments, outputs and errors are those of fos_quantize.  The scratch
- * memory (the per-batch-entry amax words) lives in a fixed array inside the
+ * memory (per-batch-entry amax words and counters) lives in a fixed array in the
  * library, sized for FOS_STATIC_MAX_BATCH batch entries; every GPU that
- * loads the library holds it (about 33 KB) until the process exits.
+ * loads the library holds it (about 49 KB) until the process exits.
  * batch > FOS_STATIC_MAX_BATCH returns FOS_ERR_WORKSPACE.  No device memory
  * is allocated or freed.
  *

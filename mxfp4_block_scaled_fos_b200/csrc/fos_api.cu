@@ -30,7 +30,7 @@ inline bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0
 
 long long round_up(long long v, long long m) { return (v + m - 1) / m * m; }
 
-size_t ws_bytes(int64_t batch) { return (size_t)(8 * round_up(batch, 64) + 256); }
+size_t ws_bytes(int64_t batch) { return (size_t)(12 * round_up(batch, 64) + 256); }
 
 // Validate one output descriptor for a tensor of R rows and C columns.
 fos_status check_out(const fos_qtensor* q, int64_t R, int64_t C, int64_t bs, bool nvfp4,
@@ -183,15 +183,6 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
     return launch_mxfp4(a, (int)batch, swz, st) == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;
   }
 
-  // per-tensor amax pass, unless the caller supplies the amaxes
-  uint32_t* amax_ws = (uint32_t*)workspace;
-  if (!amax_in) {
-    if (cudaMemsetAsync(amax_ws, 0, 4 * batch, st) != cudaSuccess) return FOS_ERR_CUDA;
-    a.units_per_cta = kUnitsAmax;
-    if (launch_amax(a, (int)batch, rht, amax_ws, st) != cudaSuccess) return FOS_ERR_CUDA;
-  }
-  a.amax_ws = amax_ws;
-
   // Which choice-bit words a CTA owns outright depends on the kernel's tiling;
   // bitmaps whose words are shared between CTAs are built with atomics on a
   // zeroed buffer.
@@ -201,7 +192,6 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
     a.row.choice_aligned = (cols / 16) % 8 == 0;
     a.col.choice_aligned = (rows / 16) % 32 == 0;
   }
-
   const int64_t nb_row = opt->blk == FOS_BLOCK_16X16 ? batch * (rows / 16) * (cols / 16)
                                                      : batch * rows * (cols / 16);
   const int64_t nb_col = opt->blk == FOS_BLOCK_16X16 ? nb_row : batch * cols * (rows / 16);
@@ -212,18 +202,43 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
     if (cudaMemsetAsync(colwise->choice_bits, 0, choice_bytes(nb_col), st) != cudaSuccess)
       return FOS_ERR_CUDA;
 
+  // workspace: amax words [batch], then the fused path's per-entry counters
+  uint32_t* amax_ws = (uint32_t*)workspace;
+  uint32_t* done_ws = amax_ws + round_up(batch, 64);
+  uint32_t* claim_ws = done_ws + round_up(batch, 64);
+  a.amax_ws = amax_ws;
   cudaError_t ce;
+  const bool rowwise_1x16 = opt->blk == FOS_BLOCK_1X16 && !colwise;
+  // contiguous rows, packed outputs, 32-byte aligned input: no index
+  // arithmetic per block and one 256-bit load per block
+  const bool dense = rowwise_1x16 && ld == cols && rowwise->codes_ld * 2 == cols && !swz &&
+                     rowwise->scales_ld * 16 == cols && aligned(x, 32);
+
+  if (!amax_in && rowwise_1x16) {
+    // one persistent launch: per-entry amax and quantize, pipelined so the
+    // second read of each entry comes from L2
+    if (cudaMemsetAsync(amax_ws, 0, 12 * round_up(batch, 64), st) != cudaSuccess) return FOS_ERR_CUDA;
+    ce = launch_q1x16_fused(a, (int)batch, opt->fmt, sr, rht, swz, dense, amax_ws, done_ws, claim_ws,
+                            st);
+    if (ce == cudaSuccess) return FOS_OK;
+    if (ce != cudaErrorNotSupported) return FOS_ERR_CUDA;
+    (void)cudaGetLastError();  // fall back to the two-kernel path below
+  }
+
+  // per-tensor amax pass, unless the caller supplies the amaxes
+  if (!amax_in) {
+    if (cudaMemsetAsync(amax_ws, 0, 4 * batch, st) != cudaSuccess) return FOS_ERR_CUDA;
+    a.units_per_cta = kUnitsAmax;
+    if (launch_amax(a, (int)batch, rht, amax_ws, st) != cudaSuccess) return FOS_ERR_CUDA;
+  }
+
   a.units_per_cta = kUnitsQuant;
-  if (opt->blk == FOS_BLOCK_1X16 && !colwise) a.units_per_cta = kBlocksRowwise;
+  if (rowwise_1x16) a.units_per_cta = kBlocksRowwise;
   if (opt->blk == FOS_BLOCK_16X16) {
     ce = launch_q16x16(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr, st);
   } else if (colwise) {
     ce = launch_q1x16_dual(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, st);
   } else {
-    // contiguous rows, packed outputs, 32-byte aligned input: no index
-    // arithmetic per block and one 256-bit load per block
-    const bool dense = ld == cols && rowwise->codes_ld * 2 == cols && !swz &&
-                       rowwise->scales_ld * 16 == cols && aligned(x, 32);
     ce = launch_q1x16_rowwise(a, (int)batch, opt->fmt, sr, rht, swz, dense, st);
   }
   if (ce == cudaErrorNotSupported) return FOS_ERR_UNSUPPORTED;

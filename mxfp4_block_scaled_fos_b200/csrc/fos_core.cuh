@@ -78,11 +78,41 @@ __device__ __forceinline__ void amax_bits_pairs(const float2 (&P)[16], uint32_t&
   }
 }
 
+// The per-tensor scale with what the block-scale step needs of it.
+struct TScale {
+  float St;   // S_t
+  float y;    // RN(1 / S_t)
+  bool fast;  // S_t >= 2^-92: RN(a / S_t) may be formed without a division
+};
+
+__device__ __forceinline__ TScale make_tscale(float St) {
+  TScale t;
+  t.St = St;
+  t.fast = St >= 2.01948391736579e-28f;  // 2^-92
+  t.y = t.fast ? __frcp_rn(St) : 0.0f;
+  return t;
+}
+
+// RN(a / S_t) for a >= 0.  Fast path: q0 = RN(a*y), one fma correction
+// q0 + (a - S_t*q0)*y (P. Markstein, IBM J. Res. Dev. 34(1), 1990).  Checked
+// against IEEE division for ~20000 divisors over the whole binary32 range,
+// every positive finite bf16 dividend and random binary32 dividends: equal
+// whenever dividend and quotient are >= 2^-100.  With S_t >= 2^-92 that
+// covers every quotient r >= 2^-8; smaller quotients give E4M3(r/4) =
+// E4M3(r/6) = 0 whichever way they round, so the scale codes are exact.
+__device__ __forceinline__ float div_tscale(float a, const TScale& t) {
+  const float q0 = __fmul_rn(a, t.y);
+  const float rem = __fmaf_rn(-q0, t.St, a);
+  float r = __fmaf_rn(rem, t.y, q0);
+  if (!t.fast) r = (t.St == 0.0f) ? 0.0f : __fdiv_rn(a, t.St);  // uniform per tensor
+  return r;
+}
+
 // Candidate scale codes of a block with amax a: (s6, s4) as E4M3 bytes,
 // s6 = E4M3(RN(r/6)), s4 = E4M3(RN(r/4)), r = RN(a/S_t).
 template <bool F46>
-__device__ __forceinline__ void cand_scales(float a, float St, uint32_t& s6, uint32_t& s4) {
-  const float r = (St == 0.0f) ? 0.0f : __fdiv_rn(a, St);
+__device__ __forceinline__ void cand_scales(float a, const TScale& ts, uint32_t& s6, uint32_t& s4) {
+  const float r = div_tscale(a, ts);
   // r >= 0 for valid input; the 0x7f mask keeps a caller-supplied negative
   // amax from indexing past the 128-entry scale table
   if (F46) {

@@ -53,6 +53,27 @@ __device__ __forceinline__ float div6_for_e4m3(float r) {
   return __fmaf_rn(rem, y, q0);
 }
 
+// L2 eviction-priority policies for the loads below (createpolicy).
+__device__ __forceinline__ unsigned long long l2_policy_evict_last() {
+  unsigned long long pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ unsigned long long l2_policy_evict_first() {
+  unsigned long long pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 32 bytes (one 16-element bf16 block) in one 256-bit load with an L2
+// eviction policy; p must be 32-byte aligned.
+__device__ __forceinline__ void ld_block256_hint(const void* p, unsigned long long pol, uint4 (&w)[2]) {
+  asm("ld.global.nc.L2::cache_hint.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], %9;"
+      : "=r"(w[0].x), "=r"(w[0].y), "=r"(w[0].z), "=r"(w[0].w), "=r"(w[1].x), "=r"(w[1].y),
+        "=r"(w[1].z), "=r"(w[1].w)
+      : "l"(p), "l"(pol));
+}
+
 // 32 bytes (one 16-element bf16 block) in one 256-bit load; p must be
 // 32-byte aligned.
 __device__ __forceinline__ void ld_block256(const void* p, uint4 (&w)[2]) {

@@ -24,7 +24,7 @@ namespace {
 constexpr int kThreads = 256;
 // resident CTAs per SM the rowwise quantizer is compiled for (register cap)
 #ifndef FOS_K1_MIN_BLOCKS
-#define FOS_K1_MIN_BLOCKS 4
+#define FOS_K1_MIN_BLOCKS 5
 #endif
 
 __device__ __forceinline__ void load_block(const QuantArgs& a, int b, uint32_t j, uint4 (&w)[2]) {
@@ -115,14 +115,18 @@ __global__ void __launch_bounds__(kThreads) k_amax(const QuantArgs a, uint32_t* 
 // (codes_ld == cols/2, linear scales with scales_ld == cols/16), so block j
 // sits at element 16j, code byte 8j and scale byte j; x is 32-byte aligned
 // and each block is one 256-bit load.
+// pol != 0: L2 eviction policy for the dense 256-bit load (0: default)
 template <bool DENSE>
-__device__ __forceinline__ void k1_load(const QuantArgs& a, int b, uint32_t j, bool v, uint4 (&w)[2]) {
+__device__ __forceinline__ void k1_load(const QuantArgs& a, int b, uint32_t j, bool v, uint4 (&w)[2],
+                                        unsigned long long pol = 0) {
   if (!v) {
     w[0] = w[1] = make_uint4(0u, 0u, 0u, 0u);
     return;
   }
   if (DENSE) {
-    ld_block256(a.x + (long long)b * a.x_bs + (long long)j * 16, w);
+    const uint16_t* p = a.x + (long long)b * a.x_bs + (long long)j * 16;
+    if (pol) ld_block256_hint(p, pol, w);
+    else     ld_block256(p, w);
   } else {
     load_block(a, b, j, w);
   }
@@ -153,29 +157,22 @@ __device__ __forceinline__ void store_choice32(const OutDesc& o, unsigned long l
   }
 }
 
+// Quantize blocks [c0, c1) of batch entry b with this CTA: lane l of warp w
+// takes block g + l for g = c0 + 32w, c0 + 32w + 256, ...  c0 must be a
+// multiple of 32 so that each 32-bit word of the choice bitmap belongs to one
+// warp.
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
-__global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS) k_q1x16(const QuantArgs a) {
-  __shared__ float2 s_tab[128];
-  const int b = blockIdx.y;
-  const float St = tensor_scale_of(a, b, F46);
-  build_scale_table(s_tab, St);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[b] = St;
-  uint32_t mask16 = 0;
-  if (RHT) mask16 = rht_sign_mask(a.seed);
-  __syncthreads();
-
+__device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
+                                              const float2* s_tab, const TScale& ts, uint32_t mask16,
+                                              uint32_t& bad, unsigned long long pol = 0) {
   const int lane = threadIdx.x & 31;
-  const uint32_t c0 = blockIdx.x * a.units_per_cta;
-  const uint32_t c1 = min(c0 + a.units_per_cta, a.nblk);
-  uint32_t bad = 0;
-
   for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += kThreads) {  // uniform per warp
     const uint32_t j = g + lane;
     const bool valid = j < c1;
     uint4 w[2];
-    k1_load<DENSE>(a, b, j, valid, w);
+    k1_load<DENSE>(a, b, j, valid, w, pol);
     uint32_t pick = 0;
-    if (valid) {
+    {  // computed for every lane (a missing block reads as zeros); only stores are predicated
       if (RHT) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -199,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS) k_q1x16(const Qua
       }
       bad |= (m >= 0x7f800000u);
       uint32_t s6, s4;
-      cand_scales<F46>(__uint_as_float(m), St, s6, s4);
+      cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
       const float2 t6 = s_tab[s6];
       const Cand1 c6 = candidate1<F46>(P, t6.y, -t6.x, a.neg_zero);
       uint32_t codes[2] = {c6.c[0], c6.c[1]};
@@ -208,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS) k_q1x16(const Qua
       if (F46) {
         const float2 t4 = s_tab[s4];
         const Cand1 c4 = candidate1<true>(P, t4.y, -t4.x, a.neg_zero);
-        pick = c4.err < c6.err;   // strictly lower wins; ties keep 6
+        pick = valid && (c4.err < c6.err);   // strictly lower wins; ties keep 6
         if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.y; }
       }
       if (SR) {
@@ -222,12 +219,201 @@ __global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS) k_q1x16(const Qua
         }
         sr_block1(P, inv, sr_bytes16(a.seed, e0), codes);
       }
-      k1_store<SWZ, DENSE>(a, b, j, codes, sc);
+      if (valid) k1_store<SWZ, DENSE>(a, b, j, codes, sc);
     }
     if (F46 && a.row.choice) {
       const uint32_t word = __ballot_sync(0xffffffffu, pick);
       if (lane == 0) store_choice32(a.row, (unsigned long long)b * a.nblk + g, word);
     }
+  }
+}
+
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
+__global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS) k_q1x16(const QuantArgs a) {
+  __shared__ float2 s_tab[128];
+  const int b = blockIdx.y;
+  const float St = tensor_scale_of(a, b, F46);
+  build_scale_table(s_tab, St);
+  const TScale ts = make_tscale(St);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[b] = St;
+  uint32_t mask16 = 0;
+  if (RHT) mask16 = rht_sign_mask(a.seed);
+  __syncthreads();
+  const uint32_t c0 = blockIdx.x * a.units_per_cta;
+  const uint32_t c1 = min(c0 + a.units_per_cta, a.nblk);
+  uint32_t bad = 0;
+  rowwise_range<F46, SR, RHT, SWZ, DENSE>(a, b, c0, c1, s_tab, ts, mask16, bad);
+  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// --------------------------------------------------------------------------
+// Fused amax + rowwise quantize for a batch of tensors with one S_t each
+// (e.g. the experts of an MoE layer), as one persistent launch fed by a work
+// queue.  The queue is a fixed sequence of items: phase p holds the amax
+// chunks of entry p (if p < batch) followed by the quantize chunks of entry
+// p - L (L = min(kLag, batch)).  CTAs claim items in sequence order with one
+// atomic counter, claiming the next item while they work on the current one.
+// An amax item reduces its chunk and counts in on done_a[entry]; a quantize
+// item first waits until every amax chunk of its entry has counted in, then
+// quantizes its chunk with that entry's S_t.  Every item an item waits on
+// precedes it in the sequence and was claimed by a running CTA that never
+// waits on a later item, so the queue needs no co-residency and cannot
+// deadlock; the wait is bounded anyway (about a second, then
+// FOS_STATUS_TIMEOUT).  Memory-bound amax chunks and compute-bound quantize
+// chunks run side by side on every SM, and with the L + 1 entries in flight
+// smaller than L2 (and the amax reads marked evict-last) the quantize reads
+// hit L2, so HBM sees the input about once.
+#ifndef FOS_FUSED_LAG
+#define FOS_FUSED_LAG 2
+#endif
+constexpr int kLag = FOS_FUSED_LAG;
+#ifndef FOS_FUSED_AMAX_UNROLL
+#define FOS_FUSED_AMAX_UNROLL 4
+#endif
+constexpr uint32_t kAChunk = 4096;         // blocks per amax item
+constexpr uint32_t kQChunk = 1024;         // blocks per quantize item
+constexpr uint32_t kSpinLimit = 1u << 23;  // x ~128 ns sleep
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until *p >= target (thread 0 of the CTA calls it).
+__device__ __forceinline__ void wait_at_least(const uint32_t* p, uint32_t target, uint32_t* status) {
+  uint32_t it = 0;
+  while (ld_acquire(p) < target) {
+    if (++it > kSpinLimit) {
+      if (status) atomicOr(status, FOS_STATUS_TIMEOUT);
+      return;
+    }
+    __nanosleep(128);
+  }
+}
+
+// max |x| (of the RHT of x) over blocks [lo, hi) of entry b, U loads in
+// flight per thread.
+template <bool RHT, bool DENSE>
+__device__ __forceinline__ uint32_t slice_amax_bits(const QuantArgs& a, int b, uint32_t lo, uint32_t hi,
+                                                    uint32_t mask16, unsigned long long pol) {
+  constexpr int U = FOS_FUSED_AMAX_UNROLL;
+  uint32_t m = 0;
+  for (uint32_t j0 = lo + threadIdx.x; j0 < hi; j0 += U * kThreads) {
+    uint4 w[U][2];
+#pragma unroll
+    for (int u = 0; u < U; ++u) k1_load<DENSE>(a, b, j0 + u * kThreads, j0 + u * kThreads < hi, w[u], pol);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (RHT) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          (&w[u][0].x)[k] ^= rht_word_mask(mask16, k);
+          (&w[u][1].x)[k] ^= rht_word_mask(mask16, k + 4);
+        }
+        const uint32_t W[8] = {w[u][0].x, w[u][0].y, w[u][0].z, w[u][0].w,
+                               w[u][1].x, w[u][1].y, w[u][1].z, w[u][1].w};
+        float2 P[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) P[k] = make_float2(bf_lo(W[k]), bf_hi(W[k]));
+        fwht16_natural(P);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
+      } else {
+        m = max(m, amax_bits_bf16(w[u]));
+      }
+    }
+  }
+  return m;
+}
+
+struct FusedItem {
+  bool amax;        // amax item (else quantize item)
+  int entry;
+  uint32_t chunk;
+};
+
+// Position i of the item sequence (i < total) -> item.
+__device__ __forceinline__ FusedItem fused_item(uint32_t i, int batch, int L, uint32_t na, uint32_t nq) {
+  FusedItem it;
+  const uint32_t head = (uint32_t)L * na;                 // phases 0 .. L-1: amax only
+  const uint32_t mid = (uint32_t)(batch - L) * (na + nq);  // phases L .. batch-1: amax + quantize
+  if (i < head) {
+    it.amax = true; it.entry = (int)(i / na); it.chunk = i % na;
+  } else if (i - head < mid) {
+    const uint32_t r = (i - head) % (na + nq);
+    const int p = L + (int)((i - head) / (na + nq));
+    if (r < na) { it.amax = true; it.entry = p; it.chunk = r; }
+    else        { it.amax = false; it.entry = p - L; it.chunk = r - na; }
+  } else {                                                 // phases batch .. batch+L-1
+    const uint32_t r = i - head - mid;
+    it.amax = false; it.entry = batch - L + (int)(r / nq); it.chunk = r % nq;
+  }
+  return it;
+}
+
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
+__global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS)
+    k_q1x16_fused(const QuantArgs a, int batch, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue) {
+  __shared__ float2 s_tab[128];
+  __shared__ uint32_t s_red[kThreads / 32];
+  __shared__ float s_St;
+  __shared__ uint32_t s_item[2];
+  const uint32_t mask16 = RHT ? rht_sign_mask(a.seed) : 0u;
+  const uint32_t na = (a.nblk + kAChunk - 1) / kAChunk;
+  const uint32_t nq = (a.nblk + kQChunk - 1) / kQChunk;
+  const int L = min(kLag, batch);
+  const uint32_t total = (uint32_t)batch * (na + nq);
+  const unsigned long long pol_keep = l2_policy_evict_last();   // amax reads: keep for quantize
+  const unsigned long long pol_done = l2_policy_evict_first();  // quantize reads: last use
+  uint32_t bad = 0;
+  int tab_entry = -1;   // entry whose scale table s_tab holds
+
+  if (threadIdx.x == 0) s_item[0] = atomicAdd(queue, 1u);
+  __syncthreads();
+  for (int k = 0;; k ^= 1) {
+    const uint32_t i = s_item[k];
+    if (i >= total) break;
+    if (threadIdx.x == 0) s_item[k ^ 1] = atomicAdd(queue, 1u);  // claim the next one now
+    const FusedItem it = fused_item(i, batch, L, na, nq);
+    if (it.amax) {
+      const uint32_t lo = it.chunk * kAChunk, hi = min(lo + kAChunk, a.nblk);
+      uint32_t m = slice_amax_bits<RHT, DENSE>(a, it.entry, lo, hi, mask16, pol_keep);
+      m = __reduce_max_sync(0xffffffffu, m);
+      if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) v = max(v, s_red[w]);
+        if (v >= 0x7f800000u) {
+          if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+        } else if (v) {
+          atomicMax(amax_ws + it.entry, v);
+        }
+        __threadfence();
+        atomicAdd(done_a + it.entry, 1u);
+      }
+    } else {
+      if (it.entry != tab_entry) {
+        if (threadIdx.x == 0) {
+          wait_at_least(done_a + it.entry, na, a.status);
+          const float A = __uint_as_float(__ldcg(amax_ws + it.entry));
+          s_St = __fdiv_rn(A, F46 ? 1792.0f : 2688.0f);
+        }
+        __syncthreads();
+        build_scale_table(s_tab, s_St);
+        __syncthreads();
+        tab_entry = it.entry;
+      }
+      const float St = s_St;
+      const TScale ts = make_tscale(St);
+      if (it.chunk == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[it.entry] = St;
+      const uint32_t lo = it.chunk * kQChunk, hi = min(lo + kQChunk, a.nblk);
+      rowwise_range<F46, SR, RHT, SWZ, DENSE>(a, it.entry, lo, hi, s_tab, ts, mask16, bad, pol_done);
+    }
+    __syncthreads();  // the next item is in s_item[k ^ 1]; s_red / s_tab may be rewritten
   }
   if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
@@ -358,6 +544,41 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 #undef FOS_D
 #undef FOS_L
   return cudaGetLastError();
+}
+
+// Persistent launch of the fused kernel: one CTA per resident slot.
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
+static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_ws, uint32_t* done_a,
+                                  uint32_t* queue, cudaStream_t st) {
+  auto kern = k_q1x16_fused<F46, SR, RHT, SWZ, DENSE>;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorNotSupported;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorNotSupported;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
+      per_sm < 1)
+    return cudaErrorNotSupported;
+  kern<<<sms * per_sm, kThreads, 0, st>>>(a, batch, amax_ws, done_a, queue);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_q1x16_fused(const QuantArgs& a, int batch, int fmt, bool sr, bool rht, bool swz,
+                               bool dense, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue,
+                               cudaStream_t st) {
+  const bool f46 = fmt == 0;
+  if (dense) swz = false;
+#define FOS_L(F, S, R, W, D) return launch_fused_t<F, S, R, W, D>(a, batch, amax_ws, done_a, queue, st)
+#define FOS_D(F, S, R, W) do { if (dense) FOS_L(F, S, R, W, true); else FOS_L(F, S, R, W, false); } while (0)
+#define FOS_W(F, S, R) do { if (swz) FOS_D(F, S, R, true); else FOS_D(F, S, R, false); } while (0)
+#define FOS_R(F, S) do { if (rht) FOS_W(F, S, true); else FOS_W(F, S, false); } while (0)
+#define FOS_S(F) do { if (sr) FOS_R(F, true); else FOS_R(F, false); } while (0)
+  if (f46) FOS_S(true);
+  else     FOS_S(false);
+#undef FOS_S
+#undef FOS_R
+#undef FOS_W
+#undef FOS_D
+#undef FOS_L
 }
 
 cudaError_t launch_mxfp4(const QuantArgs& a, int batch, bool swz, cudaStream_t st) {

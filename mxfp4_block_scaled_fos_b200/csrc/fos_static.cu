@@ -16,7 +16,7 @@ namespace {
 
 constexpr int64_t kStaticMaxBatch = FOS_STATIC_MAX_BATCH;
 // the workspace fos_quantize needs for kStaticMaxBatch entries
-constexpr size_t kScratchBytes = 8 * kStaticMaxBatch + 256;
+constexpr size_t kScratchBytes = 12 * kStaticMaxBatch + 256;
 constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];

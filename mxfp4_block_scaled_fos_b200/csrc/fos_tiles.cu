@@ -99,7 +99,7 @@ struct PairResult {
 
 template <bool F46>
 __device__ __forceinline__ PairResult<F46> quant_pair(const float2 (&P)[16], uint32_t ma, uint32_t mb,
-                                                      float St, const float2* tab, float nz) {
+                                                      const TScale& St, const float2* tab, float nz) {
   PairResult<F46> r;
   uint32_t s6a, s4a, s6b, s4b;
   cand_scales<F46>(__uint_as_float(ma), St, s6a, s4a);
@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_dual1x16(const QuantArgs a) {
   const int rs0 = blockIdx.y * (kSubRows * kStrip);
   const float St = tensor_scale_of(a, b, F46);
   build_scale_table(s_tab, St);
+  const TScale ts = make_tscale(St);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
     if (a.col.tensor_scale) a.col.tensor_scale[b] = St;
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_dual1x16(const QuantArgs a) {
         unpack_pairs(wa, wb, P);
         const uint32_t ma = amax_bits_bf16(wa), mb = amax_bits_bf16(wb);
         bad |= max(ma, mb) >= 0x7f800000u;
-        PairResult<F46> q = quant_pair<F46>(P, ma, mb, St, s_tab, a.neg_zero);
+        PairResult<F46> q = quant_pair<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
         if (SR) {
           sr_block(P, 0, q.inva, s_rnd[rr * 8 + 2 * pp], q.ca);
           sr_block(P, 1, q.invb, s_rnd[rr * 8 + 2 * pp + 1], q.cb);
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_dual1x16(const QuantArgs a) {
         }
         const uint32_t ma = (m & 0xffffu) << 16, mb = m & 0xffff0000u;
         bad |= max(ma, mb) >= 0x7f800000u;
-        PairResult<F46> q = quant_pair<F46>(P, ma, mb, St, s_tab, a.neg_zero);
+        PairResult<F46> q = quant_pair<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
         if (SR) {
           uint32_t ba[16], bb[16];
           const uint8_t* rb = reinterpret_cast<const uint8_t*>(s_rnd);
@@ -325,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_2d16x16(const QuantArgs a) {
   const int rs0 = blockIdx.y * (kSubRows * kStrip);
   const float St = tensor_scale_of(a, b, F46);
   build_scale_table(s_tab, St);
+  const TScale ts = make_tscale(St);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
     if (COL && a.col.tensor_scale) a.col.tensor_scale[b] = St;
@@ -369,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_2d16x16(const QuantArgs a) {
       m = max(m, __shfl_xor_sync(gmask, m, 4));
       bad |= m >= 0x7f800000u;
       uint32_t s6, s4;
-      cand_scales<F46>(__uint_as_float(m), St, s6, s4);
+      cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
       const float2 t6 = s_tab[s6];
       const Cand c6 = candidate<F46>(P, make_float2(t6.y, t6.y), make_float2(-t6.x, -t6.x), a.neg_zero);
       uint32_t ca[2] = {c6.ca[0], c6.ca[1]}, cb[2] = {c6.cb[0], c6.cb[1]};

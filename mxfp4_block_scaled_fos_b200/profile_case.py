@@ -7,6 +7,7 @@ a reduced batch so a capture stays small), runs one untimed call, then
 `iters` calls of the kernel of interest on the current stream.  Cases:
 
   moe46     4/6 NVFP4 1x16 rowwise on expert weights, amax supplied (k_q1x16)
+  moe46_full  the same with the per-expert amax computed in the call (k_q1x16_fused)
   moe6      6-only NVFP4 1x16 rowwise, amax supplied
   moe_amax  the per-expert amax pass (k_amax)
   moe_mx    MXFP4 1x32 (k_mxfp4)
@@ -37,7 +38,11 @@ def main():
     if c.startswith("moe"):
         x = workloads.moe_experts(args.experts, 2880, 2880, device=dev)
         amax = F.amax(x)
-        if c == "moe46":
+        if c == "moe46_full":
+            ws = torch.empty(F.workspace_size(args.experts, 2880, 2880), dtype=torch.uint8, device=dev)
+            out = F.quantize(x, workspace=ws)[0]
+            fn = lambda: F.quantize(x, out_row=out, workspace=ws)
+        elif c == "moe46":
             out = F.quantize(x, amax=amax)[0]
             fn = lambda: F.quantize(x, amax=amax, out_row=out)
         elif c == "moe6":
