@@ -5,8 +5,8 @@
 
 One step = one pass of the quantizer over the MoE expert workload
 (128 x 2880 x 2880 bf16, per-expert N(0, 0.02^2) times U(0.5, 2)): the
-per-expert amax pass and the 4/6 quantize to packed E2M1 codes + E4M3 scales +
-FP32 per-expert scales.  value = bytes / time with bytes = 2 (bf16 in) + 0.5
+per-expert amax and the 4/6 quantize to packed E2M1 codes + E4M3 scales +
+FP32 per-expert scales, which the library runs as one fused kernel launch.  value = bytes / time with bytes = 2 (bf16 in) + 0.5
 (codes) + 1/16 (scales) per element, summed over ranks (weak scaling: every
 rank quantizes its own 128 experts).  Under torchrun one process per GPU;
 rank 0 prints one JSON line.
@@ -155,6 +155,41 @@ def time_loop(fn, steps, warmup, world, stream):
     return max_over_ranks(e0.elapsed_time(e1), world)
 
 
+# ------------------------------------------------------------------ ncu traffic
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "k_q1x16_fused_moe_experts.md")
+
+
+def source_hash() -> str:
+    """SHA-256 over the CUDA sources, to tell whether a profile is current."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mxfp4_block_scaled_fos_b200", "csrc")
+    for fn in sorted(glob.glob(os.path.join(csrc, "*"))):
+        with open(fn, "rb") as f:
+            h.update(os.path.basename(fn).encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(elems):
+    """DRAM bytes per launch of the fused kernel from the committed ncu
+    summary (scaled from its capture to `elems`), or None if the sources
+    changed since the capture."""
+    try:
+        kv = {}
+        with open(PROFILE_SUMMARY) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("source_sha256") != source_hash():
+            return None
+        per_elem = float(kv["dram_bytes_per_element"])
+        return int(per_elem * elems)
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # ------------------------------------------------------------------ CPU baseline
 def cpu_baseline(x_cpu_bits, budget_s=12.0):
     """Time the oracle (single thread) on whole experts until ~budget_s."""
@@ -187,11 +222,10 @@ def run_fos(args, world, rank):
     E, R, C = 128, 2880, 2880
     x = workloads.moe_experts(E, R, C, device=dev, seed=rank)
     elems = x.numel()
-    flags = 0
     row = F.quantize(x)[0]  # allocate outputs once
     ws = torch.empty(F.workspace_size(E, R, C), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    launches_per_step = 2  # amax pass + quantize
+    launches_per_step = 1  # the fused amax + quantize kernel (plus a 1.5 KB memset)
 
     def step():
         F.quantize(x, out_row=row, workspace=ws, status=status)
@@ -202,17 +236,16 @@ def run_fos(args, world, rank):
     t_ms = time_loop(step, args.steps, args.warmup, world, stream)
     clk.stop()
 
-    # roofline of the dominant kernel: the quantize kernel alone (amax given)
-    amax = F.amax(x)
-
-    def q_only():
-        F.quantize(x, out_row=row, amax=amax, status=status)
-
-    k_steps = max(args.steps, 20)
-    tq_ms = time_loop(q_only, k_steps, 3, world, stream) / k_steps
-    ta_ms = time_loop(lambda: F.amax(x, out=amax), k_steps, 3, world, stream) / k_steps
+    # the step's only kernel is the fused one: its duration is the step time
+    ms_per_step = t_ms / args.steps
     peak, peak_kind = measured_peaks()
-    achieved = elems * BYTES_PER_ELEM / (tq_ms * 1e-3) / 1e9
+    achieved = elems * BYTES_PER_ELEM / (ms_per_step * 1e-3) / 1e9
+    # context: the quantize kernel alone with the amaxes supplied, and the amax pass
+    amax = F.amax(x)
+    k_steps = max(args.steps, 20)
+    tq_ms = time_loop(lambda: F.quantize(x, out_row=row, amax=amax, status=status), k_steps, 3,
+                      world, stream) / k_steps
+    ta_ms = time_loop(lambda: F.amax(x, out=amax), k_steps, 3, world, stream) / k_steps
 
     extra = {}
     if not args.no_modes:
@@ -222,7 +255,6 @@ def run_fos(args, world, rank):
     e2e = measure_e2e(args, world, x, row, ws, status, stream)
     assert int(status.item()) == 0, "non-finite input reported"
 
-    ms_per_step = t_ms / args.steps
     value = world * elems * BYTES_PER_ELEM / (ms_per_step * 1e-3) / 1e9
     clocks = clk.summary()
     out = {
@@ -237,10 +269,15 @@ def run_fos(args, world, rank):
                    "amax": "computed in-step (per expert)", "parallelism": "dp%d" % world,
                    "l2": "input %.2f GB > 126 MB L2; no flush needed" % (2 * elems / 1e9)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
-                     "kernel": "k_q1x16 (4/6, RNE, amax supplied)",
-                     "kernel_ms": round(tq_ms, 4), "amax_kernel_ms": round(ta_ms, 4),
-                     "peak_source": "%s hbm_gbs (burst copy)" % peak_kind},
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(elems),
+                     "kernel": "k_q1x16_fused<4/6, RNE> (per-expert amax + quantize)",
+                     "kernel_ms": round(ms_per_step, 4),
+                     "bytes_per_launch": int(elems * BYTES_PER_ELEM),
+                     "quantize_only_ms": round(tq_ms, 4),
+                     "quantize_only_GB_s": round(elems * BYTES_PER_ELEM / (tq_ms * 1e-3) / 1e9, 1),
+                     "amax_pass_ms": round(ta_ms, 4),
+                     "peak_source": "%s hbm_gbs (copy, read+write)" % peak_kind},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": e2e,
         "clocks": clocks,
@@ -253,7 +290,10 @@ def run_fos(args, world, rank):
 
 
 def measure_modes(args, world, x, dev, stream, peak):
-    """Other modes of the hot path at their workloads (context, not the headline)."""
+    """Every other mode of the hot path at its workload (context, not the
+    headline).  Full steps include the amax pass; "kernel" lines give the
+    quantize kernel alone with the amax supplied.  Inputs that fit in L2 are
+    rotated over copies whose total exceeds L2."""
     import mxfp4_block_scaled_fos_b200 as F
     from mxfp4_block_scaled_fos_b200 import workloads
     res = {}
@@ -267,14 +307,27 @@ def measure_modes(args, world, x, dev, stream, peak):
         if note:
             res[name]["note"] = note
 
+    def rotating(xs, fn, reps):
+        it = [0]
+
+        def f():
+            i = it[0] % len(xs)
+            it[0] += 1
+            fn(i)
+        return time_loop(f, reps * len(xs), len(xs), world, stream) / (reps * len(xs))
+
+    # MoE experts: 6-only, MXFP4 and the dequantizers
     try:
+        ws = torch.empty(F.workspace_size(x.shape[0], x.shape[1], x.shape[2]), dtype=torch.uint8, device=dev)
         r6 = F.quantize(x, fmt="nvfp4_6")[0]
+        ms = time_loop(lambda: F.quantize(x, fmt="nvfp4_6", out_row=r6, workspace=ws), n, 3, world, stream) / n
+        rec("moe_nvfp4_6only_step", ms, BYTES_PER_ELEM, elems, "per-expert amax in the step (fused)")
         a6 = F.amax(x)
         ms = time_loop(lambda: F.quantize(x, fmt="nvfp4_6", out_row=r6, amax=a6), n, 3, world, stream) / n
-        rec("moe_nvfp4_6only_quant", ms, BYTES_PER_ELEM, elems, "amax supplied")
+        rec("moe_nvfp4_6only_kernel", ms, BYTES_PER_ELEM, elems, "amax supplied")
         rm = F.quantize(x, fmt="mxfp4")[0]
         ms = time_loop(lambda: F.quantize(x, fmt="mxfp4", out_row=rm), n, 3, world, stream) / n
-        rec("moe_mxfp4_quant", ms, BYTES_PER_ELEM_MX, elems)
+        rec("moe_mxfp4_step", ms, BYTES_PER_ELEM_MX, elems)
         r46 = F.quantize(x)[0]
         y = torch.empty_like(x)
         ms = time_loop(lambda: F.dequantize(r46, out=y), n, 3, world, stream) / n
@@ -284,22 +337,54 @@ def measure_modes(args, world, x, dev, stream, peak):
         del y, r6, rm, r46
     except Exception as e:  # report, do not hide
         res["moe_error"] = repr(e)
-    # activation-like 8192x4096 with RHT16: rotate 4 copies (256 MiB > L2)
+    torch.cuda.empty_cache()
+    # activations 8192x4096, 1% outlier channels, RHT16, 4/6: 4 rotating copies (256 MiB)
     try:
         xs = [workloads.activation_outliers(8192, 4096, device=dev, seed=s) for s in range(4)]
         outs = [F.quantize(t, rht=True)[0] for t in xs]
+        wss = [torch.empty(F.workspace_size(1, 8192, 4096), dtype=torch.uint8, device=dev) for _ in xs]
+        ms = rotating(xs, lambda i: F.quantize(xs[i], rht=True, out_row=outs[i], workspace=wss[i]), n)
+        rec("activation_rht16_step", ms, BYTES_PER_ELEM, xs[0].numel(), "amax in the step; 4 rotating copies")
         am = [F.amax(t, rht=True) for t in xs]
-        it = [0]
-
-        def f():
-            i = it[0] % 4
-            it[0] += 1
-            F.quantize(xs[i], rht=True, out_row=outs[i], amax=am[i])
-        ms = time_loop(f, 4 * n, 4, world, stream) / (4 * n)
-        rec("activation_rht16_quant", ms, BYTES_PER_ELEM, xs[0].numel(), "amax supplied; 4 rotating copies")
-        del xs, outs
+        ms = rotating(xs, lambda i: F.quantize(xs[i], rht=True, out_row=outs[i], amax=am[i]), n)
+        rec("activation_rht16_kernel", ms, BYTES_PER_ELEM, xs[0].numel(), "amax supplied; 4 rotating copies")
+        del xs, outs, am
     except Exception as e:
         res["activation_error"] = repr(e)
+    torch.cuda.empty_cache()
+    # weights 14336x4096 N(0, 0.02^2), 16x16 2D 4/6 with the transposed copy: 2 rotating copies
+    try:
+        xs = [workloads.weight_normal(14336, 4096, device=dev, seed=s) for s in range(2)]
+        outs = [F.quantize(t, block="16x16", colwise=True) for t in xs]
+        ms = rotating(xs, lambda i: F.quantize(xs[i], block="16x16", colwise=True, out_row=outs[i][0],
+                                               out_col=outs[i][1]), n)
+        rec("weight_2d_both_step", ms, BYTES_PER_ELEM_DUAL, xs[0].numel(), "amax in the step; 2 rotating copies")
+        am = [F.amax(t) for t in xs]
+        ms = rotating(xs, lambda i: F.quantize(xs[i], block="16x16", colwise=True, amax=am[i],
+                                               out_row=outs[i][0], out_col=outs[i][1]), n)
+        rec("weight_2d_both_kernel", ms, BYTES_PER_ELEM_DUAL, xs[0].numel(), "amax supplied")
+        del xs, outs, am
+    except Exception as e:
+        res["weight_error"] = repr(e)
+    torch.cuda.empty_cache()
+    # gradients 16384x8192 Student-t(3)*1e-3, SR, rowwise + colwise (256 MiB > L2)
+    try:
+        g = workloads.gradient_student_t(16384, 8192, device=dev)
+        r, c = F.quantize(g, rounding="sr", colwise=True)
+        ms = time_loop(lambda: F.quantize(g, rounding="sr", colwise=True, out_row=r, out_col=c), n, 3,
+                       world, stream) / n
+        rec("gradient_sr_dual_step", ms, BYTES_PER_ELEM_DUAL, g.numel(), "amax in the step")
+        am = F.amax(g)
+        ms = time_loop(lambda: F.quantize(g, rounding="sr", colwise=True, amax=am, out_row=r, out_col=c),
+                       n, 3, world, stream) / n
+        rec("gradient_sr_dual_kernel", ms, BYTES_PER_ELEM_DUAL, g.numel(), "amax supplied")
+        r1 = F.quantize(g, rounding="sr")[0]
+        ms = time_loop(lambda: F.quantize(g, rounding="sr", amax=am, out_row=r1), n, 3, world, stream) / n
+        rec("gradient_sr_rowwise_kernel", ms, BYTES_PER_ELEM, g.numel(), "amax supplied")
+        del g, r, c, r1
+    except Exception as e:
+        res["gradient_error"] = repr(e)
+    torch.cuda.empty_cache()
     return res
 
 

@@ -202,7 +202,8 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
     if (cudaMemsetAsync(colwise->choice_bits, 0, choice_bytes(nb_col), st) != cudaSuccess)
       return FOS_ERR_CUDA;
 
-  // workspace: amax words [batch], then the fused path's per-entry counters
+  // workspace: amax words [batch], then the fused path's per-entry counts
+  // [batch] and its queue counter
   uint32_t* amax_ws = (uint32_t*)workspace;
   uint32_t* done_ws = amax_ws + round_up(batch, 64);
   uint32_t* claim_ws = done_ws + round_up(batch, 64);

@@ -51,7 +51,8 @@ cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_
 cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
                                  bool swz, bool dense, cudaStream_t st);
 // fused per-entry amax + rowwise quantize (one persistent launch fed by a
-// work queue); returns cudaErrorNotSupported when it cannot be launched
+// work queue); amax_ws, done_a: one zeroed word per batch entry, queue: one
+// zeroed counter.  Returns cudaErrorNotSupported when it cannot be launched.
 cudaError_t launch_q1x16_fused(const QuantArgs& a, int batch, int fmt, bool sr, bool rht, bool swz,
                                bool dense, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue,
                                cudaStream_t st);

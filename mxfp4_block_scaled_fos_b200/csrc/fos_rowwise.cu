@@ -26,6 +26,10 @@ constexpr int kThreads = 256;
 #ifndef FOS_K1_MIN_BLOCKS
 #define FOS_K1_MIN_BLOCKS 5
 #endif
+// the same for the stochastic-rounding and Hadamard variants (more registers)
+#ifndef FOS_K1_MIN_BLOCKS_HEAVY
+#define FOS_K1_MIN_BLOCKS_HEAVY 4
+#endif
 
 __device__ __forceinline__ void load_block(const QuantArgs& a, int b, uint32_t j, uint4 (&w)[2]) {
   const uint32_t row = fdiv(j, a.bpr);
@@ -229,7 +233,8 @@ __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_
 }
 
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
-__global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS) k_q1x16(const QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_K1_MIN_BLOCKS)
+    k_q1x16(const QuantArgs a) {
   __shared__ float2 s_tab[128];
   const int b = blockIdx.y;
   const float St = tensor_scale_of(a, b, F46);
