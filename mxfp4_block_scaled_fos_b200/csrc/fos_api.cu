@@ -210,10 +210,12 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
   a.amax_ws = amax_ws;
   cudaError_t ce;
   const bool rowwise_1x16 = opt->blk == FOS_BLOCK_1X16 && !colwise;
-  // contiguous rows, packed outputs, 32-byte aligned input: no index
-  // arithmetic per block and one 256-bit load per block
+  // contiguous rows, packed outputs, 32-byte aligned input and choice-bitmap
+  // words owned by one warp each: no index arithmetic per block and one
+  // 256-bit load per block
   const bool dense = rowwise_1x16 && ld == cols && rowwise->codes_ld * 2 == cols && !swz &&
-                     rowwise->scales_ld * 16 == cols && aligned(x, 32);
+                     rowwise->scales_ld * 16 == cols && aligned(x, 32) &&
+                     (!rowwise->choice_bits || a.row.choice_aligned);
 
   if (!amax_in && rowwise_1x16) {
     // one persistent launch: per-entry amax and quantize, pipelined so the

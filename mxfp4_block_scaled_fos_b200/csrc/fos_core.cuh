@@ -55,15 +55,19 @@ __device__ __forceinline__ void unpack_pairs(const uint4 (&wa)[2], const uint4 (
   }
 }
 
+// max(|a|, |b|) of each bf16 half (the result's sign is the XOR of the
+// operands' signs); a NaN operand gives a NaN.
+__device__ __forceinline__ uint32_t hmax_abs2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // max |x| of 8 bf16x2 words, as binary32 bits (NaN/Inf give >= 0x7f800000).
 __device__ __forceinline__ uint32_t amax_bits_bf16(const uint4 (&w)[2]) {
-  uint32_t m = __vmaxu2(w[0].x & 0x7fff7fffu, w[0].y & 0x7fff7fffu);
-  m = __vmaxu2(m, w[0].z & 0x7fff7fffu);
-  m = __vmaxu2(m, w[0].w & 0x7fff7fffu);
-  m = __vmaxu2(m, w[1].x & 0x7fff7fffu);
-  m = __vmaxu2(m, w[1].y & 0x7fff7fffu);
-  m = __vmaxu2(m, w[1].z & 0x7fff7fffu);
-  m = __vmaxu2(m, w[1].w & 0x7fff7fffu);
+  uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(w[0].x, w[0].y), hmax_abs2(w[0].z, w[0].w)),
+                         hmax_abs2(hmax_abs2(w[1].x, w[1].y), hmax_abs2(w[1].z, w[1].w)));
+  m &= 0x7fff7fffu;
   return max(m & 0xffffu, m >> 16) << 16;
 }
 
@@ -108,11 +112,21 @@ __device__ __forceinline__ float div_tscale(float a, const TScale& t) {
   return r;
 }
 
+// The same with the path chosen at compile time (FAST: t.fast is known true).
+template <bool FAST>
+__device__ __forceinline__ float div_tscale_t(float a, const TScale& t) {
+  if (FAST) {
+    const float q0 = __fmul_rn(a, t.y);
+    return __fmaf_rn(__fmaf_rn(-q0, t.St, a), t.y, q0);
+  }
+  return (t.St == 0.0f) ? 0.0f : __fdiv_rn(a, t.St);
+}
+
 // Candidate scale codes of a block with amax a: (s6, s4) as E4M3 bytes,
 // s6 = E4M3(RN(r/6)), s4 = E4M3(RN(r/4)), r = RN(a/S_t).
-template <bool F46>
+template <bool F46, int FAST = -1>
 __device__ __forceinline__ void cand_scales(float a, const TScale& ts, uint32_t& s6, uint32_t& s4) {
-  const float r = div_tscale(a, ts);
+  const float r = FAST < 0 ? div_tscale(a, ts) : div_tscale_t<(FAST > 0)>(a, ts);
   // r >= 0 for valid input; the 0x7f mask keeps a caller-supplied negative
   // amax from indexing past the 128-entry scale table
   if (F46) {
@@ -167,43 +181,53 @@ __device__ __forceinline__ Cand candidate(const float2 (&P)[16], float2 inv, flo
   return c;
 }
 
-// One block as 8 natural pairs P[k] = (w_2k, w_2k+1): round with one
+// One block as 8 split pairs P[k] = (w_k, w_k+8): the two halves of the
+// block side by side, so that every level of the contiguous error tree but
+// the last adds neighbouring pairs with one f32x2 add.  Round with one
 // candidate scale (inv, e) and, when WANT_ERR, form the same binary32 error
 // as above (d = fma(-q, e, w), t = d*d, pairwise tree over contiguous
-// elements); the first tree level adds the two halves of each pair.
+// elements).  Codes: word 0 holds elements 0..7, word 1 elements 8..15.
 struct Cand1 {
   uint32_t c[2];  // codes of the block
   float err;
 };
 
+// Unpack the 8 bf16x2 words of a block (element 2k in the low half of word
+// k) into split pairs.
+__device__ __forceinline__ void unpack_split(const uint32_t (&W)[8], float2 (&P)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    P[k] = (k & 1) ? make_float2(bf_hi(W[k >> 1]), bf_hi(W[4 + (k >> 1)]))
+                   : make_float2(bf_lo(W[k >> 1]), bf_lo(W[4 + (k >> 1)]));
+}
+
 template <bool WANT_ERR>
 __device__ __forceinline__ Cand1 candidate1(const float2 (&P)[8], float inv, float nege, float nz) {
   Cand1 r;
   const float2 inv2 = make_float2(inv, inv);
-  float s[8];
+  float2 v[8];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float2 v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = mul2(P[4 * h + k], inv2);
-    r.c[h] = e2m1x8(v[0].x, v[0].y, v[1].x, v[1].y, v[2].x, v[2].y, v[3].x, v[3].y);
-    if (WANT_ERR) {
-      uint32_t hq[4];
-      e2m1x8_to_h2(r.c[h], hq);
-      const float2 ne2 = make_float2(nege, nege), z2 = make_float2(nz, nz);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 q = __half22float2(as_h2(hq[k]));
-        const float2 d = fma2(q, ne2, P[4 * h + k]);
-        const float2 t = fma2(d, d, z2);   // RN(d*d), never fused into the add
-        s[4 * h + k] = __fadd_rn(t.x, t.y);
-      }
-    }
-  }
+  for (int k = 0; k < 8; ++k) v[k] = mul2(P[k], inv2);
+  r.c[0] = e2m1x8(v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x);
+  r.c[1] = e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y);
   if (WANT_ERR) {
-    const float2 l2a = add2(make_float2(s[0], s[2]), make_float2(s[1], s[3]));
-    const float2 l2b = add2(make_float2(s[4], s[6]), make_float2(s[5], s[7]));
-    const float2 l3 = add2(make_float2(l2a.x, l2b.x), make_float2(l2a.y, l2b.y));
+    uint32_t ha[4], hb[4];
+    e2m1x8_to_h2(r.c[0], ha);
+    e2m1x8_to_h2(r.c[1], hb);
+    const float2 ne2 = make_float2(nege, nege), z2 = make_float2(nz, nz);
+    float2 t[8];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float2 q0 = make_float2(h_lo(ha[m]), h_lo(hb[m]));   // elements 2m, 2m+8
+      const float2 q1 = make_float2(h_hi(ha[m]), h_hi(hb[m]));   // elements 2m+1, 2m+9
+      const float2 d0 = fma2(q0, ne2, P[2 * m]);
+      const float2 d1 = fma2(q1, ne2, P[2 * m + 1]);
+      t[2 * m] = fma2(d0, d0, z2);       // RN(d*d), never fused into the adds
+      t[2 * m + 1] = fma2(d1, d1, z2);
+    }
+    const float2 l1a = add2(t[0], t[1]), l1b = add2(t[2], t[3]);
+    const float2 l1c = add2(t[4], t[5]), l1d = add2(t[6], t[7]);
+    const float2 l3 = add2(add2(l1a, l1b), add2(l1c, l1d));   // (sum 0..7, sum 8..15)
     r.err = __fadd_rn(l3.x, l3.y);
   } else {
     r.err = 0.0f;
@@ -226,12 +250,12 @@ __device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float
   out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
 }
 
-// Stochastic rounding of one block held as 8 natural pairs.
+// Stochastic rounding of one block held as 8 split pairs.
 __device__ __forceinline__ void sr_block1(const float2 (&P)[8], float inv, uint4 rnd, uint32_t (&out)[2]) {
   float q[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float w = (i & 1) ? P[i >> 1].y : P[i >> 1].x;
+    const float w = (i < 8) ? P[i].x : P[i - 8].y;
     const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
     q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
   }
@@ -239,15 +263,10 @@ __device__ __forceinline__ void sr_block1(const float2 (&P)[8], float inv, uint4
   out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
 }
 
-// 16-point fast Walsh-Hadamard transform of one block held as natural
-// pairs: butterflies (a, b) -> (a + b, a - b) at element strides 1 (inside a
-// pair), 2, 4, 8 (between pairs), then * 0.25.
-__device__ __forceinline__ void fwht16_natural(float2 (&P)[8]) {
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float a = P[k].x, b = P[k].y;
-    P[k] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-  }
+// 16-point fast Walsh-Hadamard transform of one block held as split pairs:
+// butterflies (a, b) -> (a + b, a - b) at element strides 1, 2, 4 (between
+// pairs, both halves at once), then 8 (inside a pair), then * 0.25.
+__device__ __forceinline__ void fwht16_split(float2 (&P)[8]) {
 #pragma unroll
   for (int h = 1; h < 8; h *= 2) {
 #pragma unroll
@@ -259,6 +278,11 @@ __device__ __forceinline__ void fwht16_natural(float2 (&P)[8]) {
         P[j + h] = sub2(a, b);
       }
     }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float a = P[k].x, b = P[k].y;
+    P[k] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) P[k] = mul2(P[k], make_float2(0.25f, 0.25f));

@@ -65,6 +65,14 @@ __device__ __forceinline__ unsigned long long l2_policy_evict_first() {
   return pol;
 }
 
+// Asynchronous prefetch of [p, p + bytes) into L2 with an eviction policy
+// (p and bytes multiples of 16).  No completion tracking: later loads of the
+// range hit L2 or merge with the requests in flight.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes, unsigned long long pol) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;"
+               :: "l"(p), "r"(bytes), "l"(pol) : "memory");
+}
+
 // 32 bytes (one 16-element bf16 block) in one 256-bit load with an L2
 // eviction policy; p must be 32-byte aligned.
 __device__ __forceinline__ void ld_block256_hint(const void* p, unsigned long long pol, uint4 (&w)[2]) {

@@ -8,13 +8,12 @@
 // Options from the "Four Over Six" usage section: random Hadamard transform
 // and stochastic rounding.
 //
-// Design: each thread owns two neighbouring 16-element blocks and carries
-// them as 16 packed pairs (element i of block A, element i of block B), so
-// every binary32 step of both blocks -- scaling, the error fma, squaring and
-// the whole pairwise error tree -- is one sm_100 f32x2 instruction.  Loads are
-// 4 x 128-bit per thread with the next pair prefetched; codes leave as 8-byte
-// stores (a warp writes 512 contiguous bytes), the 4/6 choice bits as one
-// 64-bit word per warp.
+// Design: one 16-element block per thread per step, loaded with one 256-bit
+// load and carried as 8 packed f32x2 pairs, so that the scaling, the error
+// fma, the squares and the error tree of a block run as sm_100 f32x2
+// instructions.  A warp covers 32 consecutive blocks: 1 KB of contiguous
+// input, 256 contiguous code bytes, 32 scale bytes and one 32-bit word of the
+// 4/6 choice bitmap (a ballot).
 #include "fos_core.cuh"
 
 namespace fos {
@@ -112,9 +111,10 @@ __global__ void __launch_bounds__(kThreads) k_amax(const QuantArgs a, uint32_t* 
 // One block per thread per step: lane l of warp w takes block g + l, so a
 // warp reads 1 KB of contiguous input per step, writes 256 contiguous code
 // bytes and 32 scale bytes, and its ballot of 4/6 picks is one 32-bit word
-// of the choice bitmap.  The block is carried as 8 natural pairs
-// (w_2k, w_2k+1), the layout in which bf16 words unpack, E2M1 bytes pack and
-// decode, so every packed f32x2 operand is formed without moves.
+// of the choice bitmap.  The block is carried as 8 split pairs
+// (w_k, w_k+8): bf16 words unpack into them, E2M1 codes pack and decode from
+// them without moves, and the contiguous error tree adds neighbouring pairs
+// with f32x2 adds down to its last level.
 // DENSE: rows are contiguous (ld == cols) and the outputs are packed
 // (codes_ld == cols/2, linear scales with scales_ld == cols/16), so block j
 // sits at element 16j, code byte 8j and scale byte j; x is 32-byte aligned
@@ -161,6 +161,92 @@ __device__ __forceinline__ void store_choice32(const OutDesc& o, unsigned long l
   }
 }
 
+// The per-block 4/6 step of the rowwise quantizer: w (8 bf16x2 words of one
+// block) -> codes, scale byte, 4-picked flag.  FAST: the tensor scale's
+// division shortcut applies (known at compile time).
+template <bool F46, bool SR, bool RHT, int FAST>
+__device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float2* s_tab, const TScale& ts,
+                                              uint32_t mask16, float nz, unsigned long long seed,
+                                              long long e0, uint32_t& bad, uint32_t (&codes)[2],
+                                              uint32_t& sc, bool& pick) {
+  if (RHT) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      (&w[0].x)[k] ^= rht_word_mask(mask16, k);
+      (&w[1].x)[k] ^= rht_word_mask(mask16, k + 4);
+    }
+  }
+  const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+  float2 P[8];
+  unpack_split(W, P);
+  uint32_t m;
+  if (RHT) {
+    fwht16_split(P);
+    m = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
+  } else {
+    m = amax_bits_bf16(w);
+  }
+  bad |= (m >= 0x7f800000u);
+  uint32_t s6, s4;
+  cand_scales<F46, FAST>(__uint_as_float(m), ts, s6, s4);
+  const float2 t6 = s_tab[s6];
+  const Cand1 c6 = candidate1<F46>(P, t6.y, -t6.x, nz);
+  codes[0] = c6.c[0];
+  codes[1] = c6.c[1];
+  sc = s6;
+  float inv = t6.y;
+  pick = false;
+  if (F46) {
+    const float2 t4 = s_tab[s4];
+    const Cand1 c4 = candidate1<true>(P, t4.y, -t4.x, nz);
+    pick = c4.err < c6.err;   // strictly lower wins; ties keep 6
+    if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.y; }
+  }
+  if (SR) sr_block1(P, inv, sr_bytes16(seed, e0), codes);
+}
+
+// Dense rows (see k1_load): blocks [c0, c1) of entry b with per-entry base
+// pointers, a branch-free tail (a lane past c1 recomputes block c1 - 1 and
+// stores nothing) and, when choice bits are asked for, a choice bitmap whose
+// words belong to one warp each (blocks per entry % 64 == 0, c0 % 32 == 0).
+template <bool F46, bool SR, bool RHT, int FAST>
+__device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
+                                              const float2* s_tab, const TScale& ts, uint32_t mask16,
+                                              uint32_t& bad, unsigned long long pol) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint16_t* xb = a.x + (long long)b * a.x_bs;
+  uint8_t* cb = a.row.codes + (long long)b * a.row.codes_bs;
+  uint8_t* sb = a.row.scales + (long long)b * a.row.scales_bs;
+  uint32_t* chw = a.row.choice
+                      ? reinterpret_cast<uint32_t*>(a.row.choice) + (((unsigned long long)b * a.nblk) >> 5)
+                      : nullptr;
+  const long long g0 = SR ? a.elem_offset + (long long)b * a.x_bs : 0;
+  const float nz = a.neg_zero;
+  const unsigned long long seed = a.seed;
+  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += kThreads) {  // uniform per warp
+    const uint32_t j = g + lane;
+    const bool valid = j < c1;
+    const uint32_t jj = valid ? j : c1 - 1;
+    uint4 w[2];
+    ld_block256_hint(xb + (size_t)jj * 16, pol, w);
+    uint32_t codes[2], sc;
+    bool pick;
+    rowwise_block<F46, SR, RHT, FAST>(w, s_tab, ts, mask16, nz, seed, g0 + (long long)jj * 16, bad,
+                                      codes, sc, pick);
+    if (valid) {
+      *reinterpret_cast<uint2*>(cb + (size_t)j * 8) = make_uint2(codes[0], codes[1]);
+      sb[j] = (uint8_t)sc;
+    }
+    if (F46 && chw) {
+      const uint32_t word = __ballot_sync(0xffffffffu, pick && valid);
+      if (lane == 0) chw[g >> 5] = word;
+    }
+  }
+}
+
 // Quantize blocks [c0, c1) of batch entry b with this CTA: lane l of warp w
 // takes block g + l for g = c0 + 32w, c0 + 32w + 256, ...  c0 must be a
 // multiple of 32 so that each 32-bit word of the choice bitmap belongs to one
@@ -168,7 +254,12 @@ __device__ __forceinline__ void store_choice32(const OutDesc& o, unsigned long l
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
 __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
                                               const float2* s_tab, const TScale& ts, uint32_t mask16,
-                                              uint32_t& bad, unsigned long long pol = 0) {
+                                              uint32_t& bad, unsigned long long pol) {
+  if (DENSE) {
+    if (ts.fast) rowwise_dense<F46, SR, RHT, 1>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    else         rowwise_dense<F46, SR, RHT, 0>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    return;
+  }
   const int lane = threadIdx.x & 31;
   for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += kThreads) {  // uniform per warp
     const uint32_t j = g + lane;
@@ -186,11 +277,10 @@ __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_
       }
       const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
       float2 P[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) P[k] = make_float2(bf_lo(W[k]), bf_hi(W[k]));
+      unpack_split(W, P);
       uint32_t m;
       if (RHT) {
-        fwht16_natural(P);
+        fwht16_split(P);
         m = 0;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
@@ -246,8 +336,15 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
   __syncthreads();
   const uint32_t c0 = blockIdx.x * a.units_per_cta;
   const uint32_t c1 = min(c0 + a.units_per_cta, a.nblk);
+  if (DENSE && threadIdx.x < 32) {   // the CTA's input into L2 up front (bulk prefetch)
+    const uint32_t nbytes = (c1 - c0) * 32u, off = threadIdx.x * 16384u;
+    if (off < nbytes)
+      prefetch_l2(a.x + (long long)b * a.x_bs + (long long)c0 * 16 + off / 2, min(16384u, nbytes - off),
+                  l2_policy_evict_first());
+  }
   uint32_t bad = 0;
-  rowwise_range<F46, SR, RHT, SWZ, DENSE>(a, b, c0, c1, s_tab, ts, mask16, bad);
+  rowwise_range<F46, SR, RHT, SWZ, DENSE>(a, b, c0, c1, s_tab, ts, mask16, bad,
+                                          DENSE ? l2_policy_evict_first() : 0ull);
   if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
@@ -275,8 +372,14 @@ constexpr int kLag = FOS_FUSED_LAG;
 #ifndef FOS_FUSED_AMAX_UNROLL
 #define FOS_FUSED_AMAX_UNROLL 4
 #endif
-constexpr uint32_t kAChunk = 4096;         // blocks per amax item
-constexpr uint32_t kQChunk = 1024;         // blocks per quantize item
+#ifndef FOS_FUSED_ACHUNK
+#define FOS_FUSED_ACHUNK 4096
+#endif
+#ifndef FOS_FUSED_QCHUNK
+#define FOS_FUSED_QCHUNK 1024
+#endif
+constexpr uint32_t kAChunk = FOS_FUSED_ACHUNK;  // blocks per amax item
+constexpr uint32_t kQChunk = FOS_FUSED_QCHUNK;  // blocks per quantize item (multiple of 32)
 constexpr uint32_t kSpinLimit = 1u << 23;  // x ~128 ns sleep
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
@@ -319,9 +422,8 @@ __device__ __forceinline__ uint32_t slice_amax_bits(const QuantArgs& a, int b, u
         const uint32_t W[8] = {w[u][0].x, w[u][0].y, w[u][0].z, w[u][0].w,
                                w[u][1].x, w[u][1].y, w[u][1].z, w[u][1].w};
         float2 P[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) P[k] = make_float2(bf_lo(W[k]), bf_hi(W[k]));
-        fwht16_natural(P);
+        unpack_split(W, P);
+        fwht16_split(P);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
@@ -359,7 +461,7 @@ __device__ __forceinline__ FusedItem fused_item(uint32_t i, int batch, int L, ui
 }
 
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
-__global__ void __launch_bounds__(kThreads, FOS_K1_MIN_BLOCKS)
+__global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_K1_MIN_BLOCKS)
     k_q1x16_fused(const QuantArgs a, int batch, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue) {
   __shared__ float2 s_tab[128];
   __shared__ uint32_t s_red[kThreads / 32];
