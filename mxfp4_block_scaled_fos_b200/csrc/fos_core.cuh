@@ -243,7 +243,7 @@ __device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float w = which ? P[i].y : P[i].x;
-    const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
+    const float m = sr_e2m1_mag_bits(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
     q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
   }
   out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);

@@ -211,6 +211,29 @@ __device__ __forceinline__ float sr_e2m1_mag(float v, uint32_t byte) {
   return (thr < __fmul_rn(512.0f, p)) ? __fadd_rn(lo, step) : lo;
 }
 
+// The same rule in integer form on the bits of v, cheaper where the bytes
+// arrive one per register (the dual-orientation quantizer).  For v >= 1 the
+// grid holds two points per binade (mantissa 1.0 and 1.5), so lo keeps v's
+// bits down to mantissa bit 22, hi = lo + 2^22 (as bits), and 512*p =
+// (bits & 0x3fffff) / 2^13: round up iff (2*byte+1) << 13 < (bits &
+// 0x3fffff).  For 0.5 <= v < 1 the binade holds one point (0.5) and the next
+// is 1.0: the same with 23 mantissa bits.  For v < 0.5: lo = 0, hi = 0.5,
+// 512*p = 1024*v (exact).  Returns the chosen grid value, or a value >= 6
+// that the saturating E2M1 encode turns into 6.  Checked on the CPU against
+// sr_e2m1_mag for every binary32 v in [0, 16) and infinity with 12 bytes,
+// and for a stride of v with all 256 bytes: identical after saturation.
+__device__ __forceinline__ float sr_e2m1_mag_bits(float v, uint32_t byte) {
+  const uint32_t bits = __float_as_uint(v);
+  const uint32_t t13 = (byte << 14) | 0x2000u;   // (2*byte + 1) << 13
+  const bool ge1 = bits >= 0x3F800000u;
+  const uint32_t fmask = ge1 ? 0x3FFFFFu : 0x7FFFFFu;
+  const uint32_t thr = ge1 ? t13 : (t13 << 1);
+  const uint32_t qn = (bits & ~fmask) + (((bits & fmask) > thr) ? fmask + 1u : 0u);
+  const float tf = __fsub_rn(__uint_as_float(0x4B000000u | (2u * byte + 1u)), 8388608.0f);
+  const uint32_t qs = (__fmul_rn(v, 1024.0f) > tf) ? 0x3F000000u : 0u;
+  return __uint_as_float(bits >= 0x3F000000u ? qn : qs);
+}
+
 // ---------------------------------------------------------------- indexing
 // Division by a runtime constant d >= 1 for numerators n < 2^31:
 // n / d = (umulhi(n, m) + n) >> s.

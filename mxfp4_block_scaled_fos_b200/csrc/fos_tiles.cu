@@ -23,6 +23,12 @@ constexpr int kThreads = 256;
 constexpr int kSubRows = 64;
 constexpr int kSubCols = 128;
 constexpr int kStrip = 8;  // sub-tiles per CTA strip (512 rows)
+#ifndef FOS_DUAL_MIN_BLOCKS
+#define FOS_DUAL_MIN_BLOCKS 2
+#endif
+#ifndef FOS_2D_MIN_BLOCKS
+#define FOS_2D_MIN_BLOCKS 3
+#endif
 
 struct TileGeom {
   int rows, cols;     // tensor
@@ -80,7 +86,7 @@ __device__ __forceinline__ void sr_block_bytes(const float2 (&P)[16], int which,
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float w = which ? P[i].y : P[i].x;
-    const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), bytes[i]);
+    const float m = sr_e2m1_mag_bits(__fmul_rn(fabsf(w), inv), bytes[i]);
     q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
   }
   out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
@@ -122,7 +128,7 @@ __device__ __forceinline__ PairResult<F46> quant_pair(const float2 (&P)[16], uin
 // --------------------------------------------------------------------------
 // 1x16 rowwise + colwise.  grid (ceil(cols/128), ceil(rows/512), batch).
 template <bool F46, bool SR, bool SWZ, bool ROW>
-__global__ void __launch_bounds__(kThreads, 2) k_dual1x16(const QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, FOS_DUAL_MIN_BLOCKS) k_dual1x16(const QuantArgs a) {
   __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
   __shared__ __align__(16) uint4 s_rnd[SR ? kSubRows * 8 : 1];
   __shared__ float2 s_tab[128];
@@ -215,12 +221,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_dual1x16(const QuantArgs a) {
           w[i] = *reinterpret_cast<const uint32_t*>(s_tile + chunk_off<0>(r, cq >> 2) + (cq & 3) * 4);
         }
         float2 P[16];
-        uint32_t m = 0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          P[i] = make_float2(bf_lo(w[i]), bf_hi(w[i]));
-          m = __vmaxu2(m, w[i] & 0x7fff7fffu);
-        }
+        for (int i = 0; i < 16; ++i) P[i] = make_float2(bf_lo(w[i]), bf_hi(w[i]));
+        uint32_t h[8];   // max |x| of both columns: a tree of packed bf16 maxima
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = hmax_abs2(w[2 * i], w[2 * i + 1]);
+        const uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(h[0], h[1]), hmax_abs2(h[2], h[3])),
+                                     hmax_abs2(hmax_abs2(h[4], h[5]), hmax_abs2(h[6], h[7]))) &
+                           0x7fff7fffu;
         const uint32_t ma = (m & 0xffffu) << 16, mb = m & 0xffff0000u;
         bad |= max(ma, mb) >= 0x7f800000u;
         PairResult<F46> q = quant_pair<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
@@ -315,7 +323,7 @@ __device__ __forceinline__ unsigned long long zip_nibbles(uint32_t a, uint32_t b
 // and the tree over the 16 row sums is a horizontal add plus three
 // xor-shuffles.
 template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
-__global__ void __launch_bounds__(kThreads, 2) k_2d16x16(const QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, FOS_2D_MIN_BLOCKS) k_2d16x16(const QuantArgs a) {
   __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
   __shared__ __align__(16) uint8_t s_tc[COL ? kSubCols * 32 : 16];
   __shared__ float2 s_tab[128];
