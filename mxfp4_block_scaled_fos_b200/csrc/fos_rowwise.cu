@@ -212,7 +212,7 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float2* s_tab
 // pointers, a branch-free tail (a lane past c1 recomputes block c1 - 1 and
 // stores nothing) and, when choice bits are asked for, a choice bitmap whose
 // words belong to one warp each (blocks per entry % 64 == 0, c0 % 32 == 0).
-template <bool F46, bool SR, bool RHT, int FAST>
+template <bool F46, bool SR, bool RHT, int FAST, int NT = kThreads>
 __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
                                               const float2* s_tab, const TScale& ts, uint32_t mask16,
                                               uint32_t& bad, unsigned long long pol) {
@@ -226,7 +226,7 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
   const long long g0 = SR ? a.elem_offset + (long long)b * a.x_bs : 0;
   const float nz = a.neg_zero;
   const unsigned long long seed = a.seed;
-  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += kThreads) {  // uniform per warp
+  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += NT) {  // uniform per warp
     const uint32_t j = g + lane;
     const bool valid = j < c1;
     const uint32_t jj = valid ? j : c1 - 1;
@@ -251,17 +251,17 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
 // takes block g + l for g = c0 + 32w, c0 + 32w + 256, ...  c0 must be a
 // multiple of 32 so that each 32-bit word of the choice bitmap belongs to one
 // warp.
-template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, int NT = kThreads>
 __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
                                               const float2* s_tab, const TScale& ts, uint32_t mask16,
                                               uint32_t& bad, unsigned long long pol) {
   if (DENSE) {
-    if (ts.fast) rowwise_dense<F46, SR, RHT, 1>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
-    else         rowwise_dense<F46, SR, RHT, 0>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    if (ts.fast) rowwise_dense<F46, SR, RHT, 1, NT>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    else         rowwise_dense<F46, SR, RHT, 0, NT>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
     return;
   }
   const int lane = threadIdx.x & 31;
-  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += kThreads) {  // uniform per warp
+  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += NT) {  // uniform per warp
     const uint32_t j = g + lane;
     const bool valid = j < c1;
     uint4 w[2];

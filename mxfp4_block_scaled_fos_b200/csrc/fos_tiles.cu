@@ -323,7 +323,7 @@ __device__ __forceinline__ unsigned long long zip_nibbles(uint32_t a, uint32_t b
 // and the tree over the 16 row sums is a horizontal add plus three
 // xor-shuffles.
 template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
-__global__ void __launch_bounds__(kThreads, FOS_2D_MIN_BLOCKS) k_2d16x16(const QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x16(const QuantArgs a) {
   __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
   __shared__ __align__(16) uint8_t s_tc[COL ? kSubCols * 32 : 16];
   __shared__ float2 s_tab[128];
