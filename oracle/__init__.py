@@ -41,14 +41,23 @@ class Opts(ctypes.Structure):
     ]
 
 
-def build(force: bool = False) -> str:
-    """Compile fos_oracle.c into liboracle.so (gcc, binary32, no contraction)."""
-    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+def build(force: bool = False, mutant: int | None = None) -> str:
+    """Compile fos_oracle.c into liboracle.so (gcc, binary32, no contraction).
+
+    mutant k > 0 (default: the FOS_ORACLE_MUTANT environment variable, only
+    set by tests/test_oracle_mutants.py) builds liboracle_m<k>.so with one
+    planted mistake instead, to show that the pins catch it.
+    """
+    if mutant is None:
+        mutant = int(os.environ.get("FOS_ORACLE_MUTANT", "0") or 0)
+    path = _LIB if not mutant else os.path.join(_HERE, "liboracle_m%d.so" % mutant)
+    stale = (not os.path.exists(path)) or os.path.getmtime(path) < os.path.getmtime(_SRC)
     if force or stale:
-        tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+        tmp = path + ".tmp%d" % os.getpid()
+        extra = ["-DOR_MUTANT=%d" % mutant] if mutant else []
+        subprocess.check_call(["gcc", *CFLAGS, *extra, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, path)
+    return path
 
 
 def lib():

@@ -50,6 +50,14 @@
 
 #define OR_VERSION 1
 
+/* Mutation hooks for tests/test_oracle_mutants.py.  Building with
+ * -DOR_MUTANT=k plants one plausible mistake (listed in that test); the pins
+ * of tests/test_oracle_pins.py must catch every one of them.  The oracle the
+ * other tests use is built without the macro and has none. */
+#ifndef OR_MUTANT
+#define OR_MUTANT 0
+#endif
+
 enum { OR_FMT_NVFP4_46 = 0, OR_FMT_NVFP4_6 = 1, OR_FMT_MXFP4 = 2 };
 enum { OR_BLK_1X16 = 0, OR_BLK_16X16 = 1, OR_BLK_1X32 = 2 };
 enum { OR_RND_RNE = 0, OR_RND_SR = 1 };
@@ -85,7 +93,7 @@ uint16_t or_f32_to_bf16(float f) {
   uint32_t lower = u & 0xFFFF0000u;   /* truncated candidate */
   uint32_t rest = u & 0x0000FFFFu;    /* discarded bits */
   uint32_t keep = lower >> 16;
-  if (rest > 0x8000u || (rest == 0x8000u && (keep & 1u))) keep += 1; /* up */
+  if (rest > 0x8000u || (rest == 0x8000u && (OR_MUTANT == 17 || (keep & 1u)))) keep += 1; /* up */
   return (uint16_t)keep;
 }
 
@@ -112,7 +120,7 @@ static int e2m1_mag_rne(double m) {
   double bd = fabs(m - E2M1_GRID[0]);
   for (int c = 1; c < 8; c++) {
     double d = fabs(m - E2M1_GRID[c]);
-    if (d < bd || (d == bd && (c & 1) == 0)) {
+    if (d < bd || (d == bd && (OR_MUTANT == 3 || (c & 1) == 0))) {
       best = c;
       bd = d;
     }
@@ -148,7 +156,8 @@ uint8_t or_e4m3_encode(float v) {
     double bd = m; /* distance to code 0 (= 0.0) */
     for (int c = 1; c <= 0x7E; c++) {
       double d = fabs(m - (double)or_e4m3_decode((uint8_t)c));
-      if (d < bd || (d == bd && (c & 1) == 0)) {
+      if ((OR_MUTANT == 6) ? ((double)or_e4m3_decode((uint8_t)c) <= m)
+                          : (d < bd || (d == bd && (c & 1) == 0))) {
         best = c;
         bd = d;
       }
@@ -167,7 +176,7 @@ int or_e8m0_exponent(float a) {
   if (a == 0.0f) return -127;
   int ex;
   (void)frexp((double)a, &ex); /* a = f * 2^ex, f in [0.5, 1): exact */
-  int e = (ex - 1) - 2;        /* floor(log2 a) = ex - 1 */
+  int e = (ex - 1) - (OR_MUTANT == 9 ? 1 : 2); /* floor(log2 a) = ex - 1 */
   if (e < -127) e = -127;
   if (e > 127) e = 127;
   return e;
@@ -191,7 +200,7 @@ void or_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2],
   uint32_t k[2] = {key_in[0], key_in[1]};
   for (int round = 0; round < 10; round++) {
     if (round > 0) {
-      k[0] += 0x9E3779B9u;
+      k[0] += (OR_MUTANT == 16) ? 0x9E3779B8u : 0x9E3779B9u;
       k[1] += 0xBB67AE85u;
     }
     uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)c[0];
@@ -217,9 +226,10 @@ static uint8_t sr_byte(uint64_t seed, int64_t g) {
   uint32_t key[2], out[4];
   seed_key(seed, key);
   uint64_t ug = (uint64_t)g;
-  uint32_t ctr[4] = {(uint32_t)((ug >> 4) & 0xFFFFFFFFu), (uint32_t)(ug >> 36), 0u, 0u};
+  uint32_t ctr[4] = {(uint32_t)((ug >> (OR_MUTANT == 18 ? 0 : 4)) & 0xFFFFFFFFu), (uint32_t)(ug >> 36),
+                     0u, 0u};
   or_philox4x32_10(ctr, key, out);
-  int j = (int)(ug & 15);
+  int j = (int)((ug + (OR_MUTANT == 11)) & 15);
   return (uint8_t)((out[j >> 2] >> (8 * (j & 3))) & 0xFFu);
 }
 
@@ -233,7 +243,7 @@ uint32_t or_rht16_signs(uint64_t seed) {
   uint32_t key[2], out[4], ctr[4] = {0u, 0u, 1u, 0u};
   seed_key(seed, key);
   or_philox4x32_10(ctr, key, out);
-  return out[0] & 0xFFFFu;
+  return out[OR_MUTANT == 7 ? 1 : 0] & 0xFFFFu;
 }
 
 void or_rht16(float x[16], uint32_t sign_mask) {
@@ -258,7 +268,7 @@ void or_rht16(float x[16], uint32_t sign_mask) {
  * max near 6". */
 float or_tensor_scale(float amax, int fmt) {
   if (fmt == OR_FMT_NVFP4_6) return amax / 2688.0f;
-  return amax / 1792.0f;
+  return amax / (OR_MUTANT == 2 ? 2688.0f : 1792.0f);
 }
 
 /* R4: the two candidate scale codes of a block with amax a. */
@@ -270,7 +280,7 @@ static void candidate_scales(float a, float S_t, int fmt, uint8_t* s6, uint8_t* 
   }
   float r = a / S_t;
   *s6 = or_e4m3_encode(r / 6.0f);
-  *s4 = (fmt == OR_FMT_NVFP4_46) ? or_e4m3_encode(r / 4.0f) : 0;
+  *s4 = (fmt == OR_FMT_NVFP4_46) ? or_e4m3_encode(r / (OR_MUTANT == 15 ? 3.0f : 4.0f)) : 0;
 }
 
 /* R5: effective scale e = float(s) * S_t and its inverse; a zero e gives a
@@ -307,8 +317,8 @@ static void candidate_rne(const float* w, int n, uint8_t s, float S_t,
     codes[i] = (uint8_t)(mag | (signbit(w[i]) ? 8 : 0));
     float q = (float)E2M1_GRID[mag];
     float sq = signbit(w[i]) ? -q : q;
-    float d = fmaf(-sq, e, w[i]);
-    t[i] = d * d;
+    float d = fmaf((OR_MUTANT == 5) ? sq : -sq, e, w[i]);
+    t[i] = (OR_MUTANT == 4 && i == n - 1) ? 0.0f : d * d;
   }
 }
 
@@ -321,7 +331,7 @@ static int e2m1_mag_sr(float v, uint8_t byte) {
   float glo = (float)E2M1_GRID[lo], ghi = (float)E2M1_GRID[lo + 1];
   float p = (v - glo) / (ghi - glo);           /* exact */
   float thresh = (float)(2 * (int)byte + 1);   /* exact */
-  return (thresh < 512.0f * p) ? lo + 1 : lo;  /* exact compare */
+  return ((OR_MUTANT == 8) ? (thresh <= 512.0f * p) : (thresh < 512.0f * p)) ? lo + 1 : lo; /* exact */
 }
 
 /* ------------------------------------------------------------------ */
@@ -360,7 +370,7 @@ static uint8_t nvfp4_block(const float* w, const int64_t* g, int n, float S_t,
       for (int r = 0; r < 16; r++) rs[r] = tree_sum(t4 + 16 * r, 16);
       err4 = tree_sum(rs, 16);
     }
-    choose4 = err4 < err6; /* R7: strictly lower wins, ties go to 6 */
+    choose4 = (OR_MUTANT == 1) ? (err4 <= err6) : (err4 < err6); /* R7: strictly lower wins */
   }
   uint8_t s = choose4 ? s4 : s6;
   const uint8_t* cc = choose4 ? c4 : c6;
@@ -581,7 +591,7 @@ int or_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tens
           out = (float)ldexp((double)sq, (int)s - 127);
         } else {
           float p = sq * or_e4m3_decode(s);
-          out = p * tensor_scale[b];
+          out = p * (OR_MUTANT == 10 ? 1.0f : tensor_scale[b]);
         }
         y[idx] = or_f32_to_bf16(out);
       }

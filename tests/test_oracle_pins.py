@@ -526,6 +526,21 @@ def test_stochastic_rounding_properties():
     assert np.all(np.abs(mean - vv) <= step / 512 + 1e-12)
 
 
+def test_stochastic_rounding_threshold_is_strict():
+    """Over the 256 bytes, SR rounds v up for exactly the bytes with
+    2*byte+1 < 512*p (R16).  At p = k/512 with k odd the threshold itself is
+    hit by one byte, which must round down: (k-1)/2 of the bytes go up, not
+    (k+1)/2.  At p = k/512 with k even, k/2 go up."""
+    bytes_ = np.arange(256, dtype=np.uint8)
+    for lo, step in ((0.0, 0.5), (0.5, 0.5), (1.0, 0.5), (2.0, 1.0), (4.0, 2.0)):
+        for k in (1, 2, 3, 255, 256, 257, 510, 511):
+            v = np.float32(lo + step * k / 512.0)   # exact in binary32
+            m = oracle.e2m1_sr(np.full(256, v, np.float32), bytes_)
+            up = int(np.sum(E2M1[m] > lo))
+            want = (k - 1) // 2 if k % 2 else k // 2
+            assert up == want, (lo, k, up, want)
+
+
 def test_sr_tensor_unbiased_and_deterministic():
     rng = np.random.default_rng(21)
     x = _random_tensor(rng, 16, 64, "normal")
