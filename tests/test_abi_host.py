@@ -92,3 +92,23 @@ def test_library_has_no_oracle_dependency():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "oracle" not in txt.lower(), fn
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without libfos.so the binding raises: there is no CPU fallback."""
+    import subprocess
+    import sys
+    code = ("import torch, mxfp4_block_scaled_fos_b200 as F\n"
+            "try:\n"
+            "    F.quantize(torch.zeros(1, 16, 16, dtype=torch.bfloat16))\n"
+            "except (RuntimeError, TypeError) as e:\n"
+            "    print('raised', type(e).__name__)\n"
+            "try:\n"
+            "    F.lib()\n"
+            "except RuntimeError as e:\n"
+            "    print('raised', 'missing' in str(e))\n")
+    env = dict(os.environ, FOS_LIBRARY=str(tmp_path / "no_such_libfos.so"))
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split("\n")[:2] == ["raised TypeError", "raised True"], r.stdout
