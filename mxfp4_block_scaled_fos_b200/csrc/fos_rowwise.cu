@@ -14,6 +14,8 @@
 // instructions.  A warp covers 32 consecutive blocks: 1 KB of contiguous
 // input, 256 contiguous code bytes, 32 scale bytes and one 32-bit word of the
 // 4/6 choice bitmap (a ballot).
+#include <atomic>
+
 #include "fos_core.cuh"
 
 namespace fos {
@@ -653,19 +655,29 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
   return cudaGetLastError();
 }
 
-// Persistent launch of the fused kernel: one CTA per resident slot.
+// Persistent launch of the fused kernel: one CTA per resident slot.  The
+// grid (SMs x resident CTAs) is looked up once per device and kernel variant
+// and cached; 0 = not yet known, -1 = the kernel cannot be resident.
+static constexpr int kMaxDevices = 64;
+
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
 static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_ws, uint32_t* done_a,
                                   uint32_t* queue, cudaStream_t st) {
+  static std::atomic<int> grid_of[kMaxDevices];
   auto kern = k_q1x16_fused<F46, SR, RHT, SWZ, DENSE>;
-  int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorNotSupported;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return cudaErrorNotSupported;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
-      per_sm < 1)
-    return cudaErrorNotSupported;
-  kern<<<sms * per_sm, kThreads, 0, st>>>(a, batch, amax_ws, done_a, queue);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
+  int grid = grid_of[dev].load(std::memory_order_relaxed);
+  if (grid == 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess)
+      return cudaErrorNotSupported;
+    grid = per_sm >= 1 ? sms * per_sm : -1;
+    grid_of[dev].store(grid, std::memory_order_relaxed);
+  }
+  if (grid < 1) return cudaErrorNotSupported;
+  kern<<<grid, kThreads, 0, st>>>(a, batch, amax_ws, done_a, queue);
   return cudaGetLastError();
 }
 
