@@ -262,9 +262,10 @@ def run_fos(args, world, rank):
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16->e2m1+e4m3 (f32 arithmetic)", "data": "synthetic",
+        "dtype": "f32", "data": "synthetic",
         "frac_of_hbm": round(value / world / peak, 4),
         "config": {"workload": WORKLOAD, "batch": E, "rows": R, "cols": C,
+                   "formats": "bf16 in; E2M1 codes, E4M3 block scales, f32 tensor scales out",
                    "elements_per_gpu": elems, "bytes_per_elem": BYTES_PER_ELEM,
                    "amax": "computed in-step (per expert)", "parallelism": "dp%d" % world,
                    "l2": "input %.2f GB > 126 MB L2; no flush needed" % (2 * elems / 1e9)},
@@ -438,7 +439,7 @@ def run_reference(args, world, rank):
             "(bf16 in, FP4+E4M3 out)", "value": round(v, 6), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (CPU)", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": "1 of 128 experts per step"},
             "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "kind": "oracle", "cores": 1,
                              "sample": sample},
