@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 // (e.g. the experts of an MoE layer), as one persistent launch fed by a work
 // queue.  The queue is a fixed sequence of items: phase p holds the amax
 // chunks of entry p (if p < batch) followed by the quantize chunks of entry
-// p - L (L = min(kLag, batch)).  CTAs claim items in sequence order with one
+// p - L (L = min(lag, batch)).  CTAs claim items in sequence order with one
 // atomic counter, claiming the next item while they work on the current one.
 // An amax item reduces its chunk and counts in on done_a[entry]; a quantize
 // item first waits until every amax chunk of its entry has counted in, then
@@ -367,10 +367,15 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 // chunks run side by side on every SM, and with the L + 1 entries in flight
 // smaller than L2 (and the amax reads marked evict-last) the quantize reads
 // hit L2, so HBM sees the input about once.
-#ifndef FOS_FUSED_LAG
-#define FOS_FUSED_LAG 2
+// Lag in entries between an entry's amax and its quantize items, and the
+// quantize item size: measured best on the 128 x 2880 x 2880 expert batch
+// (4/6: 1536 blocks, lag 3; 6-only: 1536 blocks, lag 2).
+#ifndef FOS_FUSED_LAG_46
+#define FOS_FUSED_LAG_46 3
 #endif
-constexpr int kLag = FOS_FUSED_LAG;
+#ifndef FOS_FUSED_LAG_6
+#define FOS_FUSED_LAG_6 2
+#endif
 #ifndef FOS_FUSED_AMAX_UNROLL
 #define FOS_FUSED_AMAX_UNROLL 4
 #endif
@@ -378,7 +383,7 @@ constexpr int kLag = FOS_FUSED_LAG;
 #define FOS_FUSED_ACHUNK 4096
 #endif
 #ifndef FOS_FUSED_QCHUNK
-#define FOS_FUSED_QCHUNK 1024
+#define FOS_FUSED_QCHUNK 1536
 #endif
 constexpr uint32_t kAChunk = FOS_FUSED_ACHUNK;  // blocks per amax item
 constexpr uint32_t kQChunk = FOS_FUSED_QCHUNK;  // blocks per quantize item (multiple of 32)
@@ -472,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
   const uint32_t mask16 = RHT ? rht_sign_mask(a.seed) : 0u;
   const uint32_t na = (a.nblk + kAChunk - 1) / kAChunk;
   const uint32_t nq = (a.nblk + kQChunk - 1) / kQChunk;
-  const int L = min(kLag, batch);
+  const int L = min(F46 ? FOS_FUSED_LAG_46 : FOS_FUSED_LAG_6, batch);
   const uint32_t total = (uint32_t)batch * (na + nq);
   const unsigned long long pol_keep = l2_policy_evict_last();   // amax reads: keep for quantize
   const unsigned long long pol_done = l2_policy_evict_first();  // quantize reads: last use
