@@ -95,7 +95,9 @@ typedef struct fos_options {
  *   scales uint8: linear layout [batch][R][scales_ld], scales_ld >= C/bs
  *          (bs = 16 or 32), batch stride R * scales_ld; or, with
  *          FOS_FLAG_SCALE_SWIZZLED, fos_scales_size(R, C/bs, flags) bytes per
- *          batch entry (scales_ld ignored; padding bytes are not written).
+ *          batch entry (scales_ld ignored; padding bytes are not written:
+ *          zero them once, since block-scaled tensor-core GEMMs read the
+ *          padded scales of partial tiles).
  *          NVFP4: E4M3 codes; MXFP4: E8M0 codes (2^(byte-127)).
  *          In 16x16 mode the tile's scale is repeated in each of its 16 rows.
  *   tensor_scale float [batch]: the FP32 per-tensor scale S_t (NVFP4; the

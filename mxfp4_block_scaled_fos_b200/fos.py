@@ -136,7 +136,9 @@ def _alloc_qtensor(batch, R, C, fmt, block, flags, device, with_choice, nblocks)
     bs = 32 if fmt == "mxfp4" else 16
     codes = torch.empty(batch, R, C // 2, dtype=torch.uint8, device=device)
     if flags & FLAG_SCALE_SWIZZLED:
-        scales = torch.empty(batch, scales_size(R, C // bs, flags), dtype=torch.uint8, device=device)
+        # zeroed: the library leaves the layout's padding unwritten, and a
+        # tensor-core GEMM reads the padded scales of partial tiles
+        scales = torch.zeros(batch, scales_size(R, C // bs, flags), dtype=torch.uint8, device=device)
     else:
         scales = torch.empty(batch, R, C // bs, dtype=torch.uint8, device=device)
     ts = torch.empty(batch, dtype=torch.float32, device=device) if fmt != "mxfp4" else None

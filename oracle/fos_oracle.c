@@ -39,8 +39,9 @@
  * matrix, Triton's CPU Philox, the worked example's printed MAEs, invariants,
  * brute force).  Parity unpinned (fixed only by the readings and by GPU
  * parity, not by the pages): the binary32 evaluation order of the block
- * error tree (R6), of the effective scale (R5), of the Hadamard butterflies
- * (R10) and the bit layout of the swizzled scale array (R19).
+ * error tree (R6), of the effective scale (R5) and of the Hadamard
+ * butterflies (R10).  The NVFP4 swizzled scale layout (R19) is pinned through
+ * GPU parity and a cuBLAS block-scaled GEMM that consumes it.
  */
 #include <float.h>
 #include <math.h>
