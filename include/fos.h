@@ -104,8 +104,13 @@ typedef struct fos_options {
  *          rowwise and colwise copies get the same value; NULL allowed only
  *          for MXFP4).
  *   choice_bits uint8, nullable: bit b (byte b>>3, bit b&7) = 1 when linear
- *          block b (over [batch][R][C/16], or over the 16x16 tiles in tile
- *          row-major order) kept the 4-candidate.  ceil(nblocks/8) bytes. */
+ *          block b kept the 4-candidate: blocks over [batch][R][C/16], or,
+ *          in 16x16 mode, tiles over [batch][R/16][C/16] in the tile
+ *          row-major order of this copy's own [R][C].  For the transposed
+ *          copy (R = cols, C = rows) the source tile at tile row tr, tile
+ *          column tc is therefore bit (b*(cols/16) + tc)*(rows/16) + tr.
+ *          The buffer must hold 8*ceil(nblocks/64) bytes: the library
+ *          clears and writes it in whole 32- and 64-bit words. */
 typedef struct fos_qtensor {
   uint8_t* codes;
   uint8_t* scales;

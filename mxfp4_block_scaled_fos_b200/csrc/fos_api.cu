@@ -187,7 +187,10 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
   // bitmaps whose words are shared between CTAs are built with atomics on a
   // zeroed buffer.
   if (opt->blk == FOS_BLOCK_16X16) {
-    a.row.choice_aligned = a.col.choice_aligned = (cols / 16) % 8 == 0;
+    // rowwise: a CTA writes whole bytes (8 tile columns of one tile row);
+    // transposed copy: whole 32-bit words (32 tile rows of one tile column)
+    a.row.choice_aligned = (cols / 16) % 8 == 0;
+    a.col.choice_aligned = (rows / 16) % 32 == 0;
   } else if (colwise) {
     a.row.choice_aligned = (cols / 16) % 8 == 0;
     a.col.choice_aligned = (rows / 16) % 32 == 0;

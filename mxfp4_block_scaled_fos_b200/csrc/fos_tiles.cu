@@ -327,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
   __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
   __shared__ __align__(16) uint8_t s_tc[COL ? kSubCols * 32 : 16];
   __shared__ float2 s_tab[128];
-  __shared__ uint32_t s_bits[kSubRows / 16];
+  __shared__ uint32_t s_bits[kSubRows / 16];   // rowwise picks of a sub-tile: tile row -> 8 tile columns
+  __shared__ uint32_t s_cbits[kSubCols / 16];  // transposed copy: tile column -> 32 tile rows of the strip
 
   const int b = blockIdx.z;
   const int c0 = blockIdx.x * kSubCols;
@@ -340,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
     if (COL && a.col.tensor_scale) a.col.tensor_scale[b] = St;
   }
   if (threadIdx.x < kSubRows / 16) s_bits[threadIdx.x] = 0;
+  if (threadIdx.x < kSubCols / 16) s_cbits[threadIdx.x] = 0;
 
   const int t = threadIdx.x;
   const int tile = t >> 3, i = t & 7;
@@ -421,7 +423,10 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
         a.col.scales[scale_off<SWZ>(a.col, b, gcA, gtr)] = (uint8_t)s;
         a.col.scales[scale_off<SWZ>(a.col, b, gcA + 1, gtr)] = (uint8_t)s;
       }
-      if (F46 && i == 0 && pick && (a.row.choice || a.col.choice)) atomicOr(&s_bits[tr], 1u << tc);
+      if (F46 && i == 0 && pick) {
+        if (ROW && a.row.choice) atomicOr(&s_bits[tr], 1u << tc);
+        if (COL && a.col.choice) atomicOr(&s_cbits[tc], 1u << (4 * k + tr));
+      }
     }
     __syncthreads();
     if (COL) {
@@ -436,26 +441,44 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
         if (grow + 16 < a.rows) store_codes8(a.col, b, gc, byte_col + 8, v.z, v.w);
       }
     }
-    if (F46 && t < kSubRows / 16) {
+    // rowwise copy: one bit per tile in the tile row-major order of x, so a
+    // sub-tile row of 8 tiles is one byte
+    if (ROW && F46 && a.row.choice && t < kSubRows / 16) {
       const uint32_t v = s_bits[t];
       s_bits[t] = 0;
       const long long gtr2 = (r0 >> 4) + t;
       if (gtr2 < ntr) {
         const unsigned long long bit = ((unsigned long long)b * ntr + gtr2) * ntc + (c0 >> 4);
-        uint8_t* ch[2] = {ROW ? a.row.choice : nullptr, COL ? a.col.choice : nullptr};
-        const int aligned[2] = {a.row.choice_aligned, a.col.choice_aligned};
-#pragma unroll
-        for (int z = 0; z < 2; ++z) {
-          if (!ch[z]) continue;
-          if (aligned[z]) {
-            ch[z][bit >> 3] = (uint8_t)v;
-          } else if (v) {
-            unsigned int* wp = reinterpret_cast<unsigned int*>(ch[z]) + (bit >> 5);
-            const int sh = (int)(bit & 31);
-            const unsigned long long vv = (unsigned long long)v << sh;
-            if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
-            if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
-          }
+        if (a.row.choice_aligned) {
+          a.row.choice[bit >> 3] = (uint8_t)v;
+        } else if (v) {
+          unsigned int* wp = reinterpret_cast<unsigned int*>(a.row.choice) + (bit >> 5);
+          const int sh = (int)(bit & 31);
+          const unsigned long long vv = (unsigned long long)v << sh;
+          if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
+          if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
+        }
+      }
+    }
+  }
+  // transposed copy: one bit per tile in the tile row-major order of x^T
+  // ([cols][rows]), so source tile (gtr, gtc) is bit (b*ntc + gtc)*ntr + gtr
+  // and the strip's 32 tile rows of one tile column are 32 consecutive bits
+  if (COL && F46 && a.col.choice) {
+    __syncthreads();
+    if (t < kSubCols / 16) {
+      const long long gtc = (c0 >> 4) + t;
+      if (gtc < ntc) {
+        const uint32_t v = s_cbits[t];
+        const unsigned long long bit = ((unsigned long long)b * ntc + gtc) * ntr + (rs0 >> 4);
+        unsigned int* wp = reinterpret_cast<unsigned int*>(a.col.choice) + (bit >> 5);
+        if (a.col.choice_aligned) {
+          *wp = v;
+        } else if (v) {
+          const int sh = (int)(bit & 31);
+          const unsigned long long vv = (unsigned long long)v << sh;
+          if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
+          if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
         }
       }
     }

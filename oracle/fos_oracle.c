@@ -448,7 +448,8 @@ int or_amax(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
  *   r_choice bitmap, bit b = 1 when block b (linear index) chose 4
  *   c_codes  [batch, cols, rows/2]  colwise 1x16 (or the 16x16 transpose)
  *   c_scales [batch, cols, rows/16]
- *   c_choice bitmap over colwise blocks (1x16 only)
+ *   c_choice bitmap over the colwise copy's blocks (1x16), or over the
+ *            transposed copy's 16x16 tiles in its own tile row-major order
  *   tensor_scale [batch]  (NVFP4)
  * amax_in (nullable) gives the per-batch amax instead of computing it. */
 int or_quantize(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
@@ -550,9 +551,15 @@ int or_quantize(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
               g[i * 16 + j] = base + r * cols + c;
             }
           uint8_t s = nvfp4_block(w, g, 256, S_t, o, codes, &p4);
-          /* R7: one bit per tile in tile row-major order, for both copies */
+          /* R7: one bit per tile, in tile row-major order over each copy's
+           * own [R][C]: the rowwise copy is x ([rows][cols]), the transposed
+           * copy is x^T ([cols][rows]), where source tile (tr, tc) sits at
+           * tile row tc, tile column tr. */
           set_bit(r_choice, (b * (rows / 16) + tr) * (cols / 16) + tc, p4);
-          set_bit(c_choice, (b * (rows / 16) + tr) * (cols / 16) + tc, p4);
+          if (OR_MUTANT == 19) /* the transposed copy indexed like the source */
+            set_bit(c_choice, (b * (rows / 16) + tr) * (cols / 16) + tc, p4);
+          else
+            set_bit(c_choice, (b * (cols / 16) + tc) * (rows / 16) + tr, p4);
           for (int i = 0; i < 16; i++) {
             int64_t r = tr * 16 + i;
             if (r_scales) r_scales[(b * rows + r) * (cols / 16) + tc] = s;

@@ -25,6 +25,7 @@ MUTANTS = {
     16: "Philox first key increment off by one",
     17: "bf16 rounding breaks ties upward instead of to even",
     18: "SR Philox counter is the element index instead of index / 16",
+    19: "2D transposed copy's choice bit at the source tile's index",
 }
 
 PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")

@@ -477,6 +477,40 @@ def test_2d_transposed_copy_is_exact_transpose():
     assert np.array_equal(d_r[0].T, d_c[0])
 
 
+@pytest.mark.parametrize("rows,cols,seed", [(32, 64, 30), (48, 80, 31), (80, 48, 32)])
+def test_2d_transposed_choice_bits_follow_the_transposed_tiles(rows, cols, seed):
+    """The transposed copy's choice bitmap is indexed over its own 16x16 tiles
+    in tile row-major order: tile (i, j) of x^T is source tile (j, i).
+
+    Two checks that do not use the oracle's index formula: (1) the bitmap of
+    the transposed copy equals the rowwise tile bitmap reshaped to
+    (rows/16, cols/16) and transposed; (2) read from the transposed copy's own
+    codes, a tile whose largest magnitude code is 6 (value 4) kept the
+    4-candidate and one whose largest is 7 (value 6) kept the 6-candidate
+    (normal scales), and that is the bit at the tile's own index."""
+    rng = np.random.default_rng(seed)
+    found = False
+    for _ in range(20):
+        x = _random_tensor(rng, rows, cols, "scaled")
+        q = oracle.quantize(x, blk=oracle.BLK_16X16, colwise=True)
+        ntr, ntc = rows // 16, cols // 16
+        rbits = np.unpackbits(q["r_choice"], bitorder="little")[: ntr * ntc].reshape(ntr, ntc)
+        if 0 < rbits.sum() < ntr * ntc:
+            found = True
+            break
+    assert found, "no tensor with both choices found"
+    cbits = np.unpackbits(q["c_choice"], bitorder="little")[: ntr * ntc].reshape(ntc, ntr)
+    assert np.array_equal(cbits, rbits.T)
+    cc = _nibbles(q["c_codes"][0]) & 7                       # [cols, rows]
+    cs = _e4m3_val(q["c_scales"][0][::16])                   # [ntc, ntr]
+    for i in range(ntc):
+        for j in range(ntr):
+            if cs[i, j] < 2.0 ** -6:
+                continue
+            top = cc[16 * i:16 * i + 16, 16 * j:16 * j + 16].max()
+            assert top == (6 if cbits[i, j] else 7), (i, j, top, cbits[i, j])
+
+
 def test_colwise_is_rowwise_of_transpose():
     rng = np.random.default_rng(18)
     x = _random_tensor(rng, 64, 48, "outliers")
