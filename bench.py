@@ -44,16 +44,33 @@ def measured_peaks():
 
 
 # ------------------------------------------------------------------ dist
-def dist_setup(n_gpus):
+def relaunch_as_ranks(n: int) -> int:
+    """Run this same command as n ranks, one process per GPU, under
+    torch.distributed.run on this node (127.0.0.1); returns its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+def dist_setup(n_gpus, dry_run=False):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit("bench.py: --gpus %d but WORLD_SIZE=%d" % (n_gpus, world))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    else:
+        if dry_run:
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        else:
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local))
+    elif not dry_run:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -156,7 +173,9 @@ def time_loop(fn, steps, warmup, world, stream):
 
 
 # ------------------------------------------------------------------ ncu traffic
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "k_q1x16_fused_moe_experts.md")
+# DRAM bytes per element of each kernel's committed ncu capture, with the
+# source hash it was taken at (written beside the summaries in profiles/)
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def source_hash() -> str:
@@ -166,50 +185,71 @@ def source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mxfp4_block_scaled_fos_b200", "csrc")
     for fn in sorted(glob.glob(os.path.join(csrc, "*"))):
+        if not os.path.isfile(fn):
+            continue
         with open(fn, "rb") as f:
             h.update(os.path.basename(fn).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(elems):
-    """DRAM bytes per launch of the fused kernel from the committed ncu
-    summary (scaled from its capture to `elems`), or None if the sources
-    changed since the capture."""
+def profiled_traffic(kernel, elems):
+    """DRAM bytes per launch of `kernel` from profiles/traffic.json (its ncu
+    capture's dram__bytes_read.sum + dram__bytes_write.sum per element,
+    scaled to `elems`), or None if the sources changed since the capture."""
     try:
-        kv = {}
-        with open(PROFILE_SUMMARY) as f:
-            for line in f:
-                if ":" in line and line.startswith("- "):
-                    k, v = line[2:].split(":", 1)
-                    kv[k.strip()] = v.strip().strip("`")
-        if kv.get("source_sha256") != source_hash():
+        with open(TRAFFIC_JSON) as f:
+            d = json.load(f)[kernel]
+        if d.get("source_sha256") != source_hash():
             return None
-        per_elem = float(kv["dram_bytes_per_element"])
-        return int(per_elem * elems)
-    except (OSError, KeyError, ValueError):
+        return int(float(d["dram_bytes_per_element"]) * elems)
+    except (OSError, KeyError, ValueError, TypeError):
         return None
 
 
 # ------------------------------------------------------------------ CPU baseline
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_all_cores(entries, threads):
+    """Wall time (s) of the oracle quantizing `entries` (per-entry amax +
+    4/6 quantize) on `threads` host threads."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.quantize_parallel(entries, threads)
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(x_cpu_bits, budget_s=12.0):
-    """Time the oracle (single thread) on whole experts until ~budget_s."""
+    """The oracle as it stands on the host cores: all cores (threads over
+    row chunks of whole experts) and, beside it, one thread."""
     import numpy as np
     import oracle
+    oracle.lib()
+    per = x_cpu_bits.shape[1] * x_cpu_bits.shape[2]
+    cores = host_cores()
+    entries = [np.ascontiguousarray(x_cpu_bits[e]) for e in range(x_cpu_bits.shape[0])]
+    dt = oracle_all_cores(entries, cores)
+    elems = len(entries) * per
+    # single thread: whole experts until ~budget_s / 2
     done = 0
     t0 = time.perf_counter()
-    per = x_cpu_bits.shape[1] * x_cpu_bits.shape[2]
     while True:
-        e = done % x_cpu_bits.shape[0]
-        oracle.quantize(np.ascontiguousarray(x_cpu_bits[e:e + 1]))
+        oracle.quantize(entries[done % len(entries)][None])
         done += 1
-        if time.perf_counter() - t0 > budget_s:
+        if time.perf_counter() - t0 > budget_s / 2:
             break
-    dt = time.perf_counter() - t0
-    elems = done * per
+    dt1 = time.perf_counter() - t0
     return {"value": round(elems * BYTES_PER_ELEM / dt / 1e9, 6), "unit": "GB/s",
-            "elems_per_s": round(elems / dt, 1), "cores": 1, "kind": "oracle",
-            "sample": "%d expert(s) of 2880x2880 (%d elements), amax pass + 4/6 quantize, "
-                      "single-threaded C oracle" % (done, elems)}
+            "elems_per_s": round(elems / dt, 1), "cores": cores, "threads": cores, "kind": "oracle",
+            "sample": "%d experts of 2880x2880 (%d elements), per-expert amax + 4/6 quantize, C oracle on "
+                      "%d host threads (row chunks, GIL released)" % (len(entries), elems, cores),
+            "single_thread": {"value": round(done * per * BYTES_PER_ELEM / dt1 / 1e9, 6), "unit": "GB/s",
+                              "sample": "%d expert(s), one thread" % done}}
 
 
 # ------------------------------------------------------------------ main arms
@@ -271,7 +311,7 @@ def run_fos(args, world, rank):
                    "l2": "input %.2f GB > 126 MB L2; no flush needed" % (2 * elems / 1e9)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(elems),
+                     "traffic": profiled_traffic("k_q1x16_fused_moe_experts", elems),
                      "kernel": "k_q1x16_fused<4/6, RNE> (per-expert amax + quantize)",
                      "kernel_ms": round(ms_per_step, 4),
                      "bytes_per_launch": int(elems * BYTES_PER_ELEM),
@@ -285,7 +325,8 @@ def run_fos(args, world, rank):
         "modes": extra,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        xs = workloads.bits(x[:4])
+        n_cpu = max(4, min(E, host_cores()))
+        xs = workloads.bits(x[:n_cpu])
         out["cpu_baseline"] = cpu_baseline(xs, budget_s=args.cpu_seconds)
     return out
 
@@ -389,6 +430,46 @@ def measure_modes(args, world, x, dev, stream, peak):
     return res
 
 
+def run_rows(args, world, rank):
+    """--split rows: one tensor of world x 16384 rows x 8192 cols (Student-t
+    gradients), each rank holding its 16384 rows.  One step = the local
+    per-tensor amax, an all-reduce(MAX) of it over the ranks (NCCL), and the
+    4/6 1x16 rowwise quantize of the local rows with the global amax."""
+    import mxfp4_block_scaled_fos_b200 as F
+    from mxfp4_block_scaled_fos_b200 import shard, workloads
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    R, C = 16384, 8192
+    x = workloads.gradient_student_t(R, C, device=dev, seed=rank)
+    row0 = rank * R
+    out = F.quantize(x, amax=F.amax(x))[0]
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def step():
+        F.amax(x, out=amax)
+        shard.global_amax(amax)
+        F.quantize(x, amax=amax, elem_offset=row0 * C, out_row=out)
+
+    clk = ClockSampler(torch.cuda.current_device())
+    clk.start()
+    t_ms = time_loop(step, args.steps, args.warmup, world, stream)
+    clk.stop()
+    ms = t_ms / args.steps
+    peak, peak_kind = measured_peaks()
+    elems = x.numel()
+    value = world * elems * BYTES_PER_ELEM / (ms * 1e-3) / 1e9
+    return {"metric": "NVFP4 4/6 quantize GB/s and % of B200 HBM peak (bf16 in, FP4+E4M3 out)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "gradient_student_t_rows_split_%dx16384x8192_nvfp4_46_1x16_rne" % world,
+                       "rows_per_gpu": R, "cols": C, "collective": "all_reduce(MAX) of 1 float per step",
+                       "parallelism": "rows%d" % world},
+            "frac_of_hbm": round(value / world / peak, 4),
+            "gpu_launches": 2 * args.steps, "clocks": clk.summary(),
+            "peak_source": "%s hbm_gbs" % peak_kind}
+
+
 def measure_e2e(args, world, x, row, ws, status, stream):
     """Same metric through the public API with pinned host buffers: H2D of the
     input, quantize (amax + 4/6), D2H of codes, scales and S_t, every step."""
@@ -417,34 +498,46 @@ def measure_e2e(args, world, x, row, ws, status, stream):
 
 
 def run_reference(args, world, rank):
-    """The oracle (CPU, single thread) on a bounded sample per step."""
-    import numpy as np
+    """The oracle on the host cores, one expert of the workload per step
+    (its rows split over all host threads)."""
     import oracle
     from mxfp4_block_scaled_fos_b200 import workloads
     if rank != 0:
         return None
     x = workloads.moe_experts(1, 2880, 2880, device="cpu", seed=0)
-    xb = workloads.bits(x)
+    xb = workloads.bits(x)[0]
     oracle.lib()
+    cores = host_cores()
     for _ in range(args.warmup):
-        oracle.quantize(xb)
-    t0 = time.perf_counter()
+        oracle_all_cores([xb], cores)
+    dt = 0.0
     for _ in range(args.steps):
-        oracle.quantize(xb)
-    dt = time.perf_counter() - t0
+        dt += oracle_all_cores([xb], cores)
     elems = xb.size * args.steps
     v = elems * BYTES_PER_ELEM / dt / 1e9
-    sample = "one 2880x2880 expert per step (amax pass + 4/6 quantize), single-threaded C oracle"
+    sample = ("one 2880x2880 expert per step (per-expert amax + 4/6 quantize), C oracle on %d host "
+              "threads over row chunks" % cores)
     return {"impl": "reference", "metric": "NVFP4 4/6 quantize GB/s and % of B200 HBM peak "
             "(bf16 in, FP4+E4M3 out)", "value": round(v, 6), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": "1 of 128 experts per step"},
-            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "kind": "oracle", "cores": 1,
-                             "sample": sample},
+            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "kind": "oracle", "cores": cores,
+                             "threads": cores, "sample": sample},
             "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+
+
+def run_dry(args, world, rank):
+    """--dry-run: the launch and rank plumbing only, no GPU work."""
+    sys.stderr.write("bench dry run: rank %d of %d\n" % (rank, world))
+    if world > 1:
+        t = torch.tensor([1.0])
+        torch.distributed.all_reduce(t)
+        assert int(t.item()) == world
+    return {"metric": "dry run", "value": 0.0, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "dry_run": True, "world_size_env": int(os.environ.get("WORLD_SIZE", "1"))}
 
 
 def main():
@@ -456,9 +549,15 @@ def main():
     ap.add_argument("--no-modes", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--split", choices=["entries", "rows"], default="entries",
+                    help="entries: each rank quantizes its own 128 experts (no collective); rows: each "
+                         "rank quantizes its rows of one tensor after an amax all-reduce")
+    ap.add_argument("--dry-run", action="store_true", help="launch the ranks and exit (no GPU work)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch_as_ranks(args.gpus))
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
@@ -466,12 +565,15 @@ def main():
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    world, rank, _ = dist_setup(args.gpus)
-    from mxfp4_block_scaled_fos_b200 import build as fbuild
-    if rank == 0:
-        fbuild.build()
-    barrier(world)
-    out = run_fos(args, world, rank)
+    world, rank, _ = dist_setup(args.gpus, args.dry_run)
+    if args.dry_run:
+        out = run_dry(args, world, rank)
+    else:
+        from mxfp4_block_scaled_fos_b200 import build as fbuild
+        if rank == 0:
+            fbuild.build()
+        barrier(world)
+        out = run_rows(args, world, rank) if args.split == "rows" else run_fos(args, world, rank)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

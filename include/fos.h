@@ -181,8 +181,10 @@ fos_status fos_dequantize(const fos_qtensor* q, int32_t fmt, int64_t batch, int6
  * memory (per-batch-entry amax words and counters) lives in a fixed array in the
  * library, sized for FOS_STATIC_MAX_BATCH batch entries; every GPU that
  * loads the library holds it (about 49 KB) until the process exits.
- * batch > FOS_STATIC_MAX_BATCH returns FOS_ERR_WORKSPACE.  No device memory
- * is allocated or freed.
+ * A call that needs the scratch (NVFP4 without amax_in) with batch >
+ * FOS_STATIC_MAX_BATCH returns FOS_ERR_WORKSPACE; MXFP4 calls and calls with
+ * amax_in use no scratch and take any batch fos_quantize takes.  No device
+ * memory is allocated or freed.
  *
  * The first call on a device looks up the array's device address (with that
  * device current) and keeps it; make that first call before any stream

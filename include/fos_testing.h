@@ -1,0 +1,40 @@
+/*
+ * fos_testing.h -- test hooks exported by libfos.so.  Not part of the
+ * quantizer's interface (include/fos.h); tests use them to drive code paths
+ * that valid input never reaches, without faulting or hanging the GPU.
+ */
+#ifndef FOS_TESTING_H_
+#define FOS_TESTING_H_
+
+#include "fos.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * fos_testing_quantize_stalled -- fos_quantize (NVFP4, 1x16, rowwise, amax
+ * computed in the call, so the fused amax + quantize kernel runs) with a
+ * failure planted on the host side: the amax items of batch entry
+ * `stall_entry` never count in, and every bounded wait of the kernel gives
+ * up after `spin_limit` polls (about 128 ns apart) instead of about 2^23.
+ *
+ * Every quantize item of that entry therefore waits until its limit, sets
+ * FOS_STATUS_TIMEOUT in *status (status must not be NULL to see it) and goes
+ * on, so the launch still ends.  The other entries are quantized exactly as
+ * by fos_quantize; the stalled entry's outputs are unspecified.  Arguments
+ * are those of fos_quantize; stall_entry must be in [0, batch) and
+ * spin_limit >= 1 (FOS_ERR_ARG otherwise); other formats and block modes
+ * return FOS_ERR_UNSUPPORTED.
+ */
+fos_status fos_testing_quantize_stalled(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                                        int64_t ld, const fos_options* opt,
+                                        const fos_qtensor* rowwise, void* workspace,
+                                        size_t workspace_bytes, uint32_t* status,
+                                        int32_t stall_entry, uint32_t spin_limit, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOS_TESTING_H_ */

@@ -7,6 +7,10 @@ architectures), without fast-math, with contraction off and IEEE division,
 so that the binary32 steps the quantizer defines are rounded as written.
 Objects go to _build/ at the repository root; the library lands next to
 this file, where the Python binding loads it.
+
+The same flags build libfos_check.so from csrc/check/ (the exhaustive
+device-side checks of the kernels' arithmetic helpers, used by the tests
+only; include/fos_check.h).
 """
 from __future__ import annotations
 
@@ -23,6 +27,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfos.so")
+CHECK_SRC = os.path.join(CSRC, "check", "fos_check.cu")
+CHECK_LIB = os.path.join(PKG, "libfos_check.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -82,12 +88,29 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True,
     return lib
 
 
+def build_check(force: bool = False) -> str:
+    """Compile csrc/check/fos_check.cu into libfos_check.so (test checks)."""
+    deps = [CHECK_SRC] + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+        glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
+    if not force and os.path.exists(CHECK_LIB) and \
+            all(os.path.getmtime(d) <= os.path.getmtime(CHECK_LIB) for d in deps):
+        return CHECK_LIB
+    tmp = CHECK_LIB + ".tmp%d" % os.getpid()
+    cmd = [NVCC, *ARCH, *FLAGS, "-shared", "-cudart", "static", "-o", tmp, CHECK_SRC]
+    p = subprocess.run(cmd, capture_output=True, text=True)
+    if p.returncode != 0:
+        raise RuntimeError("nvcc failed for %s:\n%s" % (CHECK_SRC, p.stderr[-8000:]))
+    os.replace(tmp, CHECK_LIB)
+    return CHECK_LIB
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
     args = ap.parse_args()
     print(build(force=args.force, verbose_ptxas=args.verbose_ptxas, quiet=False))
+    print(build_check(force=args.force))
 
 
 if __name__ == "__main__":

@@ -20,6 +20,12 @@ FastDiv make_fastdiv(uint32_t d) {
 
 namespace {
 
+// 1: the fused amax + quantize path uses the queue-fed kernel of
+// fos_rowwise.cu instead of the cooperative pipeline of fos_pipe.cu
+#ifndef FOS_FUSED_QUEUE
+#define FOS_FUSED_QUEUE 1
+#endif
+
 constexpr uint32_t kUnitsQuant = 256 * 4;   // work units per CTA (tile kernels)
 constexpr uint32_t kBlocksRowwise = 256 * 8; // 16-element blocks per CTA (rowwise 1x16)
 constexpr uint32_t kUnitsAmax = 256 * 8;    // block pairs per CTA (amax pass)
@@ -30,7 +36,7 @@ inline bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0
 
 long long round_up(long long v, long long m) { return (v + m - 1) / m * m; }
 
-size_t ws_bytes(int64_t batch) { return (size_t)(12 * round_up(batch, 64) + 256); }
+size_t ws_bytes(int64_t batch) { return workspace_bytes_for(batch); }
 
 // Validate one output descriptor for a tensor of R rows and C columns.
 fos_status check_out(const fos_qtensor* q, int64_t R, int64_t C, int64_t bs, bool nvfp4,
@@ -68,6 +74,17 @@ OutDesc make_out(const fos_qtensor* q, int64_t R, int64_t C, int64_t bs, uint32_
 }
 
 size_t choice_bytes(int64_t nblocks) { return (size_t)(8 * ((nblocks + 63) / 64)); }
+
+// Test hooks of the fused kernel's bounded waits (fos_testing_quantize_stalled).
+struct WaitHooks {
+  uint32_t spin_limit = 1u << 23;
+  int stall_entry = -1;
+};
+
+fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
+                         const fos_options* opt, const float* amax_in, const fos_qtensor* rowwise,
+                         const fos_qtensor* colwise, void* workspace, size_t workspace_bytes,
+                         uint32_t* status, void* stream, const WaitHooks& hooks);
 
 }  // namespace
 }  // namespace fos
@@ -111,6 +128,34 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
                         const fos_qtensor* rowwise, const fos_qtensor* colwise,
                         void* workspace, size_t workspace_bytes, uint32_t* status,
                         void* stream) {
+  return quantize_impl(x, batch, rows, cols, ld, opt, amax_in, rowwise, colwise, workspace,
+                       workspace_bytes, status, stream, WaitHooks());
+}
+
+fos_status fos_testing_quantize_stalled(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                                        int64_t ld, const fos_options* opt,
+                                        const fos_qtensor* rowwise, void* workspace,
+                                        size_t workspace_bytes, uint32_t* status,
+                                        int32_t stall_entry, uint32_t spin_limit, void* stream) {
+  if (!opt || !rowwise) return FOS_ERR_NULL;
+  if (opt->fmt == FOS_FMT_MXFP4 || opt->blk != FOS_BLOCK_1X16) return FOS_ERR_UNSUPPORTED;
+  if (stall_entry < 0 || stall_entry >= batch || spin_limit < 1) return FOS_ERR_ARG;
+  WaitHooks h;
+  h.spin_limit = spin_limit;
+  h.stall_entry = stall_entry;
+  return quantize_impl(x, batch, rows, cols, ld, opt, nullptr, rowwise, nullptr, workspace,
+                       workspace_bytes, status, stream, h);
+}
+
+}  // extern "C"
+
+namespace fos {
+namespace {
+
+fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
+                         const fos_options* opt, const float* amax_in, const fos_qtensor* rowwise,
+                         const fos_qtensor* colwise, void* workspace, size_t workspace_bytes,
+                         uint32_t* status, void* stream, const WaitHooks& hooks) {
   if (!opt || !x) return FOS_ERR_NULL;
   if (!rowwise && !colwise) return FOS_ERR_NULL;
   if (opt->fmt < 0 || opt->fmt > 2 || opt->blk < 0 || opt->blk > 2 || opt->rnd < 0 ||
@@ -169,6 +214,8 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
   a.status = status;
   a.seed = opt->seed;
   a.elem_offset = opt->elem_offset;
+  a.spin_limit = hooks.spin_limit;
+  a.stall_entry = hooks.stall_entry;
   if (rowwise) {
     const int64_t nb = opt->blk == FOS_BLOCK_16X16 ? (rows / 16) * (cols / 16) : rows * (cols / bs);
     a.row = make_out(rowwise, rows, cols, bs, opt->flags, nb);
@@ -224,8 +271,13 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
     // one persistent launch: per-entry amax and quantize, pipelined so the
     // second read of each entry comes from L2
     if (cudaMemsetAsync(amax_ws, 0, 12 * round_up(batch, 64), st) != cudaSuccess) return FOS_ERR_CUDA;
+#if FOS_FUSED_QUEUE
     ce = launch_q1x16_fused(a, (int)batch, opt->fmt, sr, rht, swz, dense, amax_ws, done_ws, claim_ws,
                             st);
+#else
+    void* ring = (char*)workspace + 12 * round_up(batch, 64) + 256;
+    ce = launch_q1x16_pipe(a, (int)batch, opt->fmt, sr, rht, swz, dense, amax_ws, done_ws, ring, st);
+#endif
     if (ce == cudaSuccess) return FOS_OK;
     if (ce != cudaErrorNotSupported) return FOS_ERR_CUDA;
     (void)cudaGetLastError();  // fall back to the two-kernel path below
@@ -250,6 +302,11 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
   if (ce == cudaErrorNotSupported) return FOS_ERR_UNSUPPORTED;
   return ce == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;
 }
+
+}  // namespace
+}  // namespace fos
+
+extern "C" {
 
 fos_status fos_amax(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
                     const fos_options* opt, float* amax_out, uint32_t* status, void* stream) {

@@ -97,19 +97,24 @@ __device__ __forceinline__ TScale make_tscale(float St) {
   return t;
 }
 
-// RN(a / S_t) for a >= 0.  Fast path: q0 = RN(a*y), one fma correction
-// q0 + (a - S_t*q0)*y (P. Markstein, IBM J. Res. Dev. 34(1), 1990).  Checked
-// against IEEE division for ~20000 divisors over the whole binary32 range,
-// every positive finite bf16 dividend and random binary32 dividends: equal
-// whenever dividend and quotient are >= 2^-100.  With S_t >= 2^-92 that
-// covers every quotient r >= 2^-8; smaller quotients give E4M3(r/4) =
-// E4M3(r/6) = 0 whichever way they round, so the scale codes are exact.
+// RN(a / S_t) for a >= 0, clamped to FLT_MAX.  Fast path: q0 = RN(a*y),
+// one fma correction q0 + (a - S_t*q0)*y (P. Markstein, IBM J. Res. Dev.
+// 34(1), 1990): equal to the IEEE quotient whenever dividend and quotient
+// are >= 2^-100 and the quotient is finite.  With S_t >= 2^-92 that covers
+// every quotient r >= 2^-8; smaller quotients give E4M3(r/4) = E4M3(r/6) = 0
+// whichever way they round, so the scale codes are exact.  A quotient that
+// overflows (a caller-supplied amax far below the data) would be inf, or NaN
+// from the correction step; both are clamped to FLT_MAX, whose candidate
+// codes saturate at 448 like those of inf.  tests/test_gpu_exhaustive.py
+// checks the candidate codes against IEEE division for every pair of
+// non-negative bf16 values (block amax, tensor amax) and for random binary32
+// pairs (the RHT case), and the quotient bits where the claim above holds.
 __device__ __forceinline__ float div_tscale(float a, const TScale& t) {
   const float q0 = __fmul_rn(a, t.y);
   const float rem = __fmaf_rn(-q0, t.St, a);
   float r = __fmaf_rn(rem, t.y, q0);
   if (!t.fast) r = (t.St == 0.0f) ? 0.0f : __fdiv_rn(a, t.St);  // uniform per tensor
-  return r;
+  return fminf(r, kFltMax);
 }
 
 // The same with the path chosen at compile time (FAST: t.fast is known true).
@@ -117,9 +122,9 @@ template <bool FAST>
 __device__ __forceinline__ float div_tscale_t(float a, const TScale& t) {
   if (FAST) {
     const float q0 = __fmul_rn(a, t.y);
-    return __fmaf_rn(__fmaf_rn(-q0, t.St, a), t.y, q0);
+    return fminf(__fmaf_rn(__fmaf_rn(-q0, t.St, a), t.y, q0), kFltMax);
   }
-  return (t.St == 0.0f) ? 0.0f : __fdiv_rn(a, t.St);
+  return (t.St == 0.0f) ? 0.0f : fminf(__fdiv_rn(a, t.St), kFltMax);
 }
 
 // Candidate scale codes of a block with amax a: (s6, s4) as E4M3 bytes,
@@ -314,6 +319,87 @@ __device__ __forceinline__ void store_choice64(const OutDesc& o, unsigned long l
     if (lo) atomicOr(base + (gbit >> 6), lo);
     if (hi) atomicOr(base + (gbit >> 6) + 1, hi);
   }
+}
+
+// One 16-element block j (row-major over [rows][cols/16]) of entry b, with
+// the general row stride; 16-byte loads.
+__device__ __forceinline__ void load_block(const QuantArgs& a, int b, uint32_t j, uint4 (&w)[2]) {
+  const uint32_t row = fdiv(j, a.bpr);
+  const uint32_t cb = j - row * a.bpr.d;
+  const uint4* p = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs +
+                                                 (long long)row * a.ld + (long long)cb * 16);
+  w[0] = __ldg(p);
+  w[1] = __ldg(p + 1);
+}
+
+// Codes (8 bytes) and scale byte of block j of entry b into o (linear or
+// swizzled scales).
+template <bool SWZ>
+__device__ __forceinline__ void store_block(const OutDesc& o, int b, uint32_t j, const FastDiv& bpr,
+                                            const uint32_t (&codes)[2], uint32_t scale) {
+  const uint32_t row = fdiv(j, bpr);
+  const uint32_t cb = j - row * bpr.d;
+  uint2* cp = reinterpret_cast<uint2*>(o.codes + (long long)b * o.codes_bs +
+                                       (long long)row * o.codes_ld + (long long)cb * 8);
+  *cp = make_uint2(codes[0], codes[1]);
+  long long so;
+  if (SWZ) so = (long long)b * o.scales_bs + swz_offset(row, cb, o.col_tiles);
+  else     so = (long long)b * o.scales_bs + (long long)row * o.scales_ld + cb;
+  o.scales[so] = (uint8_t)scale;
+}
+
+// max |y| of the 16-wide RHT y of one block (as binary32 bits).
+__device__ __forceinline__ uint32_t rht_block_amax(uint4 (&w)[2], uint32_t mask16) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    (&w[0].x)[k] ^= rht_word_mask(mask16, k);
+    (&w[1].x)[k] ^= rht_word_mask(mask16, k + 4);
+  }
+  const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+  float2 P[8];
+  unpack_split(W, P);
+  fwht16_split(P);
+  uint32_t m = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
+  return m;
+}
+
+// candidate1 with the scale as a table entry t = (inv, inv, -E, -E): both
+// packed operands come straight from one 16-byte load.
+template <bool WANT_ERR>
+__device__ __forceinline__ Cand1 candidate1_t(const float2 (&P)[8], const float4 t, float nz) {
+  Cand1 r;
+  const float2 inv2 = make_float2(t.x, t.y);
+  float2 v[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = mul2(P[k], inv2);
+  r.c[0] = e2m1x8(v[0].x, v[1].x, v[2].x, v[3].x, v[4].x, v[5].x, v[6].x, v[7].x);
+  r.c[1] = e2m1x8(v[0].y, v[1].y, v[2].y, v[3].y, v[4].y, v[5].y, v[6].y, v[7].y);
+  if (WANT_ERR) {
+    uint32_t ha[4], hb[4];
+    e2m1x8_to_h2(r.c[0], ha);
+    e2m1x8_to_h2(r.c[1], hb);
+    const float2 ne2 = make_float2(t.z, t.w), z2 = make_float2(nz, nz);
+    float2 tt[8];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float2 q0 = make_float2(h_lo(ha[m]), h_lo(hb[m]));   // elements 2m, 2m+8
+      const float2 q1 = make_float2(h_hi(ha[m]), h_hi(hb[m]));   // elements 2m+1, 2m+9
+      const float2 d0 = fma2(q0, ne2, P[2 * m]);
+      const float2 d1 = fma2(q1, ne2, P[2 * m + 1]);
+      tt[2 * m] = fma2(d0, d0, z2);       // RN(d*d), never fused into the adds
+      tt[2 * m + 1] = fma2(d1, d1, z2);
+    }
+    const float2 l1a = add2(tt[0], tt[1]), l1b = add2(tt[2], tt[3]);
+    const float2 l1c = add2(tt[4], tt[5]), l1d = add2(tt[6], tt[7]);
+    const float2 l3 = add2(add2(l1a, l1b), add2(l1c, l1d));   // (sum 0..7, sum 8..15)
+    r.err = __fadd_rn(l3.x, l3.y);
+  } else {
+    r.err = 0.0f;
+  }
+  return r;
 }
 
 __device__ __forceinline__ float tensor_scale_of(const QuantArgs& a, int b, bool f46) {

@@ -39,13 +39,15 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
 
-// RN(r / 6) without a division: q0 = RN(r*y), y = RN(1/6); the remainder
-// r - 6*q0 is exact as an fma and one correction step q0 + rem*y gives the
-// correctly rounded quotient (P. Markstein, IBM J. Res. Dev. 34(1), 1990).
-// Checked against IEEE division for every binary32 r: equal for all
-// r >= 2^-125.  Below that both results are < 2^-127, far under the
-// smallest E4M3 subnormal (2^-9), so the E4M3 code of the quotient -- the
-// only use here -- is 0 either way and no fallback branch is needed.
+// RN(r / 6) without a division, for finite r >= 0: q0 = RN(r*y),
+// y = RN(1/6); the remainder r - 6*q0 is exact as an fma and one correction
+// step q0 + rem*y gives the correctly rounded quotient (P. Markstein, IBM J.
+// Res. Dev. 34(1), 1990).  Equal to IEEE division for every finite r >=
+// 2^-125 (tests/test_gpu_exhaustive.py runs all of them on the device).
+// Below that both results are < 2^-127, far under the smallest E4M3
+// subnormal (2^-9), so the E4M3 code of the quotient -- the only use here --
+// is 0 either way and no fallback branch is needed.  r = inf would give NaN:
+// the callers clamp r to FLT_MAX first.
 __device__ __forceinline__ float div6_for_e4m3(float r) {
   const float y = 1.0f / 6.0f;
   const float q0 = __fmul_rn(r, y);
@@ -219,9 +221,9 @@ __device__ __forceinline__ float sr_e2m1_mag(float v, uint32_t byte) {
 // 0x3fffff).  For 0.5 <= v < 1 the binade holds one point (0.5) and the next
 // is 1.0: the same with 23 mantissa bits.  For v < 0.5: lo = 0, hi = 0.5,
 // 512*p = 1024*v (exact).  Returns the chosen grid value, or a value >= 6
-// that the saturating E2M1 encode turns into 6.  Checked on the CPU against
-// sr_e2m1_mag for every binary32 v in [0, 16) and infinity with 12 bytes,
-// and for a stride of v with all 256 bytes: identical after saturation.
+// that the saturating E2M1 encode turns into 6.  Equal to sr_e2m1_mag after
+// that encode for every binary32 v in [0, 16] and infinity with every byte
+// (tests/test_gpu_exhaustive.py runs all of them on the device).
 __device__ __forceinline__ float sr_e2m1_mag_bits(float v, uint32_t byte) {
   const uint32_t bits = __float_as_uint(v);
   const uint32_t t13 = (byte << 14) | 0x2000u;   // (2*byte + 1) << 13

@@ -41,6 +41,12 @@ struct QuantArgs {
   // product and fused into the following add
   float neg_zero = -0.0f;
   OutDesc row, col;
+  // Bounded waits of the fused kernel: polls (about 128 ns apart) before a
+  // wait gives up and reports FOS_STATUS_TIMEOUT.  stall_entry >= 0 is a test
+  // hook (fos_testing_quantize_stalled): that entry's amax items never count
+  // in, so every wait on it runs out.
+  uint32_t spin_limit = 1u << 23;
+  int stall_entry = -1;
 };
 
 FastDiv make_fastdiv(uint32_t d);
@@ -56,6 +62,21 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 cudaError_t launch_q1x16_fused(const QuantArgs& a, int batch, int fmt, bool sr, bool rht, bool swz,
                                bool dense, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue,
                                cudaStream_t st);
+// The same as one cooperative launch with a static schedule and no work
+// queue (fos_pipe.cu): amax_ws, cnt: one zeroed word per batch entry; ring:
+// pipe_ring_bytes() of 16-byte aligned workspace (no initialisation needed).
+// Returns cudaErrorNotSupported when the grid cannot be co-resident.
+cudaError_t launch_q1x16_pipe(const QuantArgs& a, int batch, int fmt, bool sr, bool rht, bool swz,
+                              bool dense, uint32_t* amax_ws, uint32_t* cnt, void* ring, cudaStream_t st);
+size_t pipe_ring_bytes();
+
+// Workspace bytes of fos_quantize for `batch` entries: per-entry words
+// (amax, counters, one spare array) then the pipeline's record ring.
+constexpr size_t kRingBytesMax = 16384;
+constexpr size_t workspace_bytes_for(long long batch) {
+  return (size_t)(12 * ((batch + 63) / 64 * 64) + 256) + kRingBytesMax;
+}
+
 cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
                               bool want_row, cudaStream_t st);
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,

@@ -32,29 +32,6 @@ constexpr int kThreads = 256;
 #define FOS_K1_MIN_BLOCKS_HEAVY 4
 #endif
 
-__device__ __forceinline__ void load_block(const QuantArgs& a, int b, uint32_t j, uint4 (&w)[2]) {
-  const uint32_t row = fdiv(j, a.bpr);
-  const uint32_t cb = j - row * a.bpr.d;
-  const uint4* p = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs +
-                                                 (long long)row * a.ld + (long long)cb * 16);
-  w[0] = __ldg(p);
-  w[1] = __ldg(p + 1);
-}
-
-template <bool SWZ>
-__device__ __forceinline__ void store_block(const OutDesc& o, int b, uint32_t j, const FastDiv& bpr,
-                                            const uint32_t (&codes)[2], uint32_t scale) {
-  const uint32_t row = fdiv(j, bpr);
-  const uint32_t cb = j - row * bpr.d;
-  uint2* cp = reinterpret_cast<uint2*>(o.codes + (long long)b * o.codes_bs +
-                                       (long long)row * o.codes_ld + (long long)cb * 8);
-  *cp = make_uint2(codes[0], codes[1]);
-  long long so;
-  if (SWZ) so = (long long)b * o.scales_bs + swz_offset(row, cb, o.col_tiles);
-  else     so = (long long)b * o.scales_bs + (long long)row * o.scales_ld + cb;
-  o.scales[so] = (uint8_t)scale;
-}
-
 // --------------------------------------------------------------------------
 // K0: per-batch-entry amax of |x| (or of the RHT of x).
 // grid (chunks, batch); each thread handles pairs of blocks.
@@ -387,7 +364,6 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 #endif
 constexpr uint32_t kAChunk = FOS_FUSED_ACHUNK;  // blocks per amax item
 constexpr uint32_t kQChunk = FOS_FUSED_QCHUNK;  // blocks per quantize item (multiple of 32)
-constexpr uint32_t kSpinLimit = 1u << 23;  // x ~128 ns sleep
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
@@ -395,11 +371,13 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   return v;
 }
 
-// Bounded wait until *p >= target (thread 0 of the CTA calls it).
-__device__ __forceinline__ void wait_at_least(const uint32_t* p, uint32_t target, uint32_t* status) {
+// Bounded wait until *p >= target (thread 0 of the CTA calls it): at most
+// `limit` polls, then FOS_STATUS_TIMEOUT and return.
+__device__ __forceinline__ void wait_at_least(const uint32_t* p, uint32_t target, uint32_t* status,
+                                              uint32_t limit) {
   uint32_t it = 0;
   while (ld_acquire(p) < target) {
-    if (++it > kSpinLimit) {
+    if (++it > limit) {
       if (status) atomicOr(status, FOS_STATUS_TIMEOUT);
       return;
     }
@@ -507,12 +485,12 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
           atomicMax(amax_ws + it.entry, v);
         }
         __threadfence();
-        atomicAdd(done_a + it.entry, 1u);
+        if (it.entry != a.stall_entry) atomicAdd(done_a + it.entry, 1u);
       }
     } else {
       if (it.entry != tab_entry) {
         if (threadIdx.x == 0) {
-          wait_at_least(done_a + it.entry, na, a.status);
+          wait_at_least(done_a + it.entry, na, a.status, a.spin_limit);
           const float A = __uint_as_float(__ldcg(amax_ws + it.entry));
           s_St = __fdiv_rn(A, F46 ? 1792.0f : 2688.0f);
         }

@@ -16,7 +16,7 @@ namespace {
 
 constexpr int64_t kStaticMaxBatch = FOS_STATIC_MAX_BATCH;
 // the workspace fos_quantize needs for kStaticMaxBatch entries
-constexpr size_t kScratchBytes = 12 * kStaticMaxBatch + 256;
+constexpr size_t kScratchBytes = fos::workspace_bytes_for(kStaticMaxBatch);
 constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
@@ -48,7 +48,10 @@ fos_status fos_quantize_static(const void* x, int64_t batch, int64_t rows, int64
                                int64_t ld, const fos_options* opt, const float* amax_in,
                                const fos_qtensor* rowwise, const fos_qtensor* colwise,
                                uint32_t* status, void* stream) {
-  if (batch > kStaticMaxBatch) return FOS_ERR_WORKSPACE;
+  // only calls that compute the amax use scratch (MXFP4 and calls with
+  // amax_in need none): the batch limit applies to those alone
+  const bool needs_scratch = opt && opt->fmt != FOS_FMT_MXFP4 && !amax_in;
+  if (needs_scratch && batch > kStaticMaxBatch) return FOS_ERR_WORKSPACE;
   void* scratch = nullptr;
   const fos_status e = scratch_address(&scratch);
   if (e != FOS_OK) return e;

@@ -35,7 +35,8 @@ ERRORS = {
 
 # every symbol include/fos.h declares
 EXPORTS = ("fos_quantize", "fos_amax", "fos_dequantize", "fos_workspace_size",
-           "fos_scales_size", "fos_status_string", "fos_version", "fos_quantize_static")
+           "fos_scales_size", "fos_status_string", "fos_version", "fos_quantize_static",
+           "fos_testing_quantize_stalled")
 
 
 class Options(ctypes.Structure):
@@ -76,6 +77,10 @@ def lib(path: str = LIB_PATH):
     L.fos_quantize_static.restype = i32
     L.fos_quantize_static.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P,
                                       ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), P, P]
+    L.fos_testing_quantize_stalled.restype = i32
+    L.fos_testing_quantize_stalled.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options),
+                                               ctypes.POINTER(QTensorC), P, ctypes.c_size_t, P,
+                                               i32, u32, P]
     L.fos_amax.restype = i32
     L.fos_amax.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P, P, P]
     L.fos_dequantize.restype = i32

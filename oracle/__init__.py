@@ -281,6 +281,47 @@ def quantize(x_bits: np.ndarray, fmt: int = FMT_NVFP4_46, blk: int = BLK_1X16,
     return out
 
 
+def quantize_parallel(entries, threads: int, chunk_rows: int = 64, **kw) -> list:
+    """Quantize a list of [rows, cols] bf16-bit arrays (one batch entry each)
+    with the oracle on `threads` host threads, for timing on many cores.
+
+    The C calls release the GIL, so threads run in parallel.  Each entry is
+    cut into row chunks: the per-entry amax is the max over the chunks'
+    amaxes, then every chunk is quantized with that amax supplied (the same
+    result as one call on the whole entry, since each block depends only on
+    its values and S_t).  Returns the per-entry lists of chunk outputs."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    tasks = []
+    for e, x in enumerate(entries):
+        rows = x.shape[-2]
+        for r0 in range(0, rows, chunk_rows):
+            tasks.append((e, r0, min(rows, r0 + chunk_rows)))
+
+    def _amax(t):
+        e, r0, r1 = t
+        return amax(np.ascontiguousarray(entries[e][..., r0:r1, :]).reshape(1, r1 - r0, -1),
+                    rht=kw.get("rht", False), seed=kw.get("seed", 0))[0]
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        part = list(ex.map(_amax, tasks))
+        A = np.zeros(len(entries), np.float32)
+        for (e, _, _), a in zip(tasks, part):
+            A[e] = max(A[e], a)
+
+        def _quant(t):
+            e, r0, r1 = t
+            xs = np.ascontiguousarray(entries[e][..., r0:r1, :]).reshape(1, r1 - r0, -1)
+            rows, cols = entries[e].shape[-2], entries[e].shape[-1]
+            return quantize(xs, amax_in=A[e:e + 1], elem_offset=(e * rows + r0) * cols, **kw)
+
+        outs = list(ex.map(_quant, tasks))
+    per = [[] for _ in entries]
+    for (e, _, _), o in zip(tasks, outs):
+        per[e].append(o)
+    return per
+
+
 def dequantize(codes: np.ndarray, scales: np.ndarray, tensor_scale: np.ndarray | None,
                fmt: int = FMT_NVFP4_46) -> np.ndarray:
     """codes [b,rows,cols/2], scales [b,rows,cols/bs] -> bf16 bits [b,rows,cols]."""

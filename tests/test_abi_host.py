@@ -38,6 +38,17 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def test_check_library_exports_every_declared_symbol():
+    """libfos_check.so (the tests' exhaustive device checks) exports what
+    include/fos_check.h declares."""
+    txt = open(os.path.join(ROOT, "include", "fos_check.h")).read()
+    declared = set(re.findall(r"^int\s+(fosck_\w+)\s*\(", txt, re.M))
+    assert len(declared) >= 10
+    C = ctypes.CDLL(fbuild.build_check())
+    for name in declared:
+        assert hasattr(C, name), name
+
+
 def test_version_and_strings(L):
     assert F.version() == 1
     assert F.status_string(0) == "ok"

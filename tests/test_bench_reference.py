@@ -22,3 +22,25 @@ def test_reference_arm_prints_one_json_line():
     assert d["steps"] == 1 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_gpus_n_launches_n_ranks():
+    """bench.py --gpus 2 without a launcher re-runs itself as 2 ranks under
+    torch.distributed.run; each rank sees WORLD_SIZE=2 and rank 0 prints one
+    line with n_gpus 2 (--dry-run: gloo, no GPU work)."""
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--dry-run", "--steps", "1"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["world_size_env"] == 2 and d["dry_run"]
+    ranks = sorted(ln for ln in r.stderr.splitlines() if ln.startswith("bench dry run"))
+    assert ranks == ["bench dry run: rank 0 of 2", "bench dry run: rank 1 of 2"], r.stderr[-2000:]
+
+
+def test_gpus_must_match_world_size():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--dry-run"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE" in (r.stderr + r.stdout)

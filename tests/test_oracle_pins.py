@@ -670,3 +670,18 @@ def test_swizzle_is_a_permutation_with_128x4_tiles():
     # one 128x4 tile spans exactly 512 contiguous bytes
     assert sorted(o[:128, :4].ravel().tolist()) == list(range(512))
     del lin
+
+
+def test_threaded_oracle_equals_one_call():
+    """The host-core timing helper (row chunks on threads, amax supplied)
+    gives the same bytes as one oracle call per entry."""
+    rng = np.random.default_rng(40)
+    xs = [_random_tensor(rng, 48, 64, kind)[0] for kind in ("normal", "outliers", "scaled")]
+    par = oracle.quantize_parallel(xs, threads=4, chunk_rows=16, rnd=oracle.RND_SR, seed=9)
+    whole = oracle.quantize(np.stack(xs), rnd=oracle.RND_SR, seed=9)
+    for e in range(len(xs)):
+        codes = np.concatenate([o["r_codes"][0] for o in par[e]])
+        scales = np.concatenate([o["r_scales"][0] for o in par[e]])
+        assert np.array_equal(codes, whole["r_codes"][e])
+        assert np.array_equal(scales, whole["r_scales"][e])
+        assert par[e][0]["tensor_scale"][0] == whole["tensor_scale"][e]

@@ -89,3 +89,34 @@ def test_static_scratch_rejects_batch_beyond_limit():
                                      ctypes.byref(rc), None, None,
                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 5  # FOS_ERR_WORKSPACE
+
+
+def test_static_scratch_limit_applies_only_to_calls_that_use_scratch():
+    """MXFP4 calls and calls with a caller-supplied amax need no scratch, so
+    they take a batch beyond the limit and match fos_quantize."""
+    dev = require_gpu()
+    batch = FOS_STATIC_MAX_BATCH + 3
+    x = _input((batch, 16, 32), 5, 1.0, dev)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    amax = F.amax(x)
+    for fmt, blk, use_amax in ((2, 2, False), (0, 0, True)):
+        name = "mxfp4" if fmt == 2 else "nvfp4_46"
+        block = "1x32" if fmt == 2 else "1x16"
+        outs = []
+        for static in (True, False):
+            r = zeroed_out(batch, 16, 32, name, block, 0, dev, batch * 16 * 2)
+            rc = r.c_struct()
+            args = (ctypes.c_void_p(x.data_ptr()), batch, 16, 32, 32, ctypes.byref(Options(fmt, blk, 0, 0, 0, 0)),
+                    ctypes.c_void_p(amax.data_ptr()) if use_amax else None, ctypes.byref(rc), None)
+            if static:
+                st = F.lib().fos_quantize_static(*args, None, stream)
+            else:
+                st = F.lib().fos_quantize(*args, None, 0, None, stream)
+            assert st == 0, F.status_string(st)
+            outs.append(r)
+        torch.cuda.synchronize()
+        for name_ in ("codes", "scales"):
+            assert torch.equal(getattr(outs[0], name_), getattr(outs[1], name_)), name_
+        if fmt == 0:
+            assert torch.equal(outs[0].tensor_scale, outs[1].tensor_scale)
+            assert torch.equal(outs[0].choice, outs[1].choice)
