@@ -43,6 +43,19 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def fp4_peak_tflops():
+    """Dense FP4 tensor peak: the measured bf16 GEMM peak (burst) times the
+    nominal FP4 : bf16 ratio of 4 (9 : 2.25 PFLOP/s dense); fallback 1590 TF/s
+    bf16 when no measurement is present."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return 4.0 * float(d["bf16_tflops"]), "measured bf16_tflops x 4"
+    return 4.0 * 1590.0, "fallback 1590 TF/s bf16 x 4"
+
+
 # ------------------------------------------------------------------ dist
 def relaunch_as_ranks(n: int) -> int:
     """Run this same command as n ranks, one process per GPU, under
@@ -311,8 +324,8 @@ def run_fos(args, world, rank):
                    "l2": "input %.2f GB > 126 MB L2; no flush needed" % (2 * elems / 1e9)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic("k_q1x16_fused_moe_experts", elems),
-                     "kernel": "k_q1x16_fused<4/6, RNE> (per-expert amax + quantize)",
+                     "traffic": profiled_traffic("k_q1x16_pipe_moe_experts", elems),
+                     "kernel": "k_q1x16_pipe<4/6, RNE> (per-expert amax + quantize, one cooperative launch)",
                      "kernel_ms": round(ms_per_step, 4),
                      "bytes_per_launch": int(elems * BYTES_PER_ELEM),
                      "quantize_only_ms": round(tq_ms, 4),
@@ -376,6 +389,9 @@ def measure_modes(args, world, x, dev, stream, peak):
         rec("moe_nvfp4_dequant", ms, BYTES_PER_ELEM_DEQ, elems)
         ms = time_loop(lambda: F.dequantize(rm, out=y), n, 3, world, stream) / n
         rec("moe_mxfp4_dequant", ms, 0.5 + 1 / 32 + 2, elems)
+        ms = time_loop(lambda: F.fake_quantize(x, out=y, workspace=ws), n, 3, world, stream) / n
+        rec("moe_nvfp4_46_fake_quant_step", ms, 4.0, elems,
+            "quantize + dequantize in one launch, bf16 in and out, per-expert amax in the step")
         del y, r6, rm, r46
     except Exception as e:  # report, do not hide
         res["moe_error"] = repr(e)
@@ -426,6 +442,26 @@ def measure_modes(args, world, x, dev, stream, peak):
         del g, r, c, r1
     except Exception as e:
         res["gradient_error"] = repr(e)
+    torch.cuda.empty_cache()
+    # NVFP4 block-scaled GEMM on the tensor cores, fed by the quantizer
+    try:
+        peak_tf, peak_src = fp4_peak_tflops()
+        for n_ in (4096, 8192):
+            g_ = torch.Generator(device=dev).manual_seed(0)
+            xa = torch.randn(n_, n_, generator=g_, device=dev).to(torch.bfloat16)
+            xb = torch.randn(n_, n_, generator=g_, device=dev).to(torch.bfloat16)
+            qa = F.quantize(xa, swizzle=True, choice=False)[0]
+            qb = F.quantize(xb, swizzle=True, choice=False)[0]
+            d_ = torch.empty(n_, n_, dtype=torch.bfloat16, device=dev)
+            ms = time_loop(lambda: F.gemm_nvfp4(qa, qb, out=d_), n, 3, world, stream) / n
+            tf = 2.0 * n_ ** 3 / (ms * 1e-3) / 1e12
+            res["gemm_nvfp4_%d" % n_] = {"ms": round(ms, 4), "TFLOP_s": round(tf, 1),
+                                         "frac": round(tf / peak_tf, 4), "peak_TFLOP_s": peak_tf,
+                                         "peak_source": peak_src, "shape": [n_, n_, n_],
+                                         "note": "bf16 out, 128x128 tiles, kind::mxf4nvf4"}
+            del xa, xb, qa, qb, d_
+    except Exception as e:
+        res["gemm_error"] = repr(e)
     torch.cuda.empty_cache()
     return res
 

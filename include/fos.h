@@ -170,6 +170,48 @@ fos_status fos_dequantize(const fos_qtensor* q, int32_t fmt, int64_t batch, int6
                           int64_t cols, uint32_t flags, void* y, int64_t ldy, void* stream);
 
 /*
+ * fos_fake_quantize -- quantize x and dequantize it again in one pass, with
+ * bf16 output y [batch][rows][ldy] (16-byte aligned, ldy % 8 == 0,
+ * ldy >= cols): y = fos_dequantize(fos_quantize(x)) bit for bit, without
+ * writing codes or scales.  This is the simulated-FP4 path ("fake
+ * quantization") that the Hugging Face transformers doc "Four Over Six"
+ * names for hardware without FP4 tensor cores (introduction), and the
+ * forward of quantization-aware training.
+ *  NVFP4 (4/6 or 6-only): blk 1X16 rowwise, RNE or SR, with or without
+ *    FOS_FLAG_RHT16 (y is then in the rotated domain, like fos_dequantize's);
+ *    the per-entry amax is amax_in or computed in the call (workspace as for
+ *    fos_quantize).
+ *  MXFP4: blk 1X32, RNE; no workspace.
+ *  16x16 tiles return FOS_ERR_UNSUPPORTED.  Other arguments and errors are
+ *  those of fos_quantize; NaN/Inf input sets FOS_STATUS_NONFINITE.
+ */
+fos_status fos_fake_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
+                             const fos_options* opt, const float* amax_in, void* y, int64_t ldy,
+                             void* workspace, size_t workspace_bytes, uint32_t* status, void* stream);
+
+/*
+ * fos_gemm_nvfp4 -- the FP4 matrix product the quantized tensors are made
+ * for, on the B200 tensor cores (tcgen05.mma kind::mxf4nvf4, 16-element
+ * E4M3 block scales, FP32 accumulation):
+ *   D[m][n] = (S_tA * S_tB) * sum_k A[m][k] * B[n][k]
+ * where A (M x K) and B (N x K) are rowwise NVFP4 quantizations along K
+ * from fos_quantize with FOS_FLAG_SCALE_SWIZZLED (a and b as filled by it,
+ * batch 1; 6-only and 4/6 alike: the 4/6 choice is already in the scales).
+ * Ultralytics glossary "FP4", "Inferencia e Treinamento FP4": FP4 matrix
+ * multiplication on Blackwell tensor cores.
+ *  a->codes [M][codes_ld] (codes_ld >= K/2, multiple of 16), a->scales the
+ *  swizzled [M][K/16] scales (fos_scales_size(M, K/16, swizzled) bytes),
+ *  a->tensor_scale one float; the same for b with N.  choice_bits unused.
+ *  d: [M][ldd] bf16 (out_dtype 0) or f32 (out_dtype 1), 16-byte aligned,
+ *  ldd >= N, ldd * element size a multiple of 16.
+ *  M and N multiples of 128, K a multiple of 256 (FOS_ERR_SHAPE otherwise).
+ *  A device-side wait that gives up sets FOS_STATUS_TIMEOUT in *status
+ *  (nullable); D is then unspecified.
+ */
+fos_status fos_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int64_t M, int64_t N, int64_t K,
+                          void* d, int64_t ldd, int32_t out_dtype, uint32_t* status, void* stream);
+
+/*
  * fos_quantize_static -- fos_quantize without a workspace argument, for
  * callers that cannot allocate device memory: code that runs inside a stream
  * capture (cudaMalloc cannot be captured), serving paths that must not

@@ -17,12 +17,14 @@ extern "C" {
  * computed in the call, so the fused amax + quantize kernel runs) with a
  * failure planted on the host side: the amax items of batch entry
  * `stall_entry` never count in, and every bounded wait of the kernel gives
- * up after `spin_limit` polls (about 128 ns apart) instead of about 2^23.
+ * up after `spin_limit` polls (each an L2 round trip plus a 128 ns sleep)
+ * instead of 2^21.
  *
- * Every quantize item of that entry therefore waits until its limit, sets
- * FOS_STATUS_TIMEOUT in *status (status must not be NULL to see it) and goes
- * on, so the launch still ends.  The other entries are quantized exactly as
- * by fos_quantize; the stalled entry's outputs are unspecified.  Arguments
+ * The first wait on that entry runs out, sets FOS_STATUS_TIMEOUT in *status
+ * (status must not be NULL to see it) and ends every other wait of the
+ * launch, so the launch still ends.  The entries before the stalled one are
+ * quantized exactly as by fos_quantize; the outputs of the stalled entry and
+ * of the entries after it are unspecified.  Arguments
  * are those of fos_quantize; stall_entry must be in [0, batch) and
  * spin_limit >= 1 (FOS_ERR_ARG otherwise); other formats and block modes
  * return FOS_ERR_UNSUPPORTED.

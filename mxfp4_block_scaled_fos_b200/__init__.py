@@ -5,6 +5,6 @@ ctypes binding that passes torch device buffers and the current stream to it.
 """
 from .fos import (  # noqa: F401
     FLAG_RHT16, FLAG_SCALE_SWIZZLED, STATUS_NONFINITE, STATUS_TIMEOUT, FosError, Options,
-    QTensor, amax, dequantize, lib, quantize, scales_size, status_string, version,
+    QTensor, amax, dequantize, fake_quantize, gemm_nvfp4, lib, quantize, scales_size, status_string, version,
     workspace_size,
 )

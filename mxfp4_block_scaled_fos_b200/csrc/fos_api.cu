@@ -20,12 +20,6 @@ FastDiv make_fastdiv(uint32_t d) {
 
 namespace {
 
-// 1: the fused amax + quantize path uses the queue-fed kernel of
-// fos_rowwise.cu instead of the cooperative pipeline of fos_pipe.cu
-#ifndef FOS_FUSED_QUEUE
-#define FOS_FUSED_QUEUE 1
-#endif
-
 constexpr uint32_t kUnitsQuant = 256 * 4;   // work units per CTA (tile kernels)
 constexpr uint32_t kBlocksRowwise = 256 * 8; // 16-element blocks per CTA (rowwise 1x16)
 constexpr uint32_t kUnitsAmax = 256 * 8;    // block pairs per CTA (amax pass)
@@ -77,7 +71,7 @@ size_t choice_bytes(int64_t nblocks) { return (size_t)(8 * ((nblocks + 63) / 64)
 
 // Test hooks of the fused kernel's bounded waits (fos_testing_quantize_stalled).
 struct WaitHooks {
-  uint32_t spin_limit = 1u << 23;
+  uint32_t spin_limit = 1u << 21;
   int stall_entry = -1;
 };
 
@@ -234,13 +228,22 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
   // bitmaps whose words are shared between CTAs are built with atomics on a
   // zeroed buffer.
   if (opt->blk == FOS_BLOCK_16X16) {
+#if FOS_2D_WARP
+    // the warp-based kernel sets every bit with an atomic on a zeroed bitmap
+    a.row.choice_aligned = a.col.choice_aligned = 0;
+#else
     // rowwise: a CTA writes whole bytes (8 tile columns of one tile row);
     // transposed copy: whole 32-bit words (32 tile rows of one tile column)
     a.row.choice_aligned = (cols / 16) % 8 == 0;
     a.col.choice_aligned = (rows / 16) % 32 == 0;
+#endif
   } else if (colwise) {
+#if FOS_DUAL_WARP
+    a.row.choice_aligned = a.col.choice_aligned = 0;  // atomics on zeroed bitmaps
+#else
     a.row.choice_aligned = (cols / 16) % 8 == 0;
     a.col.choice_aligned = (rows / 16) % 32 == 0;
+#endif
   }
   const int64_t nb_row = opt->blk == FOS_BLOCK_16X16 ? batch * (rows / 16) * (cols / 16)
                                                      : batch * rows * (cols / 16);
@@ -271,13 +274,8 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
     // one persistent launch: per-entry amax and quantize, pipelined so the
     // second read of each entry comes from L2
     if (cudaMemsetAsync(amax_ws, 0, 12 * round_up(batch, 64), st) != cudaSuccess) return FOS_ERR_CUDA;
-#if FOS_FUSED_QUEUE
     ce = launch_q1x16_fused(a, (int)batch, opt->fmt, sr, rht, swz, dense, amax_ws, done_ws, claim_ws,
                             st);
-#else
-    void* ring = (char*)workspace + 12 * round_up(batch, 64) + 256;
-    ce = launch_q1x16_pipe(a, (int)batch, opt->fmt, sr, rht, swz, dense, amax_ws, done_ws, ring, st);
-#endif
     if (ce == cudaSuccess) return FOS_OK;
     if (ce != cudaErrorNotSupported) return FOS_ERR_CUDA;
     (void)cudaGetLastError();  // fall back to the two-kernel path below
@@ -307,6 +305,103 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
 }  // namespace fos
 
 extern "C" {
+
+fos_status fos_fake_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
+                             const fos_options* opt, const float* amax_in, void* y, int64_t ldy,
+                             void* workspace, size_t workspace_bytes, uint32_t* status, void* stream) {
+  if (!opt || !x || !y) return FOS_ERR_NULL;
+  if (opt->fmt < 0 || opt->fmt > 2 || opt->blk < 0 || opt->blk > 2 || opt->rnd < 0 ||
+      opt->rnd > 1 || (opt->flags & ~(FOS_FLAG_RHT16 | FOS_FLAG_SCALE_SWIZZLED)))
+    return FOS_ERR_ARG;
+  if (batch < 0 || rows < 0 || cols < 0 || batch > 65535) return FOS_ERR_SHAPE;
+  const bool mx = opt->fmt == FOS_FMT_MXFP4;
+  const bool rht = (opt->flags & FOS_FLAG_RHT16) != 0;
+  const bool sr = opt->rnd == FOS_ROUND_SR;
+  if (mx != (opt->blk == FOS_BLOCK_1X32)) return FOS_ERR_UNSUPPORTED;
+  if (opt->blk == FOS_BLOCK_16X16) return FOS_ERR_UNSUPPORTED;
+  if (mx && (sr || rht)) return FOS_ERR_UNSUPPORTED;
+  const int64_t bs = mx ? 32 : 16;
+  if (cols % bs) return FOS_ERR_SHAPE;
+  if (sr && (opt->elem_offset < 0 || opt->elem_offset % 16)) return FOS_ERR_ARG;
+  if (!aligned(x, 16) || ld % 8 != 0 || !aligned(y, 16) || ldy % 8 != 0) return FOS_ERR_ALIGN;
+  if (ld < cols || ldy < cols) return FOS_ERR_SHAPE;
+  if (rows > 0 && cols > 0 && rows * (cols / 16) >= (1ll << 31)) return FOS_ERR_SHAPE;
+  const bool need_ws = !mx && !amax_in;
+  if (need_ws) {
+    if (!workspace || workspace_bytes < ws_bytes(batch)) return FOS_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return FOS_ERR_ALIGN;
+  }
+  if (amax_in && !aligned(amax_in, 4)) return FOS_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (batch == 0 || rows == 0 || cols == 0) return FOS_OK;
+
+  QuantArgs a;
+  a.x = (const uint16_t*)x;
+  a.ld = ld;
+  a.x_bs = rows * ld;
+  a.rows = (int)rows;
+  a.cols = (int)cols;
+  a.nblk = (uint32_t)(rows * (cols / bs));
+  a.bpr = make_fastdiv((uint32_t)(cols / bs));
+  a.amax_in = amax_in;
+  a.status = status;
+  a.seed = opt->seed;
+  a.elem_offset = opt->elem_offset;
+  a.y = (uint16_t*)y;
+  a.ldy = ldy;
+  a.y_bs = rows * ldy;
+  if (mx) {
+    a.units_per_cta = kUnitsMx;
+    return launch_fake_mx(a, (int)batch, st) == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;
+  }
+  const bool dense = ld == cols && ldy == cols && aligned(x, 32) && aligned(y, 32);
+  uint32_t* amax_ws = (uint32_t*)workspace;
+  a.amax_ws = amax_ws;
+  if (!amax_in) {  // the fused amax + (fake) quantize kernel, as in fos_quantize
+    uint32_t* done_ws = amax_ws + round_up(batch, 64);
+    uint32_t* claim_ws = done_ws + round_up(batch, 64);
+    if (cudaMemsetAsync(amax_ws, 0, 12 * round_up(batch, 64), st) != cudaSuccess) return FOS_ERR_CUDA;
+    cudaError_t ce = launch_q1x16_fused(a, (int)batch, opt->fmt, sr, rht, false, dense, amax_ws, done_ws,
+                                        claim_ws, st, true);
+    if (ce == cudaSuccess) return FOS_OK;
+    if (ce != cudaErrorNotSupported) return FOS_ERR_CUDA;
+    (void)cudaGetLastError();  // amax pass, then the fake quantizer
+    if (cudaMemsetAsync(amax_ws, 0, 4 * batch, st) != cudaSuccess) return FOS_ERR_CUDA;
+    QuantArgs am = a;
+    am.units_per_cta = kUnitsAmax;
+    if (launch_amax(am, (int)batch, rht, amax_ws, st) != cudaSuccess) return FOS_ERR_CUDA;
+  }
+  a.units_per_cta = kBlocksRowwise;
+  return launch_q1x16_rowwise(a, (int)batch, opt->fmt, sr, rht, false, dense, st, true) == cudaSuccess
+             ? FOS_OK : FOS_ERR_CUDA;
+}
+
+fos_status fos_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int64_t M, int64_t N, int64_t K,
+                          void* d, int64_t ldd, int32_t out_dtype, uint32_t* status, void* stream) {
+  if (!a || !b || !d) return FOS_ERR_NULL;
+  if (!a->codes || !a->scales || !a->tensor_scale || !b->codes || !b->scales || !b->tensor_scale)
+    return FOS_ERR_NULL;
+  if (out_dtype != 0 && out_dtype != 1) return FOS_ERR_ARG;
+  if (M < 0 || N < 0 || K < 0) return FOS_ERR_SHAPE;
+  if (M % 128 || N % 128 || K % 256) return FOS_ERR_SHAPE;
+  if (M > (1 << 24) || N > (1 << 24) || K > (1 << 24)) return FOS_ERR_SHAPE;
+  if (ldd < N) return FOS_ERR_SHAPE;
+  if (!aligned(a->codes, 16) || !aligned(b->codes, 16) || !aligned(a->scales, 16) || !aligned(b->scales, 16) ||
+      !aligned(d, 16) || !aligned(a->tensor_scale, 4) || !aligned(b->tensor_scale, 4))
+    return FOS_ERR_ALIGN;
+  if (a->codes_ld < K / 2 || b->codes_ld < K / 2) return FOS_ERR_SHAPE;
+  if (a->codes_ld % 16 || b->codes_ld % 16 || ldd % (out_dtype ? 4 : 8)) return FOS_ERR_ALIGN;
+  if (M == 0 || N == 0) return FOS_OK;
+  if (K == 0) {
+    const size_t es = out_dtype ? 4 : 2;
+    return cudaMemset2DAsync(d, (size_t)ldd * es, 0, (size_t)N * es, (size_t)M, (cudaStream_t)stream) == cudaSuccess
+               ? FOS_OK : FOS_ERR_CUDA;
+  }
+  const cudaError_t e = launch_gemm_nvfp4(a, b, (int)M, (int)N, (int)K, d, ldd, out_dtype, status,
+                                          (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return FOS_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;
+}
 
 fos_status fos_amax(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
                     const fos_options* opt, float* amax_out, uint32_t* status, void* stream) {
@@ -370,10 +465,11 @@ fos_status fos_dequantize(const fos_qtensor* q, int32_t fmt, int64_t batch, int6
   a.nblk = (uint32_t)(rows * (cols / bs));
   a.bpr = make_fastdiv((uint32_t)(cols / bs));
   a.units_per_cta = kUnitsDeq;
-  return launch_dequant(a, (int)batch, mx, (flags & FOS_FLAG_SCALE_SWIZZLED) != 0,
-                        (cudaStream_t)stream) == cudaSuccess
-             ? FOS_OK
-             : FOS_ERR_CUDA;
+  const bool swz = (flags & FOS_FLAG_SCALE_SWIZZLED) != 0;
+  const bool dense = !swz && q->codes_ld * 2 == cols && q->scales_ld * bs == cols && ldy == cols &&
+                     aligned(y, 32);
+  return launch_dequant(a, (int)batch, mx, swz, dense, (cudaStream_t)stream) == cudaSuccess ? FOS_OK
+                                                                                            : FOS_ERR_CUDA;
 }
 
 }  // extern "C"

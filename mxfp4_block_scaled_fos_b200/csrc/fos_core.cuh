@@ -402,6 +402,36 @@ __device__ __forceinline__ Cand1 candidate1_t(const float2 (&P)[8], const float4
   return r;
 }
 
+// Fake quantization of one block: the kept codes back to bf16 with the
+// dequantization rule y = bf16_RNE((q * float(s)) * S_t) (the first product
+// is exact), 16 values = 32 bytes to y.
+template <bool DENSE>
+__device__ __forceinline__ void store_fake_block(const QuantArgs& a, int b, uint32_t j, const uint32_t (&codes)[2],
+                                                 float s, float St) {
+  uint32_t h[8];
+  e2m1x8_to_h2(codes[0], h);
+  e2m1x8_to_h2(codes[1], h + 4);
+  const float2 s2 = make_float2(s, s), t2 = make_float2(St, St);
+  uint32_t o[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float2 q = make_float2(h_lo(h[k]), h_hi(h[k]));
+    q = mul2(mul2(q, s2), t2);
+    const __nv_bfloat162 r = __floats2bfloat162_rn(q.x, q.y);
+    o[k] = *reinterpret_cast<const uint32_t*>(&r);
+  }
+  uint16_t* yp;
+  if (DENSE) {
+    yp = a.y + (long long)b * a.y_bs + (long long)j * 16;
+  } else {
+    const uint32_t row = fdiv(j, a.bpr), cb = j - row * a.bpr.d;
+    yp = a.y + (long long)b * a.y_bs + (long long)row * a.ldy + (long long)cb * 16;
+  }
+  uint4* q4 = reinterpret_cast<uint4*>(yp);
+  q4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  q4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 __device__ __forceinline__ float tensor_scale_of(const QuantArgs& a, int b, bool f46) {
   const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_ws[b]);
   return __fdiv_rn(A, f46 ? 1792.0f : 2688.0f);
@@ -415,6 +445,16 @@ __device__ __forceinline__ void build_scale_table(float2* tab, float St) {
     const float E = __fmul_rn(e4m3_to_f32((uint32_t)c), St);
     const float inv = (E == 0.0f) ? 0.0f : fminf(__frcp_rn(E), kFltMax);
     tab[c] = make_float2(E, inv);
+  }
+}
+
+// The same table as (inv, inv, -E, -E) per code: the two packed operands of
+// the candidate step (candidate1_t) in one 16-byte load.
+__device__ __forceinline__ void build_scale_table4(float4* tab, float St) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float E = __fmul_rn(e4m3_to_f32((uint32_t)c), St);
+    const float inv = (E == 0.0f) ? 0.0f : fminf(__frcp_rn(E), kFltMax);
+    tab[c] = make_float4(inv, inv, -E, -E);
   }
 }
 

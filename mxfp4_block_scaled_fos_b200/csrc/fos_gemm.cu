@@ -1,0 +1,341 @@
+// fos_gemm.cu -- the consumer of the quantizer's output: an NVFP4
+// block-scaled GEMM on the sm_100a tensor cores,
+//   D[m][n] = (S_tA * S_tB) * sum_k A[m][k] * B[n][k],
+// with A and B given as packed E2M1 codes and E4M3 16-element block scales
+// in the tensor-core layout that fos_quantize writes with
+// FOS_FLAG_SCALE_SWIZZLED, and S_t their FP32 per-tensor scales.
+//
+// Sources: Ultralytics glossary "FP4", "Como funciona FP4" (NVFP4: 16
+// values, E4M3 block scale, FP32 tensor scale) and "Inferencia e
+// Treinamento FP4" (FP4 matrix multiplication on Blackwell tensor cores);
+// Hugging Face transformers doc "Four Over Six", introduction (the codes
+// feed FP4 GEMMs on Blackwell).
+//
+// One CTA computes a 128 x 128 tile of D with 6 warps:
+//   warp 0     TMA producer: per 256-wide K step, the A and B code tiles
+//              (128 rows x 128 bytes each, 128-byte swizzle) as 2D tensor
+//              copies and the four 512-byte scale atoms of each as one
+//              2 KB bulk copy, into a 4-stage shared-memory ring;
+//   warp 1     allocates the tensor memory; one thread copies the stage's
+//              scale atoms into tensor memory (tcgen05.cp 32x128b.warpx4)
+//              and issues the four K=64 tcgen05.mma of the stage
+//              (kind::mxf4nvf4, block16, f32 accumulator in tensor memory);
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp its
+//              32-lane quarter), scale by S_tA * S_tB, store bf16 or f32.
+// Every mbarrier wait is bounded: after the limit the kernel sets
+// FOS_STATUS_TIMEOUT, stops issuing work, waits (bounded) for its own copies
+// in flight, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "fos.h"
+#include "fos_internal.h"
+
+namespace fos {
+
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 256;      // BK in FP4 elements (128 bytes)
+constexpr int kStages = 4;
+constexpr int kTileA = BM * BK / 2;              // 16384 bytes
+constexpr int kTileB = BN * BK / 2;              // 16384 bytes
+constexpr int kSFTile = 2048;                    // 4 atoms of 128 rows x 4 scales
+constexpr uint32_t kStageTx = kTileA + kTileB + 2 * kSFTile;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;              // accumulator 128 + scale buffers 64
+constexpr uint32_t kColSFA = 128, kColSFB = 160; // + 16 * (k step & 1)
+constexpr uint32_t kWaitLimit = 1u << 22;        // polls of one mbarrier wait
+
+// dynamic shared memory layout (from a 1024-byte aligned base)
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kStages * kTileA;
+constexpr int kOffSFA = kOffB + kStages * kTileB;
+constexpr int kOffSFB = kOffSFA + kStages * kSFTile;
+constexpr int kOffBar = kOffSFB + kStages * kSFTile;   // full[S], empty[S], accum
+constexpr int kOffTmem = kOffBar + (2 * kStages + 1) * 8;
+constexpr int kOffFlag = kOffTmem + 8;
+constexpr int kSmemBytes = kOffFlag + 8 + 1024;        // + alignment slack
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+
+// Bounded wait for the phase with the given parity; false if it ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (tile base 1024-byte aligned).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Descriptor of one 512-byte scale atom (32 rows of 16 bytes, no swizzle,
+// 8-row groups 128 bytes apart) as the source of tcgen05.cp.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
+  return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(128 >> 4) << 32) |
+         ((uint64_t)1 << 46);
+}
+
+// Instruction descriptor: kind::mxf4nvf4, A and B E2M1, K-major, UE4M3
+// scales, M = 128, N = 128, K = 64 per instruction.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void umma(uint32_t tmem_c, uint64_t da, uint64_t db, uint32_t tsfa, uint32_t tsfb,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      :: "r"(tmem_c), "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate), "r"(tsfa), "r"(tsfb) : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+}
+
+struct GemmArgs {
+  const uint8_t* sfa;  // swizzled scales of A (E4M3)
+  const uint8_t* sfb;
+  const float* sta;    // S_t of A and of B
+  const float* stb;
+  void* d;
+  long long ldd;       // elements
+  int M, N, K;
+  int f32_out;
+  long long sf_col_tiles;  // K / 64 (4-scale column tiles per 128-row tile)
+  uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_nvfp4(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + kOffBar, bar_empty = bar_full + 8 * kStages, bar_acc = bar_empty + 8 * kStages;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+  volatile uint32_t* fail = reinterpret_cast<volatile uint32_t*>(smem + kOffFlag);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_n = blockIdx.x, tile_m = blockIdx.y;
+  const int ksteps = g.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_acc, 1);
+    *fail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {  // tensor memory for the accumulator and the scale buffers
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(sbase + kOffTmem), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // producer: stage s of k step kt, after the MMAs of k step kt - S freed it
+      int issued = 0;
+      for (int kt = 0; kt < ksteps && !*fail; ++kt) {
+        const int s = kt % kStages;
+        if (kt >= kStages && !mbar_wait(bar_empty + 8 * s, ((kt / kStages) - 1) & 1)) { *fail = 1; break; }
+        const uint32_t fb = bar_full + 8 * s;
+        mbar_expect_tx(fb, kStageTx);
+        tma_load_2d(sbase + kOffA + s * kTileA, &map_a, kt * (BK / 2), tile_m * BM, fb);
+        tma_load_2d(sbase + kOffB + s * kTileB, &map_b, kt * (BK / 2), tile_n * BN, fb);
+        // the 4 scale atoms of rows [128 tile, +128) and scale columns [16 kt, +16)
+        bulk_load(sbase + kOffSFA + s * kSFTile, g.sfa + ((long long)tile_m * g.sf_col_tiles + 4 * kt) * 512,
+                  kSFTile, fb);
+        bulk_load(sbase + kOffSFB + s * kSFTile, g.sfb + ((long long)tile_n * g.sf_col_tiles + 4 * kt) * 512,
+                  kSFTile, fb);
+        issued = kt + 1;
+      }
+      // before leaving, every copy this thread started must have landed
+      for (int kt = (issued > kStages ? issued - kStages : 0); kt < issued; ++kt)
+        if (!mbar_wait(bar_full + 8 * (kt % kStages), (kt / kStages) & 1)) *fail = 1;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int kt = 0; kt < ksteps; ++kt) {
+        const int s = kt % kStages;
+        if (*fail || !mbar_wait(bar_full + 8 * s, (kt / kStages) & 1)) { *fail = 1; break; }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t buf = 16u * (kt & 1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tmem_cp_sf(tmem + kColSFA + buf + 4 * j, desc_sf(sbase + kOffSFA + s * kSFTile + 512 * j));
+          tmem_cp_sf(tmem + kColSFB + buf + 4 * j, desc_sf(sbase + kOffSFB + s * kSFTile + 512 * j));
+        }
+        const uint64_t da = desc_sw128(sbase + kOffA + s * kTileA);
+        const uint64_t db = desc_sw128(sbase + kOffB + s * kTileB);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)  // K = 64 (32 bytes) per instruction
+          umma(tmem, da + 2 * j, db + 2 * j, tmem + kColSFA + buf + 4 * j, tmem + kColSFB + buf + 4 * j,
+               (kt | j) != 0);
+        umma_commit(bar_empty + 8 * s);  // the stage's smem is free once these MMAs are done
+      }
+      umma_commit(bar_acc);  // the accumulator is complete (or the loop stopped)
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) ..
+    const int q = warp & 3;
+    const bool ok = mbar_wait(bar_acc, 0);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (!ok) *fail = 1;
+    if (ok && !*fail) {
+      const float alpha = __fmul_rn(g.sta[0], g.stb[0]);
+      const long long row = (long long)tile_m * BM + 32 * q + lane;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+            "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+              "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+              "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+              "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+            : "r"(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        const long long col = (long long)tile_n * BN + c0;
+        if (g.f32_out) {
+          float4* dp = reinterpret_cast<float4*>(static_cast<float*>(g.d) + row * g.ldd + col);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dp[k] = make_float4(__fmul_rn(__uint_as_float(r[4 * k]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * k + 1]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * k + 2]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * k + 3]), alpha));
+        } else {
+          uint4* dp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.d) + row * g.ldd + col);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint32_t o[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[8 * k + 2 * h]), alpha),
+                                                              __fmul_rn(__uint_as_float(r[8 * k + 2 * h + 1]), alpha));
+              o[h] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            dp[k] = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 1) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
+  }
+  if (threadIdx.x == 0 && *fail && g.status) atomicOr(g.status, FOS_STATUS_TIMEOUT);
+}
+
+// ---------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D map over packed codes [rows][ld bytes]: boxes of 128 bytes x 128 rows,
+// 128-byte swizzle.
+bool make_code_map(CUtensorMap* m, const void* codes, long long rows, long long kbytes, long long ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, void* d,
+                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_code_map(&ma, a->codes, M, K / 2, a->codes_ld) || !make_code_map(&mb, b->codes, N, K / 2, b->codes_ld))
+    return cudaErrorNotSupported;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(k_gemm_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  GemmArgs g;
+  g.sfa = a->scales;
+  g.sfb = b->scales;
+  g.sta = a->tensor_scale;
+  g.stb = b->tensor_scale;
+  g.d = d;
+  g.ldd = ldd;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.f32_out = f32_out;
+  g.sf_col_tiles = K / 64;
+  g.status = status;
+  k_gemm_nvfp4<<<dim3(N / BN, M / BM), kThreads, kSmemBytes, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+}  // namespace fos

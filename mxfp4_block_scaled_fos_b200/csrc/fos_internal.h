@@ -5,7 +5,19 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "fos.h"
 #include "fos_device.cuh"
+
+// 1: 16x16 tiles by the warp-based kernel (k_2d_warp in fos_tiles.cu);
+// 0: the strip kernel (k_2d16x16)
+#ifndef FOS_2D_WARP
+#define FOS_2D_WARP 1
+#endif
+// 1: rowwise + colwise 1x16 by the warp-based kernel (k_dual_warp);
+// 0: the strip kernel (k_dual1x16)
+#ifndef FOS_DUAL_WARP
+#define FOS_DUAL_WARP 1
+#endif
 
 namespace fos {
 
@@ -41,12 +53,17 @@ struct QuantArgs {
   // product and fused into the following add
   float neg_zero = -0.0f;
   OutDesc row, col;
-  // Bounded waits of the fused kernel: polls (about 128 ns apart) before a
-  // wait gives up and reports FOS_STATUS_TIMEOUT.  stall_entry >= 0 is a test
+  // Bounded waits of the fused kernel: polls (each an L2 round trip plus a
+  // 128 ns sleep, about 2^21 polls to a second and a half) before a wait
+  // gives up and reports FOS_STATUS_TIMEOUT.  stall_entry >= 0 is a test
   // hook (fos_testing_quantize_stalled): that entry's amax items never count
   // in, so every wait on it runs out.
-  uint32_t spin_limit = 1u << 23;
+  uint32_t spin_limit = 1u << 21;
   int stall_entry = -1;
+  // fake quantization (fos_fake_quantize): bf16 output y [batch][rows][ldy]
+  // instead of codes and scales
+  uint16_t* y = nullptr;
+  long long ldy = 0, y_bs = 0;
 };
 
 FastDiv make_fastdiv(uint32_t d);
@@ -54,27 +71,28 @@ FastDiv make_fastdiv(uint32_t d);
 // Kernel launchers (return the launch's cudaError_t).
 cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_ws,
                         cudaStream_t st);
+// fake: write the dequantized bf16 values to a.y instead of codes and scales
 cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
-                                 bool swz, bool dense, cudaStream_t st);
+                                 bool swz, bool dense, cudaStream_t st, bool fake = false);
 // fused per-entry amax + rowwise quantize (one persistent launch fed by a
 // work queue); amax_ws, done_a: one zeroed word per batch entry, queue: one
 // zeroed counter.  Returns cudaErrorNotSupported when it cannot be launched.
 cudaError_t launch_q1x16_fused(const QuantArgs& a, int batch, int fmt, bool sr, bool rht, bool swz,
                                bool dense, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue,
-                               cudaStream_t st);
-// The same as one cooperative launch with a static schedule and no work
-// queue (fos_pipe.cu): amax_ws, cnt: one zeroed word per batch entry; ring:
-// pipe_ring_bytes() of 16-byte aligned workspace (no initialisation needed).
-// Returns cudaErrorNotSupported when the grid cannot be co-resident.
-cudaError_t launch_q1x16_pipe(const QuantArgs& a, int batch, int fmt, bool sr, bool rht, bool swz,
-                              bool dense, uint32_t* amax_ws, uint32_t* cnt, void* ring, cudaStream_t st);
-size_t pipe_ring_bytes();
+                               cudaStream_t st, bool fake = false);
+// MXFP4 fake quantization (bf16 out); the NVFP4 one runs through the rowwise
+// launchers with fake = true.
+cudaError_t launch_fake_mx(const QuantArgs& a, int batch, cudaStream_t st);
 
-// Workspace bytes of fos_quantize for `batch` entries: per-entry words
-// (amax, counters, one spare array) then the pipeline's record ring.
-constexpr size_t kRingBytesMax = 16384;
+// NVFP4 block-scaled GEMM on the tensor cores (fos_gemm.cu); shapes checked
+// by the caller (M, N multiples of 128, K of 256).
+cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, void* d,
+                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st);
+
+// Workspace bytes of fos_quantize for `batch` entries: per-entry amax words,
+// per-entry completion counters and the fused kernel's queue counter.
 constexpr size_t workspace_bytes_for(long long batch) {
-  return (size_t)(12 * ((batch + 63) / 64 * 64) + 256) + kRingBytesMax;
+  return (size_t)(12 * ((batch + 63) / 64 * 64) + 256);
 }
 
 cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
@@ -97,6 +115,8 @@ struct DequantArgs {
   uint32_t units_per_cta = 0;
 };
 
-cudaError_t launch_dequant(const DequantArgs& a, int batch, bool mx, bool swz, cudaStream_t st);
+// dense: codes rows contiguous (codes_ld = cols/2), linear scales with
+// scales_ld = cols/bs, y rows contiguous (ldy = cols), 32-byte aligned y
+cudaError_t launch_dequant(const DequantArgs& a, int batch, bool mx, bool swz, bool dense, cudaStream_t st);
 
 }  // namespace fos

@@ -144,7 +144,7 @@ __device__ __forceinline__ void store_choice32(const OutDesc& o, unsigned long l
 // block) -> codes, scale byte, 4-picked flag.  FAST: the tensor scale's
 // division shortcut applies (known at compile time).
 template <bool F46, bool SR, bool RHT, int FAST>
-__device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float2* s_tab, const TScale& ts,
+__device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float4* s_tab, const TScale& ts,
                                               uint32_t mask16, float nz, unsigned long long seed,
                                               long long e0, uint32_t& bad, uint32_t (&codes)[2],
                                               uint32_t& sc, bool& pick) {
@@ -171,18 +171,18 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float2* s_tab
   bad |= (m >= 0x7f800000u);
   uint32_t s6, s4;
   cand_scales<F46, FAST>(__uint_as_float(m), ts, s6, s4);
-  const float2 t6 = s_tab[s6];
-  const Cand1 c6 = candidate1<F46>(P, t6.y, -t6.x, nz);
+  const float4 t6 = s_tab[s6];
+  const Cand1 c6 = candidate1_t<F46>(P, t6, nz);
   codes[0] = c6.c[0];
   codes[1] = c6.c[1];
   sc = s6;
-  float inv = t6.y;
+  float inv = t6.x;
   pick = false;
   if (F46) {
-    const float2 t4 = s_tab[s4];
-    const Cand1 c4 = candidate1<true>(P, t4.y, -t4.x, nz);
+    const float4 t4 = s_tab[s4];
+    const Cand1 c4 = candidate1_t<true>(P, t4, nz);
     pick = c4.err < c6.err;   // strictly lower wins; ties keep 6
-    if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.y; }
+    if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.x; }
   }
   if (SR) sr_block1(P, inv, sr_bytes16(seed, e0), codes);
 }
@@ -191,15 +191,15 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float2* s_tab
 // pointers, a branch-free tail (a lane past c1 recomputes block c1 - 1 and
 // stores nothing) and, when choice bits are asked for, a choice bitmap whose
 // words belong to one warp each (blocks per entry % 64 == 0, c0 % 32 == 0).
-template <bool F46, bool SR, bool RHT, int FAST, int NT = kThreads>
+template <bool F46, bool SR, bool RHT, int FAST, int NT = kThreads, bool FAKE = false>
 __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
-                                              const float2* s_tab, const TScale& ts, uint32_t mask16,
+                                              const float4* s_tab, const TScale& ts, uint32_t mask16,
                                               uint32_t& bad, unsigned long long pol) {
   const uint32_t lane = threadIdx.x & 31;
   const uint16_t* xb = a.x + (long long)b * a.x_bs;
   uint8_t* cb = a.row.codes + (long long)b * a.row.codes_bs;
   uint8_t* sb = a.row.scales + (long long)b * a.row.scales_bs;
-  uint32_t* chw = a.row.choice
+  uint32_t* chw = (!FAKE && a.row.choice)
                       ? reinterpret_cast<uint32_t*>(a.row.choice) + (((unsigned long long)b * a.nblk) >> 5)
                       : nullptr;
   const long long g0 = SR ? a.elem_offset + (long long)b * a.x_bs : 0;
@@ -215,11 +215,13 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
     bool pick;
     rowwise_block<F46, SR, RHT, FAST>(w, s_tab, ts, mask16, nz, seed, g0 + (long long)jj * 16, bad,
                                       codes, sc, pick);
-    if (valid) {
+    if (FAKE) {
+      if (valid) store_fake_block<true>(a, b, j, codes, e4m3_to_f32(sc), ts.St);
+    } else if (valid) {
       *reinterpret_cast<uint2*>(cb + (size_t)j * 8) = make_uint2(codes[0], codes[1]);
       sb[j] = (uint8_t)sc;
     }
-    if (F46 && chw) {
+    if (!FAKE && F46 && chw) {
       const uint32_t word = __ballot_sync(0xffffffffu, pick && valid);
       if (lane == 0) chw[g >> 5] = word;
     }
@@ -230,13 +232,13 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
 // takes block g + l for g = c0 + 32w, c0 + 32w + 256, ...  c0 must be a
 // multiple of 32 so that each 32-bit word of the choice bitmap belongs to one
 // warp.
-template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, int NT = kThreads>
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, int NT = kThreads, bool FAKE = false>
 __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
-                                              const float2* s_tab, const TScale& ts, uint32_t mask16,
+                                              const float4* s_tab, const TScale& ts, uint32_t mask16,
                                               uint32_t& bad, unsigned long long pol) {
   if (DENSE) {
-    if (ts.fast) rowwise_dense<F46, SR, RHT, 1, NT>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
-    else         rowwise_dense<F46, SR, RHT, 0, NT>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    if (ts.fast) rowwise_dense<F46, SR, RHT, 1, NT, FAKE>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    else         rowwise_dense<F46, SR, RHT, 0, NT, FAKE>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
     return;
   }
   const int lane = threadIdx.x & 31;
@@ -270,16 +272,16 @@ __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_
       bad |= (m >= 0x7f800000u);
       uint32_t s6, s4;
       cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
-      const float2 t6 = s_tab[s6];
-      const Cand1 c6 = candidate1<F46>(P, t6.y, -t6.x, a.neg_zero);
+      const float4 t6 = s_tab[s6];
+      const Cand1 c6 = candidate1_t<F46>(P, t6, a.neg_zero);
       uint32_t codes[2] = {c6.c[0], c6.c[1]};
       uint32_t sc = s6;
-      float inv = t6.y;
+      float inv = t6.x;
       if (F46) {
-        const float2 t4 = s_tab[s4];
-        const Cand1 c4 = candidate1<true>(P, t4.y, -t4.x, a.neg_zero);
+        const float4 t4 = s_tab[s4];
+        const Cand1 c4 = candidate1_t<true>(P, t4, a.neg_zero);
         pick = valid && (c4.err < c6.err);   // strictly lower wins; ties keep 6
-        if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.y; }
+        if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.x; }
       }
       if (SR) {
         const long long g0 = a.elem_offset + (long long)b * a.rows * a.cols;
@@ -292,22 +294,26 @@ __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_
         }
         sr_block1(P, inv, sr_bytes16(a.seed, e0), codes);
       }
-      if (valid) k1_store<SWZ, DENSE>(a, b, j, codes, sc);
+      if (FAKE) {
+        if (valid) store_fake_block<false>(a, b, j, codes, e4m3_to_f32(sc), ts.St);
+      } else if (valid) {
+        k1_store<SWZ, DENSE>(a, b, j, codes, sc);
+      }
     }
-    if (F46 && a.row.choice) {
+    if (!FAKE && F46 && a.row.choice) {
       const uint32_t word = __ballot_sync(0xffffffffu, pick);
       if (lane == 0) store_choice32(a.row, (unsigned long long)b * a.nblk + g, word);
     }
   }
 }
 
-template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE>
 __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_K1_MIN_BLOCKS)
     k_q1x16(const QuantArgs a) {
-  __shared__ float2 s_tab[128];
+  __shared__ float4 s_tab[128];
   const int b = blockIdx.y;
   const float St = tensor_scale_of(a, b, F46);
-  build_scale_table(s_tab, St);
+  build_scale_table4(s_tab, St);
   const TScale ts = make_tscale(St);
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[b] = St;
   uint32_t mask16 = 0;
@@ -322,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
                   l2_policy_evict_first());
   }
   uint32_t bad = 0;
-  rowwise_range<F46, SR, RHT, SWZ, DENSE>(a, b, c0, c1, s_tab, ts, mask16, bad,
-                                          DENSE ? l2_policy_evict_first() : 0ull);
+  rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, b, c0, c1, s_tab, ts, mask16, bad,
+                                                          DENSE ? l2_policy_evict_first() : 0ull);
   if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
@@ -361,6 +367,11 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 #endif
 #ifndef FOS_FUSED_QCHUNK
 #define FOS_FUSED_QCHUNK 1536
+#endif
+// 1: the CTA that claims an amax item starts a bulk L2 prefetch of its chunk
+// at claim time, so that the item itself reads from L2
+#ifndef FOS_FUSED_PREFETCH
+#define FOS_FUSED_PREFETCH 1
 #endif
 constexpr uint32_t kAChunk = FOS_FUSED_ACHUNK;  // blocks per amax item
 constexpr uint32_t kQChunk = FOS_FUSED_QCHUNK;  // blocks per quantize item (multiple of 32)
@@ -445,10 +456,10 @@ __device__ __forceinline__ FusedItem fused_item(uint32_t i, int batch, int L, ui
   return it;
 }
 
-template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE>
 __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_K1_MIN_BLOCKS)
     k_q1x16_fused(const QuantArgs a, int batch, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue) {
-  __shared__ float2 s_tab[128];
+  __shared__ float4 s_tab[128];
   __shared__ uint32_t s_red[kThreads / 32];
   __shared__ float s_St;
   __shared__ uint32_t s_item[2];
@@ -467,7 +478,21 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
   for (int k = 0;; k ^= 1) {
     const uint32_t i = s_item[k];
     if (i >= total) break;
-    if (threadIdx.x == 0) s_item[k ^ 1] = atomicAdd(queue, 1u);  // claim the next one now
+    if (threadIdx.x == 0) {  // claim the next item now
+      const uint32_t nx = atomicAdd(queue, 1u);
+      s_item[k ^ 1] = nx;
+#if FOS_FUSED_PREFETCH
+      if (DENSE && nx < total) {  // an amax chunk is read from HBM: start it into L2 now
+        const FusedItem ni = fused_item(nx, batch, L, na, nq);
+        if (ni.amax) {
+          const uint32_t lo = ni.chunk * kAChunk, hi = min(lo + kAChunk, a.nblk);
+          const char* base = reinterpret_cast<const char*>(a.x + (long long)ni.entry * a.x_bs + (long long)lo * 16);
+          for (uint32_t off = 0; off < (hi - lo) * 32u; off += 32768u)
+            prefetch_l2(base + off, min(32768u, (hi - lo) * 32u - off), pol_keep);
+        }
+      }
+#endif
+    }
     const FusedItem it = fused_item(i, batch, L, na, nq);
     if (it.amax) {
       const uint32_t lo = it.chunk * kAChunk, hi = min(lo + kAChunk, a.nblk);
@@ -495,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
           s_St = __fdiv_rn(A, F46 ? 1792.0f : 2688.0f);
         }
         __syncthreads();
-        build_scale_table(s_tab, s_St);
+        build_scale_table4(s_tab, s_St);
         __syncthreads();
         tab_entry = it.entry;
       }
@@ -503,7 +528,8 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
       const TScale ts = make_tscale(St);
       if (it.chunk == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[it.entry] = St;
       const uint32_t lo = it.chunk * kQChunk, hi = min(lo + kQChunk, a.nblk);
-      rowwise_range<F46, SR, RHT, SWZ, DENSE>(a, it.entry, lo, hi, s_tab, ts, mask16, bad, pol_done);
+      rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, it.entry, lo, hi, s_tab, ts, mask16, bad,
+                                                              pol_done);
     }
     __syncthreads();  // the next item is in s_item[k ^ 1]; s_red / s_tab may be rewritten
   }
@@ -561,38 +587,109 @@ __global__ void __launch_bounds__(kThreads) k_mxfp4(const QuantArgs a) {
 
 // --------------------------------------------------------------------------
 // Dequantize: NVFP4 y = bf16_rne((q * float(s)) * S_t); MXFP4 y = q * 2^(s-127).
-template <bool MX, bool SWZ>
+// One 16-element group per thread (an NVFP4 block, or half an MXFP4 block):
+// 8 code bytes in, 32 bytes of bf16 out.  DENSE: codes and y rows
+// contiguous, linear scales and a 32-byte aligned y, so group j sits at code
+// byte 8j and element 16j and is written with one 256-bit store (a warp
+// writes 1 KB of contiguous output per store instruction).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&o)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               :: "l"(p), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+               : "memory");
+}
+
+template <bool MX, bool SWZ, bool DENSE>
 __global__ void __launch_bounds__(kThreads) k_dequant(const DequantArgs a) {
   const int b = blockIdx.y;
+  constexpr uint32_t GPB = MX ? 2 : 1;  // 16-element groups per block
+  const uint32_t ngroups = a.nblk * GPB;
   const uint32_t u0 = blockIdx.x * a.units_per_cta;
-  const uint32_t u1 = min(u0 + a.units_per_cta, a.nblk);
+  const uint32_t u1 = min(u0 + a.units_per_cta, ngroups);
   const float St = MX ? 1.0f : a.tensor_scale[b];
-  constexpr int BS = MX ? 32 : 16;
+  const float2 t2 = make_float2(St, St);
   for (uint32_t j = u0 + threadIdx.x; j < u1; j += kThreads) {
-    const uint32_t row = fdiv(j, a.bpr);
-    const uint32_t cb = j - row * a.bpr.d;
+    const uint32_t blk = MX ? (j >> 1) : j;
+    uint32_t row, cb;
+    if (DENSE) {
+      row = 0;
+      cb = blk;
+    } else {
+      row = fdiv(blk, a.bpr);
+      cb = blk - row * a.bpr.d;
+    }
     long long so;
     if (SWZ) so = (long long)b * a.scales_bs + swz_offset(row, cb, a.col_tiles);
     else     so = (long long)b * a.scales_bs + (long long)row * a.scales_ld + cb;
     const uint32_t sc = a.scales[so];
     const float s = MX ? __uint_as_float(sc == 0 ? 0x00400000u : (sc << 23)) : e4m3_to_f32(sc);
-    const uint2* cp = reinterpret_cast<const uint2*>(a.codes + (long long)b * a.codes_bs +
-                                                     (long long)row * a.codes_ld +
-                                                     (long long)cb * (BS / 2));
-    uint4* yp = reinterpret_cast<uint4*>(a.y + (long long)b * a.y_bs + (long long)row * a.ldy +
-                                         (long long)cb * BS);
+    const long long goff = (long long)cb * (MX ? 2 : 1) + (MX ? (j & 1) : 0);  // group within the row
+    const uint2 cw = *reinterpret_cast<const uint2*>(a.codes + (long long)b * a.codes_bs +
+                                                     (long long)row * a.codes_ld + goff * 8);
+    uint32_t h[8];
+    e2m1x8_to_h2(cw.x, h);
+    e2m1x8_to_h2(cw.y, h + 4);
+    const float2 s2 = make_float2(s, s);
+    uint32_t o[8];
 #pragma unroll
-    for (int part = 0; part < BS / 16; ++part) {
-      const uint2 cw = cp[part];
+    for (int k = 0; k < 8; ++k) {
+      float2 q = mul2(make_float2(h_lo(h[k]), h_hi(h[k])), s2);
+      if (!MX) q = mul2(q, t2);
+      const __nv_bfloat162 r = __floats2bfloat162_rn(q.x, q.y);
+      o[k] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+    uint16_t* yp = a.y + (long long)b * a.y_bs + (long long)row * a.ldy + goff * 16;
+    if (DENSE) {  // 32-byte aligned
+      st_global_v8(yp, o);
+    } else {      // rows only 16-byte aligned
+      reinterpret_cast<uint4*>(yp)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<uint4*>(yp)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+// MXFP4 fake quantization: E = floor(log2 amax) - 2 per 32-block (clamped),
+// codes = E2M1_rne(w * 2^-E), y = bf16(q * 2^E) (exact).  grid (chunks, batch).
+__global__ void __launch_bounds__(kThreads) k_fake_mx(const QuantArgs a) {
+  const int b = blockIdx.y;
+  const uint32_t u0 = blockIdx.x * a.units_per_cta;
+  const uint32_t u1 = min(u0 + a.units_per_cta, a.nblk);
+  uint32_t bad = 0;
+  for (uint32_t j = u0 + threadIdx.x; j < u1; j += kThreads) {
+    const uint32_t row = fdiv(j, a.bpr);
+    const uint32_t cb = j - row * a.bpr.d;
+    const uint4* p = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs + (long long)row * a.ld +
+                                                   (long long)cb * 32);
+    uint4 w4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w4[k] = __ldg(p + k);
+    const uint4 lo[2] = {w4[0], w4[1]}, hi[2] = {w4[2], w4[3]};
+    const uint32_t am = max(amax_bits_bf16(lo), amax_bits_bf16(hi));
+    bad |= am >= 0x7f800000u;
+    const uint32_t ex = max(am >> 23, 2u);                     // biased exponent, >= 2
+    const float inv = __uint_as_float((256u - ex) << 23);      // 2^-E, E = ex - 129
+    const uint32_t sc = ex - 2u;                               // E + 127
+    const float sE = __uint_as_float(sc == 0 ? 0x00400000u : (sc << 23));  // 2^E
+    const float2 inv2 = make_float2(inv, inv), s2 = make_float2(sE, sE);
+    const uint32_t* w = &w4[0].x;
+    uint4* yp = reinterpret_cast<uint4*>(a.y + (long long)b * a.y_bs + (long long)row * a.ldy + (long long)cb * 32);
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float2 r = mul2(make_float2(bf_lo(w[8 * part + k]), bf_hi(w[8 * part + k])), inv2);
+        v[2 * k] = r.x;
+        v[2 * k + 1] = r.y;
+      }
+      const uint32_t c0 = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+      const uint32_t c1 = e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
       uint32_t h[8];
-      e2m1x8_to_h2(cw.x, h);
-      e2m1x8_to_h2(cw.y, h + 4);
+      e2m1x8_to_h2(c0, h);
+      e2m1x8_to_h2(c1, h + 4);
       uint32_t o[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        float2 q = make_float2(h_lo(h[k]), h_hi(h[k]));
-        q = mul2(q, make_float2(s, s));
-        if (!MX) q = mul2(q, make_float2(St, St));
+        const float2 q = mul2(make_float2(h_lo(h[k]), h_hi(h[k])), s2);
         const __nv_bfloat162 r = __floats2bfloat162_rn(q.x, q.y);
         o[k] = *reinterpret_cast<const uint32_t*>(&r);
       }
@@ -600,6 +697,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(const DequantArgs a) {
       yp[2 * part + 1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
   }
+  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
 }  // namespace
@@ -619,11 +717,24 @@ cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_
 }
 
 cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
-                                 bool swz, bool dense, cudaStream_t st) {
+                                 bool swz, bool dense, cudaStream_t st, bool fake) {
   const dim3 g = grid_for(a.nblk, a.units_per_cta, batch);
   const bool f46 = fmt == 0;
-  if (dense) swz = false;
-#define FOS_L(F, S, R, W, D) k_q1x16<F, S, R, W, D><<<g, kThreads, 0, st>>>(a)
+  if (dense || fake) swz = false;
+  if (fake) {
+#define FOS_L(F, S, R, D) k_q1x16<F, S, R, false, D, true><<<g, kThreads, 0, st>>>(a)
+#define FOS_D(F, S, R) do { if (dense) FOS_L(F, S, R, true); else FOS_L(F, S, R, false); } while (0)
+#define FOS_R(F, S) do { if (rht) FOS_D(F, S, true); else FOS_D(F, S, false); } while (0)
+#define FOS_S(F) do { if (sr) FOS_R(F, true); else FOS_R(F, false); } while (0)
+    if (f46) FOS_S(true);
+    else     FOS_S(false);
+#undef FOS_S
+#undef FOS_R
+#undef FOS_D
+#undef FOS_L
+    return cudaGetLastError();
+  }
+#define FOS_L(F, S, R, W, D) k_q1x16<F, S, R, W, D, false><<<g, kThreads, 0, st>>>(a)
 #define FOS_D(F, S, R, W) do { if (dense) FOS_L(F, S, R, W, true); else FOS_L(F, S, R, W, false); } while (0)
 #define FOS_W(F, S, R) do { if (swz) FOS_D(F, S, R, true); else FOS_D(F, S, R, false); } while (0)
 #define FOS_R(F, S) do { if (rht) FOS_W(F, S, true); else FOS_W(F, S, false); } while (0)
@@ -643,11 +754,11 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 // and cached; 0 = not yet known, -1 = the kernel cannot be resident.
 static constexpr int kMaxDevices = 64;
 
-template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE>
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE = false>
 static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_ws, uint32_t* done_a,
                                   uint32_t* queue, cudaStream_t st) {
   static std::atomic<int> grid_of[kMaxDevices];
-  auto kern = k_q1x16_fused<F46, SR, RHT, SWZ, DENSE>;
+  auto kern = k_q1x16_fused<F46, SR, RHT, SWZ, DENSE, FAKE>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
   int grid = grid_of[dev].load(std::memory_order_relaxed);
@@ -666,9 +777,21 @@ static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_
 
 cudaError_t launch_q1x16_fused(const QuantArgs& a, int batch, int fmt, bool sr, bool rht, bool swz,
                                bool dense, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool fake) {
   const bool f46 = fmt == 0;
-  if (dense) swz = false;
+  if (dense || fake) swz = false;
+  if (fake) {
+#define FOS_L(F, S, R, D) return launch_fused_t<F, S, R, false, D, true>(a, batch, amax_ws, done_a, queue, st)
+#define FOS_D(F, S, R) do { if (dense) FOS_L(F, S, R, true); else FOS_L(F, S, R, false); } while (0)
+#define FOS_R(F, S) do { if (rht) FOS_D(F, S, true); else FOS_D(F, S, false); } while (0)
+#define FOS_S(F) do { if (sr) FOS_R(F, true); else FOS_R(F, false); } while (0)
+    if (f46) FOS_S(true);
+    else     FOS_S(false);
+#undef FOS_S
+#undef FOS_R
+#undef FOS_D
+#undef FOS_L
+  }
 #define FOS_L(F, S, R, W, D) return launch_fused_t<F, S, R, W, D>(a, batch, amax_ws, done_a, queue, st)
 #define FOS_D(F, S, R, W) do { if (dense) FOS_L(F, S, R, W, true); else FOS_L(F, S, R, W, false); } while (0)
 #define FOS_W(F, S, R) do { if (swz) FOS_D(F, S, R, true); else FOS_D(F, S, R, false); } while (0)
@@ -690,15 +813,23 @@ cudaError_t launch_mxfp4(const QuantArgs& a, int batch, bool swz, cudaStream_t s
   return cudaGetLastError();
 }
 
-cudaError_t launch_dequant(const DequantArgs& a, int batch, bool mx, bool swz, cudaStream_t st) {
-  const dim3 g = grid_for(a.nblk, a.units_per_cta, batch);
-  if (mx) {
-    if (swz) k_dequant<true, true><<<g, kThreads, 0, st>>>(a);
-    else     k_dequant<true, false><<<g, kThreads, 0, st>>>(a);
-  } else {
-    if (swz) k_dequant<false, true><<<g, kThreads, 0, st>>>(a);
-    else     k_dequant<false, false><<<g, kThreads, 0, st>>>(a);
-  }
+cudaError_t launch_dequant(const DequantArgs& a, int batch, bool mx, bool swz, bool dense, cudaStream_t st) {
+  const dim3 g = grid_for(a.nblk * (mx ? 2 : 1), a.units_per_cta, batch);
+  if (swz) dense = false;
+#define FOS_L(M, W, D) k_dequant<M, W, D><<<g, kThreads, 0, st>>>(a)
+#define FOS_D(M, W) do { if (dense) FOS_L(M, W, true); else FOS_L(M, W, false); } while (0)
+#define FOS_W(M) do { if (swz) FOS_D(M, true); else FOS_D(M, false); } while (0)
+  if (mx) FOS_W(true);
+  else    FOS_W(false);
+#undef FOS_W
+#undef FOS_D
+#undef FOS_L
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fake_mx(const QuantArgs& a, int batch, cudaStream_t st) {
+  const dim3 g((a.nblk + a.units_per_cta - 1) / a.units_per_cta, (unsigned)batch, 1);
+  k_fake_mx<<<g, kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -125,6 +125,29 @@ __device__ __forceinline__ PairResult<F46> quant_pair(const float2 (&P)[16], uin
   return r;
 }
 
+// quant_pair with the (inv, inv, -E, -E) table of build_scale_table4.
+template <bool F46>
+__device__ __forceinline__ PairResult<F46> quant_pair4(const float2 (&P)[16], uint32_t ma, uint32_t mb,
+                                                       const TScale& St, const float4* tab, float nz) {
+  PairResult<F46> r;
+  uint32_t s6a, s4a, s6b, s4b;
+  cand_scales<F46>(__uint_as_float(ma), St, s6a, s4a);
+  cand_scales<F46>(__uint_as_float(mb), St, s6b, s4b);
+  const float4 t6a = tab[s6a], t6b = tab[s6b];
+  const Cand c6 = candidate<F46>(P, make_float2(t6a.x, t6b.x), make_float2(t6a.z, t6b.z), nz);
+  r.ca[0] = c6.ca[0]; r.ca[1] = c6.ca[1]; r.cb[0] = c6.cb[0]; r.cb[1] = c6.cb[1];
+  r.sa = s6a; r.sb = s6b; r.inva = t6a.x; r.invb = t6b.x; r.pa = 0; r.pb = 0;
+  if (F46) {
+    const float4 t4a = tab[s4a], t4b = tab[s4b];
+    const Cand c4 = candidate<true>(P, make_float2(t4a.x, t4b.x), make_float2(t4a.z, t4b.z), nz);
+    r.pa = c4.err.x < c6.err.x;
+    r.pb = c4.err.y < c6.err.y;
+    if (r.pa) { r.ca[0] = c4.ca[0]; r.ca[1] = c4.ca[1]; r.sa = s4a; r.inva = t4a.x; }
+    if (r.pb) { r.cb[0] = c4.cb[0]; r.cb[1] = c4.cb[1]; r.sb = s4b; r.invb = t4b.x; }
+  }
+  return r;
+}
+
 // --------------------------------------------------------------------------
 // 1x16 rowwise + colwise.  grid (ceil(cols/128), ceil(rows/512), batch).
 template <bool F46, bool SR, bool SWZ, bool ROW>
@@ -317,6 +340,305 @@ __device__ __forceinline__ unsigned long long zip_nibbles(uint32_t a, uint32_t b
 }
 
 // --------------------------------------------------------------------------
+// 1x16 rowwise + colwise from one read, warp-based.  grid (CTAs, batch);
+// every warp takes units of 4 horizontally adjacent 16x16 tiles, 8 lanes per
+// tile.  Lane i of a tile first holds the tile's rows 2i and 2i+1 as a pair
+// of rowwise blocks; the tile then goes through this warp's shared buffer so
+// that lane j holds its columns 2j and 2j+1 as a pair of colwise blocks.
+// With stochastic rounding the Philox bytes of each rowwise block (one call
+// per 16 consecutive elements) take the same way, so both orientations use
+// the byte of the same source element.  Choice bits go into zeroed bitmaps
+// with atomics.  No CTA barrier in the loop.
+constexpr int kDwGroup = 16 * 32 + 32;   // bytes per tile in the buffer: 16 rows of
+                                         // 32 bytes, padded so the 4 tiles' column
+                                         // reads fall into distinct banks
+#ifndef FOS_DUALW_MIN_BLOCKS
+#define FOS_DUALW_MIN_BLOCKS 3
+#endif
+
+// 4 bits at lanes i, 8+i, 16+i, 24+i of a ballot -> bits 0..3
+__device__ __forceinline__ uint32_t gather4(uint32_t bal, int i) {
+  const uint32_t x = bal >> i;
+  return (x & 1u) | ((x >> 7) & 2u) | ((x >> 14) & 4u) | ((x >> 21) & 8u);
+}
+
+__device__ __forceinline__ void or_bits(uint8_t* bitmap, unsigned long long bit, uint32_t v) {
+  if (!v) return;
+  unsigned int* wp = reinterpret_cast<unsigned int*>(bitmap) + (bit >> 5);
+  const unsigned long long vv = (unsigned long long)v << (bit & 31);
+  if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
+  if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
+}
+
+template <bool F46, bool SR, bool SWZ, bool ROW>
+__global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_DUALW_MIN_BLOCKS) k_dual_warp(const QuantArgs a, FastDiv ntc4) {
+  __shared__ __align__(16) float4 s_tab[128];
+  __shared__ __align__(16) uint8_t s_x[kThreads / 32][4 * kDwGroup];
+  __shared__ __align__(16) uint8_t s_r[SR ? kThreads / 32 : 1][SR ? 4 * 256 : 16];
+  const int b = blockIdx.y;
+  const float St = tensor_scale_of(a, b, F46);
+  build_scale_table4(s_tab, St);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
+    if (a.col.tensor_scale) a.col.tensor_scale[b] = St;
+  }
+  __syncthreads();
+  const TScale ts = make_tscale(St);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 3, i = lane & 7;
+  const uint32_t ntr = a.rows / 16, ntc = a.cols / 16;
+  const uint32_t nunits = ntr * ntc4.d;
+  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
+  uint8_t* xb = s_x[warp] + g * kDwGroup;
+  uint8_t* rbuf = SR ? s_r[warp] + g * 256 : nullptr;
+  uint32_t badmax = 0;
+  for (uint32_t u = blockIdx.x * (kThreads / 32) + warp; u < nunits; u += gridDim.x * (kThreads / 32)) {
+    const uint32_t trow = fdiv(u, ntc4), tq = u - trow * ntc4.d;
+    const uint32_t tc = tq * 4 + g;
+    const bool valid = tc < ntc;
+    const long long r0 = (long long)trow * 16 + 2 * i;
+    uint4 wa[2], wb[2];
+    if (valid) {
+      const uint4* pa = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs + r0 * a.ld + (long long)tc * 16);
+      const uint4* pb = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(pa) + a.ld);
+      wa[0] = __ldg(pa); wa[1] = __ldg(pa + 1);
+      wb[0] = __ldg(pb); wb[1] = __ldg(pb + 1);
+    } else {
+      wa[0] = wa[1] = wb[0] = wb[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // the tile into the warp's buffer (row r at byte 32 r), for the colwise pass
+    reinterpret_cast<uint4*>(xb + (2 * i) * 32)[0] = wa[0];
+    reinterpret_cast<uint4*>(xb + (2 * i) * 32)[1] = wa[1];
+    reinterpret_cast<uint4*>(xb + (2 * i + 1) * 32)[0] = wb[0];
+    reinterpret_cast<uint4*>(xb + (2 * i + 1) * 32)[1] = wb[1];
+    uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+    if (SR) {
+      ra = sr_bytes16(a.seed, gbase + r0 * a.cols + (long long)tc * 16);
+      rb = sr_bytes16(a.seed, gbase + (r0 + 1) * a.cols + (long long)tc * 16);
+      reinterpret_cast<uint4*>(rbuf)[2 * i] = ra;
+      reinterpret_cast<uint4*>(rbuf)[2 * i + 1] = rb;
+    }
+    // ---------------- rowwise: blocks (row 2i) and (row 2i+1) as a pair
+    uint32_t pra = 0, prb = 0;
+    if (ROW) {
+      float2 P[16];
+      unpack_pairs(wa, wb, P);
+      const uint32_t ma = amax_bits_bf16(wa), mb = amax_bits_bf16(wb);
+      badmax = max(badmax, max(ma, mb));
+      PairResult<F46> q = quant_pair4<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
+      if (SR) {
+        sr_block(P, 0, q.inva, ra, q.ca);
+        sr_block(P, 1, q.invb, rb, q.cb);
+      }
+      if (valid) {
+        store_codes8(a.row, b, r0, (long long)tc * 8, q.ca[0], q.ca[1]);
+        store_codes8(a.row, b, r0 + 1, (long long)tc * 8, q.cb[0], q.cb[1]);
+        a.row.scales[scale_off<SWZ>(a.row, b, r0, tc)] = (uint8_t)q.sa;
+        a.row.scales[scale_off<SWZ>(a.row, b, r0 + 1, tc)] = (uint8_t)q.sb;
+      }
+      pra = q.pa && valid;
+      prb = q.pb && valid;
+    }
+    __syncwarp();
+    // ---------------- colwise: columns 2i and 2i+1 of the tile as a pair
+    uint32_t pca = 0, pcb = 0;
+    {
+      uint32_t w[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) w[r] = *reinterpret_cast<const uint32_t*>(xb + r * 32 + 4 * i);
+      float2 P[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) P[r] = make_float2(bf_lo(w[r]), bf_hi(w[r]));
+      uint32_t h[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) h[k] = hmax_abs2(w[2 * k], w[2 * k + 1]);
+      const uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(h[0], h[1]), hmax_abs2(h[2], h[3])),
+                                   hmax_abs2(hmax_abs2(h[4], h[5]), hmax_abs2(h[6], h[7]))) & 0x7fff7fffu;
+      const uint32_t ma = (m & 0xffffu) << 16, mb = m & 0xffff0000u;
+      badmax = max(badmax, max(ma, mb));
+      PairResult<F46> q = quant_pair4<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
+      if (SR) {
+        uint32_t ba[16], bb[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const uint32_t two = *reinterpret_cast<const uint16_t*>(rbuf + r * 16 + 2 * i);
+          ba[r] = two & 0xffu;
+          bb[r] = two >> 8;
+        }
+        sr_block_bytes(P, 0, q.inva, ba, q.ca);
+        sr_block_bytes(P, 1, q.invb, bb, q.cb);
+      }
+      if (valid) {
+        const long long c0 = (long long)tc * 16 + 2 * i;
+        store_codes8(a.col, b, c0, (long long)trow * 8, q.ca[0], q.ca[1]);
+        store_codes8(a.col, b, c0 + 1, (long long)trow * 8, q.cb[0], q.cb[1]);
+        a.col.scales[scale_off<SWZ>(a.col, b, c0, trow)] = (uint8_t)q.sa;
+        a.col.scales[scale_off<SWZ>(a.col, b, c0 + 1, trow)] = (uint8_t)q.sb;
+      }
+      pca = q.pa && valid;
+      pcb = q.pb && valid;
+    }
+    __syncwarp();  // the buffers are rewritten by the next unit
+    if (F46) {
+      const uint32_t nbc = a.cols / 16;
+      if (ROW && a.row.choice) {  // rows r0, r0+1: 4 consecutive blocks (tiles tq*4 ..) each
+        const uint32_t ba = __ballot_sync(0xffffffffu, pra), bb = __ballot_sync(0xffffffffu, prb);
+        if (lane < 8) {
+          or_bits(a.row.choice, ((unsigned long long)b * a.rows + r0) * nbc + (unsigned long long)tq * 4,
+                  gather4(ba, i));
+          or_bits(a.row.choice, ((unsigned long long)b * a.rows + r0 + 1) * nbc + (unsigned long long)tq * 4,
+                  gather4(bb, i));
+        }
+      }
+      if (a.col.choice) {  // column c: block trow of [cols][rows/16]
+        const unsigned long long c0 = (unsigned long long)tc * 16 + 2 * i;
+        if (pca) or_bits(a.col.choice, ((unsigned long long)b * a.cols + c0) * ntr + trow, 1u);
+        if (pcb) or_bits(a.col.choice, ((unsigned long long)b * a.cols + c0 + 1) * ntr + trow, 1u);
+      }
+    }
+  }
+  badmax = __reduce_max_sync(0xffffffffu, badmax);
+  if (lane == 0 && badmax >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// --------------------------------------------------------------------------
+// 16x16 2D block scaling, warp-based.  grid (CTAs, batch); every warp takes
+// units of 4 horizontally adjacent tiles (tile row tr, tile columns 4u ..
+// 4u+3), 8 lanes per tile, lane i of a tile holding its rows 2i and 2i+1 as
+// the pair (A, B), loaded straight from global memory (32 bytes per row).
+// The tile amax and the tree over the 16 row error sums are 8-lane xor
+// shuffles; the transposed copy is zipped into bytes (rows 2i, 2i+1 of a
+// column) and transposed through this warp's own shared buffer, so the loop
+// has no CTA barrier.  Choice bits go into zeroed bitmaps with atomics.
+constexpr int kTrStride = 144;   // bytes between the 8-lane groups' rows in the
+                                 // transpose buffer: 9 x 16, so that the 4
+                                 // groups' reads fall into distinct banks
+#ifndef FOS_2DW_MIN_BLOCKS
+#define FOS_2DW_MIN_BLOCKS 3
+#endif
+
+template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
+__global__ void __launch_bounds__(kThreads, FOS_2DW_MIN_BLOCKS) k_2d_warp(const QuantArgs a, FastDiv ntc4) {
+  __shared__ __align__(16) float4 s_tab[128];
+  __shared__ __align__(16) uint8_t s_tr[kThreads / 32][4 * kTrStride];
+  const int b = blockIdx.y;
+  const float St = tensor_scale_of(a, b, F46);
+  build_scale_table4(s_tab, St);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
+    if (COL && a.col.tensor_scale) a.col.tensor_scale[b] = St;
+  }
+  __syncthreads();
+  const TScale ts = make_tscale(St);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 3, i = lane & 7;
+  const uint32_t ntr = a.rows / 16, ntc = a.cols / 16;
+  const uint32_t nunits = ntr * ntc4.d;
+  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
+  uint8_t* trb = s_tr[warp];
+  uint32_t badmax = 0;
+  for (uint32_t u = blockIdx.x * (kThreads / 32) + warp; u < nunits; u += gridDim.x * (kThreads / 32)) {
+    const uint32_t trow = fdiv(u, ntc4), tq = u - trow * ntc4.d;
+    const uint32_t tc = tq * 4 + g;
+    const bool valid = tc < ntc;  // uniform over the 8 lanes of a tile
+    const long long r0 = (long long)trow * 16 + 2 * i;
+    uint4 wa[2], wb[2];
+    if (valid) {
+      const uint4* pa = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs + r0 * a.ld + (long long)tc * 16);
+      const uint4* pb = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(pa) + a.ld);
+      wa[0] = __ldg(pa); wa[1] = __ldg(pa + 1);
+      wb[0] = __ldg(pb); wb[1] = __ldg(pb + 1);
+    } else {
+      wa[0] = wa[1] = wb[0] = wb[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    float2 P[16];
+    unpack_pairs(wa, wb, P);
+    uint32_t m = max(amax_bits_bf16(wa), amax_bits_bf16(wb));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    badmax = max(badmax, m);
+    uint32_t s6, s4;
+    cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
+    const float4 t6 = s_tab[s6];
+    const Cand c6 = candidate<F46>(P, make_float2(t6.x, t6.y), make_float2(t6.z, t6.w), a.neg_zero);
+    uint32_t ca[2] = {c6.ca[0], c6.ca[1]}, cb[2] = {c6.cb[0], c6.cb[1]};
+    uint32_t sc = s6;
+    float inv = t6.x;
+    bool pick = false;
+    if (F46) {
+      const float4 t4 = s_tab[s4];
+      const Cand c4 = candidate<true>(P, make_float2(t4.x, t4.y), make_float2(t4.z, t4.w), a.neg_zero);
+      // tree over the 16 row sums: rows (2i, 2i+1) here, then pairs of lanes
+      float e6 = __fadd_rn(c6.err.x, c6.err.y), e4 = __fadd_rn(c4.err.x, c4.err.y);
+#pragma unroll
+      for (int sh = 1; sh < 8; sh *= 2) {
+        e6 = __fadd_rn(e6, __shfl_xor_sync(0xffffffffu, e6, sh));
+        e4 = __fadd_rn(e4, __shfl_xor_sync(0xffffffffu, e4, sh));
+      }
+      pick = e4 < e6;  // strictly lower wins; ties keep 6
+      if (pick) { ca[0] = c4.ca[0]; ca[1] = c4.ca[1]; cb[0] = c4.cb[0]; cb[1] = c4.cb[1]; sc = s4; inv = t4.x; }
+    }
+    if (SR) {
+      sr_block(P, 0, inv, sr_bytes16(a.seed, gbase + r0 * a.cols + (long long)tc * 16), ca);
+      sr_block(P, 1, inv, sr_bytes16(a.seed, gbase + (r0 + 1) * a.cols + (long long)tc * 16), cb);
+    }
+    if (ROW && valid) {
+      store_codes8(a.row, b, r0, (long long)tc * 8, ca[0], ca[1]);
+      store_codes8(a.row, b, r0 + 1, (long long)tc * 8, cb[0], cb[1]);
+      a.row.scales[scale_off<SWZ>(a.row, b, r0, tc)] = (uint8_t)sc;
+      a.row.scales[scale_off<SWZ>(a.row, b, r0 + 1, tc)] = (uint8_t)sc;
+    }
+    if (COL) {
+      // byte c of lane i: column c of rows 2i (low nibble) and 2i+1 (high)
+      const unsigned long long lo = zip_nibbles(ca[0], cb[0]), hi = zip_nibbles(ca[1], cb[1]);
+      *reinterpret_cast<uint4*>(trb + g * kTrStride + i * 16) =
+          make_uint4((uint32_t)lo, (uint32_t)(lo >> 32), (uint32_t)hi, (uint32_t)(hi >> 32));
+      __syncwarp();
+      // lane i now takes columns 2i and 2i+1 of its tile: 8 bytes each, one
+      // per row pair
+      uint32_t v[8];
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) v[ii] = *reinterpret_cast<const uint16_t*>(trb + g * kTrStride + ii * 16 + 2 * i);
+      __syncwarp();
+      const uint32_t t01 = __byte_perm(v[0], v[1], 0x5140), t23 = __byte_perm(v[2], v[3], 0x5140);
+      const uint32_t t45 = __byte_perm(v[4], v[5], 0x5140), t67 = __byte_perm(v[6], v[7], 0x5140);
+      if (valid) {
+        const long long c0 = (long long)tc * 16 + 2 * i;
+        store_codes8(a.col, b, c0, (long long)trow * 8, __byte_perm(t01, t23, 0x5410), __byte_perm(t45, t67, 0x5410));
+        store_codes8(a.col, b, c0 + 1, (long long)trow * 8, __byte_perm(t01, t23, 0x7632),
+                     __byte_perm(t45, t67, 0x7632));
+        a.col.scales[scale_off<SWZ>(a.col, b, c0, trow)] = (uint8_t)sc;
+        a.col.scales[scale_off<SWZ>(a.col, b, c0 + 1, trow)] = (uint8_t)sc;
+      }
+    }
+    if (F46 && ((ROW && a.row.choice) || (COL && a.col.choice))) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, pick && valid && i == 0);
+      if (lane == 0 && bal) {
+        const uint32_t v4 = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u);
+        if (ROW && a.row.choice) {  // 4 consecutive tiles of tile row trow
+          const unsigned long long bit = ((unsigned long long)b * ntr + trow) * ntc + (unsigned long long)tq * 4;
+          unsigned int* wp = reinterpret_cast<unsigned int*>(a.row.choice) + (bit >> 5);
+          const unsigned long long vv = (unsigned long long)v4 << (bit & 31);
+          if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
+          if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
+        }
+        if (COL && a.col.choice) {  // tile (trow, tc) is tile (tc, trow) of x^T
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            if (!((v4 >> gg) & 1u)) continue;
+            const unsigned long long bit = ((unsigned long long)b * ntc + tq * 4 + gg) * ntr + trow;
+            atomicOr(reinterpret_cast<unsigned int*>(a.col.choice) + (bit >> 5), 1u << (bit & 31));
+          }
+        }
+      }
+    }
+  }
+  badmax = __reduce_max_sync(0xffffffffu, badmax);
+  if (lane == 0 && badmax >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// --------------------------------------------------------------------------
 // 16x16 2D block scaling.  grid (ceil(cols/128), ceil(rows/512), batch).
 // In a sub-tile, 8 threads own one 16x16 tile; thread i holds rows 2i, 2i+1
 // as the pair (A, B), so the per-row error trees come out of the pair code
@@ -490,10 +812,18 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
 
 cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
                               bool want_row, cudaStream_t st) {
+  const bool f46 = fmt == 0;
+#if FOS_DUAL_WARP
+  const uint32_t ntc4 = (uint32_t)((a.cols / 16 + 3) / 4);
+  const uint32_t units = (uint32_t)(a.rows / 16) * ntc4;
+  const FastDiv fd = make_fastdiv(ntc4);
+  const dim3 g(min((units + kThreads / 32 - 1) / (kThreads / 32), 148u * 8u), (unsigned)batch);
+#define FOS_L(F, S, W, R) k_dual_warp<F, S, W, R><<<g, kThreads, 0, st>>>(a, fd)
+#else
   const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * kStrip - 1) / (kSubRows * kStrip),
                (unsigned)batch);
-  const bool f46 = fmt == 0;
 #define FOS_L(F, S, W, R) k_dual1x16<F, S, W, R><<<g, kThreads, 0, st>>>(a)
+#endif
 #define FOS_R(F, S, W) do { if (want_row) FOS_L(F, S, W, true); else FOS_L(F, S, W, false); } while (0)
 #define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)
 #define FOS_S(F) do { if (sr) FOS_W(F, true); else FOS_W(F, false); } while (0)
@@ -508,10 +838,18 @@ cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, b
 
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz, bool want_row,
                           bool want_col, cudaStream_t st) {
+  const bool f46 = fmt == 0;
+#if FOS_2D_WARP
+  const uint32_t ntc4 = (uint32_t)((a.cols / 16 + 3) / 4);
+  const uint32_t units = (uint32_t)(a.rows / 16) * ntc4;
+  const FastDiv fd = make_fastdiv(ntc4);
+  const dim3 g(min((units + kThreads / 32 - 1) / (kThreads / 32), 148u * 8u), (unsigned)batch);
+#define FOS_L(F, S, W, R, C) k_2d_warp<F, S, W, R, C><<<g, kThreads, 0, st>>>(a, fd)
+#else
   const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * kStrip - 1) / (kSubRows * kStrip),
                (unsigned)batch);
-  const bool f46 = fmt == 0;
 #define FOS_L(F, S, W, R, C) k_2d16x16<F, S, W, R, C><<<g, kThreads, 0, st>>>(a)
+#endif
 #define FOS_C(F, S, W, R) do { if (want_col) FOS_L(F, S, W, R, true); else FOS_L(F, S, W, R, false); } while (0)
 #define FOS_R(F, S, W) do { if (want_row) FOS_C(F, S, W, true); else FOS_C(F, S, W, false); } while (0)
 #define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)

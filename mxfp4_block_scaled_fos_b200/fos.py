@@ -36,7 +36,7 @@ ERRORS = {
 # every symbol include/fos.h declares
 EXPORTS = ("fos_quantize", "fos_amax", "fos_dequantize", "fos_workspace_size",
            "fos_scales_size", "fos_status_string", "fos_version", "fos_quantize_static",
-           "fos_testing_quantize_stalled")
+           "fos_testing_quantize_stalled", "fos_fake_quantize", "fos_gemm_nvfp4")
 
 
 class Options(ctypes.Structure):
@@ -81,6 +81,12 @@ def lib(path: str = LIB_PATH):
     L.fos_testing_quantize_stalled.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options),
                                                ctypes.POINTER(QTensorC), P, ctypes.c_size_t, P,
                                                i32, u32, P]
+    L.fos_fake_quantize.restype = i32
+    L.fos_fake_quantize.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P, P, i64, P,
+                                    ctypes.c_size_t, P, P]
+    L.fos_gemm_nvfp4.restype = i32
+    L.fos_gemm_nvfp4.argtypes = [ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), i64, i64, i64, P, i64,
+                                 i32, P, P]
     L.fos_amax.restype = i32
     L.fos_amax.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P, P, P]
     L.fos_dequantize.restype = i32
@@ -211,6 +217,34 @@ def quantize(x: torch.Tensor, fmt: str = "nvfp4_46", block: Optional[str] = None
     return out_row, out_col
 
 
+def fake_quantize(x: torch.Tensor, fmt: str = "nvfp4_46", rounding: str = "rne", rht: bool = False,
+                  seed: int = 0, elem_offset: int = 0, amax: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Quantize and dequantize a CUDA bf16 tensor in one pass (bf16 out, same
+    shape): the simulated-FP4 forward, equal to dequantize(quantize(x))."""
+    x3 = _as3d(x)
+    if x3.dtype != torch.bfloat16 or not x3.is_cuda:
+        raise TypeError("x must be a CUDA bfloat16 tensor")
+    if x3.stride(-1) != 1 or x3.stride(0) != x3.shape[1] * x3.stride(1):
+        raise ValueError("x rows must be contiguous with batch stride rows * ld")
+    batch, rows, cols = x3.shape
+    block = "1x32" if fmt == "mxfp4" else "1x16"
+    opts = Options(FMT[fmt], BLK[block], RND[rounding], FLAG_RHT16 if rht else 0, seed, elem_offset)
+    if out is None:
+        out = torch.empty(batch, rows, cols, dtype=torch.bfloat16, device=x3.device)
+    out3 = _as3d(out)
+    if workspace is None and amax is None and fmt != "mxfp4":
+        workspace = torch.empty(workspace_size(batch, rows, cols, opts), dtype=torch.uint8, device=x3.device)
+    st = lib().fos_fake_quantize(
+        ctypes.c_void_p(x3.data_ptr()), batch, rows, cols, x3.stride(1), ctypes.byref(opts), _ptr(amax),
+        ctypes.c_void_p(out3.data_ptr()), out3.stride(1), _ptr(workspace),
+        workspace.numel() if workspace is not None else 0, _ptr(status), _stream(stream))
+    if st != 0:
+        raise FosError(st, "fos_fake_quantize")
+    return out
+
+
 def amax(x: torch.Tensor, rht: bool = False, seed: int = 0, out: Optional[torch.Tensor] = None,
          status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Per-batch-entry amax of |x| (of the 16-wide RHT of x when rht)."""
@@ -236,6 +270,28 @@ def dequantize(q: QTensor, out: Optional[torch.Tensor] = None, stream=None) -> t
                               out.stride(-2), _stream(stream))
     if st != 0:
         raise FosError(st, "fos_dequantize")
+    return out
+
+
+def gemm_nvfp4(a: QTensor, b: QTensor, out: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16,
+               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """D = (S_tA * S_tB) * A @ B^T on the tensor cores, for rowwise NVFP4
+    quantizations A [M, K] and B [N, K] with swizzled scales (batch 1)."""
+    if not (a.flags & FLAG_SCALE_SWIZZLED and b.flags & FLAG_SCALE_SWIZZLED):
+        raise ValueError("gemm_nvfp4 needs scales in the swizzled tensor-core layout")
+    if a.fmt == "mxfp4" or b.fmt == "mxfp4" or a.batch != 1 or b.batch != 1 or a.cols != b.cols:
+        raise ValueError("gemm_nvfp4 takes two NVFP4 [rows, K] operands with the same K")
+    M, N, K = a.rows, b.rows, a.cols
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=a.codes.device)
+    if out.dtype not in (torch.bfloat16, torch.float32) or out.stride(-1) != 1:
+        raise ValueError("out must be a row-contiguous bf16 or f32 tensor")
+    ac, bc = a.c_struct(), b.c_struct()
+    st = lib().fos_gemm_nvfp4(ctypes.byref(ac), ctypes.byref(bc), M, N, K, ctypes.c_void_p(out.data_ptr()),
+                              out.stride(0), 1 if out.dtype == torch.float32 else 0, _ptr(status),
+                              _stream(stream))
+    if st != 0:
+        raise FosError(st, "fos_gemm_nvfp4")
     return out
 
 

@@ -1,6 +1,6 @@
-"""Small, self-contained launches of one quantizer kernel for profiler captures.
+"""Small, self-contained launches of one kernel for profiler captures.
 
-    python -m mxfp4_block_scaled_fos_b200.profile_case --case moe46 --experts 8 --iters 3
+    python profile_case.py --case moe46 --experts 8 --iters 3
 
 Each case builds its synthetic input (the same recipes as the benchmark, at
 a reduced batch so a capture stays small), runs one untimed call, then
@@ -15,6 +15,8 @@ a reduced batch so a capture stays small), runs one untimed call, then
   act_rht   4/6 with the 16-wide RHT on activation rows (8192 x cols), amax supplied
   grad_dual 4/6 SR rowwise + colwise on Student-t gradients (rows x 8192)
   weight_2d 4/6 16x16 2D with the transposed copy on 0.02-normal weights (rows x 4096)
+  moe_fake  4/6 fake quantization (quantize + dequantize, bf16 out), amax in the call
+  gemm      NVFP4 block-scaled GEMM, rows x rows x rows (rows a multiple of 256)
 """
 from __future__ import annotations
 
@@ -22,8 +24,13 @@ import argparse
 
 import torch
 
-from . import fos as F
-from . import workloads
+import os
+import sys
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import mxfp4_block_scaled_fos_b200 as F  # noqa: E402
+from mxfp4_block_scaled_fos_b200 import workloads  # noqa: E402
 
 
 def main():
@@ -57,6 +64,10 @@ def main():
             q = F.quantize(x, amax=amax)[0]
             y = torch.empty_like(x)
             fn = lambda: F.dequantize(q, out=y)
+        elif c == "moe_fake":
+            ws = torch.empty(F.workspace_size(args.experts, 2880, 2880), dtype=torch.uint8, device=dev)
+            y = torch.empty_like(x)
+            fn = lambda: F.fake_quantize(x, out=y, workspace=ws)
         else:
             raise SystemExit("unknown case " + c)
     elif c == "act_rht":
@@ -74,6 +85,15 @@ def main():
         amax = F.amax(x)
         r, cc = F.quantize(x, block="16x16", colwise=True, amax=amax)
         fn = lambda: F.quantize(x, block="16x16", colwise=True, amax=amax, out_row=r, out_col=cc)
+    elif c == "gemm":
+        n = args.rows
+        g = torch.Generator(device=dev).manual_seed(0)
+        xa = torch.randn(n, n, generator=g, device=dev).to(torch.bfloat16)
+        xb = torch.randn(n, n, generator=g, device=dev).to(torch.bfloat16)
+        qa = F.quantize(xa, swizzle=True, choice=False)[0]
+        qb = F.quantize(xb, swizzle=True, choice=False)[0]
+        d = torch.empty(n, n, dtype=torch.bfloat16, device=dev)
+        fn = lambda: F.gemm_nvfp4(qa, qb, out=d)
     else:
         raise SystemExit("unknown case " + c)
     fn()

@@ -193,6 +193,22 @@ def test_dequantize_oracle_codes(fmt, swizzle):
     assert_bytes_equal(np_bits(y), ref, "dequantized")
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4_46", "mxfp4"])
+def test_dequantize_strided_output(fmt):
+    """Output rows 8 elements longer than the tensor (16-byte but not
+    32-byte aligned rows): the strided path, and nothing written past a row."""
+    dev = require_gpu()
+    batch, R, C = 2, 48, 320
+    x = _rand((batch, R, C), "heavy", 13, dev)
+    q = F.quantize(x, fmt=fmt)[0]
+    want = F.dequantize(q)
+    yf = torch.full((batch, R, C + 8), 3.0, dtype=torch.bfloat16, device=dev)
+    F.dequantize(q, out=yf[:, :, :C])
+    torch.cuda.synchronize()
+    assert torch.equal(yf[:, :, :C].view(torch.int16), want.view(torch.int16))
+    assert torch.all(yf[:, :, C:] == 3.0)
+
+
 # A block whose two candidate errors are exactly equal in binary32 (found in a
 # seeded Student-t tensor): the tie must keep 6.  Rows 0 and 1 carry the same
 # block in both halves of a pair, row 2 sets the tensor amax.
