@@ -324,8 +324,8 @@ def run_fos(args, world, rank):
                    "l2": "input %.2f GB > 126 MB L2; no flush needed" % (2 * elems / 1e9)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic("k_q1x16_pipe_moe_experts", elems),
-                     "kernel": "k_q1x16_pipe<4/6, RNE> (per-expert amax + quantize, one cooperative launch)",
+                     "traffic": profiled_traffic("k_q1x16_fused_moe_experts", elems),
+                     "kernel": "k_q1x16_fused<4/6, RNE> (per-expert amax + quantize, one persistent launch)",
                      "kernel_ms": round(ms_per_step, 4),
                      "bytes_per_launch": int(elems * BYTES_PER_ELEM),
                      "quantize_only_ms": round(tq_ms, 4),

@@ -11,7 +11,8 @@
 // Hugging Face transformers doc "Four Over Six", introduction (the codes
 // feed FP4 GEMMs on Blackwell).
 //
-// One CTA computes a 128 x 128 tile of D with 6 warps:
+// Persistent: one CTA per SM walks 128 x 128 tiles of D (grouped by 8 tile
+// rows for L2 reuse of B) with 6 warps:
 //   warp 0     TMA producer: per 256-wide K step, the A and B code tiles
 //              (128 rows x 128 bytes each, 128-byte swizzle) as 2D tensor
 //              copies and the four 512-byte scale atoms of each as one
@@ -22,6 +23,9 @@
 //              (kind::mxf4nvf4, block16, f32 accumulator in tensor memory);
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp its
 //              32-lane quarter), scale by S_tA * S_tB, store bf16 or f32.
+// The accumulator is double-buffered in tensor memory (2 x 128 columns), so
+// the epilogue of one tile runs while the MMAs of the next one are issued;
+// the shared-memory ring and its barriers run on across tiles.
 // Every mbarrier wait is bounded: after the limit the kernel sets
 // FOS_STATUS_TIMEOUT, stops issuing work, waits (bounded) for its own copies
 // in flight, frees its tensor memory and returns.
@@ -38,14 +42,15 @@ namespace fos {
 namespace {
 
 constexpr int BM = 128, BN = 128, BK = 256;      // BK in FP4 elements (128 bytes)
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kTileA = BM * BK / 2;              // 16384 bytes
 constexpr int kTileB = BN * BK / 2;              // 16384 bytes
 constexpr int kSFTile = 2048;                    // 4 atoms of 128 rows x 4 scales
 constexpr uint32_t kStageTx = kTileA + kTileB + 2 * kSFTile;
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 256;              // accumulator 128 + scale buffers 64
-constexpr uint32_t kColSFA = 128, kColSFB = 160; // + 16 * (k step & 1)
+constexpr uint32_t kTmemCols = 512;              // 2 accumulators of 128 + scale buffers 64
+constexpr uint32_t kColSFA = 256, kColSFB = 288; // + 16 * (k step & 1)
+constexpr int kGroupM = 8;                       // tile rows per group of the tile order
 constexpr uint32_t kWaitLimit = 1u << 22;        // polls of one mbarrier wait
 
 // dynamic shared memory layout (from a 1024-byte aligned base)
@@ -53,8 +58,8 @@ constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kTileA;
 constexpr int kOffSFA = kOffB + kStages * kTileB;
 constexpr int kOffSFB = kOffSFA + kStages * kSFTile;
-constexpr int kOffBar = kOffSFB + kStages * kSFTile;   // full[S], empty[S], accum
-constexpr int kOffTmem = kOffBar + (2 * kStages + 1) * 8;
+constexpr int kOffBar = kOffSFB + kStages * kSFTile;   // full[S], empty[S], acc_full[2], acc_empty[2]
+constexpr int kOffTmem = kOffBar + (2 * kStages + 4) * 8;
 constexpr int kOffFlag = kOffTmem + 8;
 constexpr int kSmemBytes = kOffFlag + 8 + 1024;        // + alignment slack
 
@@ -143,29 +148,45 @@ struct GemmArgs {
   uint32_t* status;
 };
 
+// Tile t of the persistent order -> (tile row, tile column): groups of
+// kGroupM tile rows, column-major inside a group.
+__device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int& tm, int& tn) {
+  const int per_group = kGroupM * ntn;
+  const int grp = t / per_group;
+  const int first = grp * kGroupM;
+  const int gm = min(kGroupM, ntm - first);
+  const int r = t - grp * per_group;
+  tm = first + r % gm;
+  tn = r / gm;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_nvfp4(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + kOffBar, bar_empty = bar_full + 8 * kStages, bar_acc = bar_empty + 8 * kStages;
+  const uint32_t bar_full = sbase + kOffBar, bar_empty = bar_full + 8 * kStages;
+  const uint32_t bar_accf = bar_empty + 8 * kStages, bar_acce = bar_accf + 16;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
   volatile uint32_t* fail = reinterpret_cast<volatile uint32_t*>(smem + kOffFlag);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile_n = blockIdx.x, tile_m = blockIdx.y;
   const int ksteps = g.K / BK;
+  const int ntm = g.M / BM, ntn = g.N / BN, ntiles = ntm * ntn;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_acc, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 4);  // one arrive per epilogue warp
+    }
     *fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {  // tensor memory for the accumulator and the scale buffers
+  if (warp == 1) {  // tensor memory for the accumulators and the scale buffers
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(sbase + kOffTmem), "r"(kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -177,57 +198,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // producer: stage s of k step kt, after the MMAs of k step kt - S freed it
-      int issued = 0;
-      for (int kt = 0; kt < ksteps && !*fail; ++kt) {
-        const int s = kt % kStages;
-        if (kt >= kStages && !mbar_wait(bar_empty + 8 * s, ((kt / kStages) - 1) & 1)) { *fail = 1; break; }
-        const uint32_t fb = bar_full + 8 * s;
-        mbar_expect_tx(fb, kStageTx);
-        tma_load_2d(sbase + kOffA + s * kTileA, &map_a, kt * (BK / 2), tile_m * BM, fb);
-        tma_load_2d(sbase + kOffB + s * kTileB, &map_b, kt * (BK / 2), tile_n * BN, fb);
-        // the 4 scale atoms of rows [128 tile, +128) and scale columns [16 kt, +16)
-        bulk_load(sbase + kOffSFA + s * kSFTile, g.sfa + ((long long)tile_m * g.sf_col_tiles + 4 * kt) * 512,
-                  kSFTile, fb);
-        bulk_load(sbase + kOffSFB + s * kSFTile, g.sfb + ((long long)tile_n * g.sf_col_tiles + 4 * kt) * 512,
-                  kSFTile, fb);
-        issued = kt + 1;
+      // producer: k step number `it` counts on across this CTA's tiles
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && !*fail; t += gridDim.x) {
+        int tm, tn;
+        tile_coords(t, ntm, ntn, tm, tn);
+        for (int kt = 0; kt < ksteps; ++kt, ++it) {
+          const int s = it % kStages;
+          if (it >= kStages && !mbar_wait(bar_empty + 8 * s, ((it / kStages) - 1) & 1)) { *fail = 1; break; }
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_expect_tx(fb, kStageTx);
+          tma_load_2d(sbase + kOffA + s * kTileA, &map_a, kt * (BK / 2), tm * BM, fb);
+          tma_load_2d(sbase + kOffB + s * kTileB, &map_b, kt * (BK / 2), tn * BN, fb);
+          // the 4 scale atoms of rows [128 tile, +128) and scale columns [16 kt, +16)
+          bulk_load(sbase + kOffSFA + s * kSFTile, g.sfa + ((long long)tm * g.sf_col_tiles + 4 * kt) * 512,
+                    kSFTile, fb);
+          bulk_load(sbase + kOffSFB + s * kSFTile, g.sfb + ((long long)tn * g.sf_col_tiles + 4 * kt) * 512,
+                    kSFTile, fb);
+        }
       }
       // before leaving, every copy this thread started must have landed
-      for (int kt = (issued > kStages ? issued - kStages : 0); kt < issued; ++kt)
-        if (!mbar_wait(bar_full + 8 * (kt % kStages), (kt / kStages) & 1)) *fail = 1;
+      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j)
+        if (!mbar_wait(bar_full + 8 * (j % kStages), (j / kStages) & 1)) *fail = 1;
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      for (int kt = 0; kt < ksteps; ++kt) {
-        const int s = kt % kStages;
-        if (*fail || !mbar_wait(bar_full + 8 * s, (kt / kStages) & 1)) { *fail = 1; break; }
+      int it = 0, lt = 0;
+      for (int t = blockIdx.x; t < ntiles && !*fail; t += gridDim.x, ++lt) {
+        const int acc = lt & 1;
+        // the epilogue must have drained this accumulator (tile lt - 2)
+        if (lt >= 2 && !mbar_wait(bar_acce + 8 * acc, ((lt >> 1) - 1) & 1)) { *fail = 1; break; }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t buf = 16u * (kt & 1);
+        const uint32_t tacc = tmem + (uint32_t)(acc * BN);
+        for (int kt = 0; kt < ksteps; ++kt, ++it) {
+          const int s = it % kStages;
+          if (*fail || !mbar_wait(bar_full + 8 * s, (it / kStages) & 1)) { *fail = 1; break; }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const uint32_t buf = 16u * (it & 1);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          tmem_cp_sf(tmem + kColSFA + buf + 4 * j, desc_sf(sbase + kOffSFA + s * kSFTile + 512 * j));
-          tmem_cp_sf(tmem + kColSFB + buf + 4 * j, desc_sf(sbase + kOffSFB + s * kSFTile + 512 * j));
+          for (int j = 0; j < 4; ++j) {
+            tmem_cp_sf(tmem + kColSFA + buf + 4 * j, desc_sf(sbase + kOffSFA + s * kSFTile + 512 * j));
+            tmem_cp_sf(tmem + kColSFB + buf + 4 * j, desc_sf(sbase + kOffSFB + s * kSFTile + 512 * j));
+          }
+          const uint64_t da = desc_sw128(sbase + kOffA + s * kTileA);
+          const uint64_t db = desc_sw128(sbase + kOffB + s * kTileB);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)  // K = 64 (32 bytes) per instruction
+            umma(tacc, da + 2 * j, db + 2 * j, tmem + kColSFA + buf + 4 * j, tmem + kColSFB + buf + 4 * j,
+                 (kt | j) != 0);
+          umma_commit(bar_empty + 8 * s);  // the stage's smem is free once these MMAs are done
         }
-        const uint64_t da = desc_sw128(sbase + kOffA + s * kTileA);
-        const uint64_t db = desc_sw128(sbase + kOffB + s * kTileB);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)  // K = 64 (32 bytes) per instruction
-          umma(tmem, da + 2 * j, db + 2 * j, tmem + kColSFA + buf + 4 * j, tmem + kColSFB + buf + 4 * j,
-               (kt | j) != 0);
-        umma_commit(bar_empty + 8 * s);  // the stage's smem is free once these MMAs are done
+        umma_commit(bar_accf + 8 * acc);  // this tile's accumulator is complete
       }
-      umma_commit(bar_acc);  // the accumulator is complete (or the loop stopped)
     }
   } else {
     // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) ..
     const int q = warp & 3;
-    const bool ok = mbar_wait(bar_acc, 0);
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (!ok) *fail = 1;
-    if (ok && !*fail) {
-      const float alpha = __fmul_rn(g.sta[0], g.stb[0]);
-      const long long row = (long long)tile_m * BM + 32 * q + lane;
+    const float alpha = __fmul_rn(g.sta[0], g.stb[0]);
+    int lt = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      const bool ok = mbar_wait(bar_accf + 8 * acc, (lt >> 1) & 1);
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      if (!ok) *fail = 1;
+      if (!ok || *fail) break;
+      int tm, tn;
+      tile_coords(t, ntm, ntn, tm, tn);
+      const long long row = (long long)tm * BM + 32 * q + lane;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t r[32];
@@ -239,9 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
               "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
               "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-            : "r"(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0));
+            : "r"(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN + c0)));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        const long long col = (long long)tile_n * BN + c0;
+        const long long col = (long long)tn * BN + c0;
         if (g.f32_out) {
           float4* dp = reinterpret_cast<float4*>(static_cast<float*>(g.d) + row * g.ldd + col);
 #pragma unroll
@@ -265,6 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // this warp is done reading the accumulator: the MMA warp may reuse it
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar_acce + 8 * acc) : "memory");
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -334,7 +375,12 @@ cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M,
   g.f32_out = f32_out;
   g.sf_col_tiles = K / 64;
   g.status = status;
-  k_gemm_nvfp4<<<dim3(N / BN, M / BM), kThreads, kSmemBytes, st>>>(ma, mb, g);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return cudaErrorNotSupported;
+  const int ntiles = (M / BM) * (N / BN);
+  k_gemm_nvfp4<<<dim3(ntiles < sms ? ntiles : sms), kThreads, kSmemBytes, st>>>(ma, mb, g);
   return cudaGetLastError();
 }
 

@@ -168,7 +168,7 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float4* s_tab
   } else {
     m = amax_bits_bf16(w);
   }
-  bad |= (m >= 0x7f800000u);
+  bad = max(bad, m);  // largest amax bits seen: >= 0x7f800000 means NaN/Inf
   uint32_t s6, s4;
   cand_scales<F46, FAST>(__uint_as_float(m), ts, s6, s4);
   const float4 t6 = s_tab[s6];
@@ -187,10 +187,14 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float4* s_tab
   if (SR) sr_block1(P, inv, sr_bytes16(seed, e0), codes);
 }
 
-// Dense rows (see k1_load): blocks [c0, c1) of entry b with per-entry base
-// pointers, a branch-free tail (a lane past c1 recomputes block c1 - 1 and
-// stores nothing) and, when choice bits are asked for, a choice bitmap whose
-// words belong to one warp each (blocks per entry % 64 == 0, c0 % 32 == 0).
+// Dense rows (see k1_load): blocks [c0, c1) of entry b.  Whole warp groups
+// of 32 blocks run without tail checks: the lane's input, code and scale
+// addresses are 32-bit offsets from per-entry base pointers, every store is
+// unconditional and the 4/6 choice word is one ballot stored by lane 0.  A
+// partial last group (c1 - g < 32) runs once with a branch-free tail (a lane
+// past c1 recomputes block c1 - 1 and stores nothing).  With choice bits the
+// bitmap words must belong to one warp each (blocks per entry % 64 == 0,
+// c0 % 32 == 0).
 template <bool F46, bool SR, bool RHT, int FAST, int NT = kThreads, bool FAKE = false>
 __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
                                               const float4* s_tab, const TScale& ts, uint32_t mask16,
@@ -205,7 +209,28 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
   const long long g0 = SR ? a.elem_offset + (long long)b * a.x_bs : 0;
   const float nz = a.neg_zero;
   const unsigned long long seed = a.seed;
-  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += NT) {  // uniform per warp
+  uint32_t g = c0 + 32 * (threadIdx.x >> 5);  // uniform per warp
+#pragma unroll 1
+  for (; g + 32 <= c1; g += NT) {
+    const uint32_t j = g + lane;
+    uint4 w[2];
+    ld_block256_hint(xb + (size_t)j * 16, pol, w);
+    uint32_t codes[2], sc;
+    bool pick;
+    rowwise_block<F46, SR, RHT, FAST>(w, s_tab, ts, mask16, nz, seed, g0 + (long long)j * 16, bad, codes,
+                                      sc, pick);
+    if (FAKE) {
+      store_fake_block<true>(a, b, j, codes, e4m3_to_f32(sc), ts.St);
+    } else {
+      *reinterpret_cast<uint2*>(cb + (size_t)j * 8) = make_uint2(codes[0], codes[1]);
+      sb[j] = (uint8_t)sc;
+      if (F46 && chw) {
+        const uint32_t word = __ballot_sync(0xffffffffu, pick);
+        if (lane == 0) chw[g >> 5] = word;
+      }
+    }
+  }
+  if (g < c1) {  // the partial last group
     const uint32_t j = g + lane;
     const bool valid = j < c1;
     const uint32_t jj = valid ? j : c1 - 1;
@@ -217,13 +242,15 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
                                       codes, sc, pick);
     if (FAKE) {
       if (valid) store_fake_block<true>(a, b, j, codes, e4m3_to_f32(sc), ts.St);
-    } else if (valid) {
-      *reinterpret_cast<uint2*>(cb + (size_t)j * 8) = make_uint2(codes[0], codes[1]);
-      sb[j] = (uint8_t)sc;
-    }
-    if (!FAKE && F46 && chw) {
-      const uint32_t word = __ballot_sync(0xffffffffu, pick && valid);
-      if (lane == 0) chw[g >> 5] = word;
+    } else {
+      if (valid) {
+        *reinterpret_cast<uint2*>(cb + (size_t)j * 8) = make_uint2(codes[0], codes[1]);
+        sb[j] = (uint8_t)sc;
+      }
+      if (F46 && chw) {
+        const uint32_t word = __ballot_sync(0xffffffffu, pick && valid);
+        if (lane == 0) chw[g >> 5] = word;
+      }
     }
   }
 }
@@ -269,7 +296,7 @@ __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_
       } else {
         m = amax_bits_bf16(w);
       }
-      bad |= (m >= 0x7f800000u);
+      bad = max(bad, m);  // largest amax bits seen: >= 0x7f800000 means NaN/Inf
       uint32_t s6, s4;
       cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
       const float4 t6 = s_tab[s6];
@@ -330,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
   uint32_t bad = 0;
   rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, b, c0, c1, s_tab, ts, mask16, bad,
                                                           DENSE ? l2_policy_evict_first() : 0ull);
-  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+  if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
 // --------------------------------------------------------------------------
@@ -371,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 // 1: the CTA that claims an amax item starts a bulk L2 prefetch of its chunk
 // at claim time, so that the item itself reads from L2
 #ifndef FOS_FUSED_PREFETCH
-#define FOS_FUSED_PREFETCH 1
+#define FOS_FUSED_PREFETCH 0
 #endif
 constexpr uint32_t kAChunk = FOS_FUSED_ACHUNK;  // blocks per amax item
 constexpr uint32_t kQChunk = FOS_FUSED_QCHUNK;  // blocks per quantize item (multiple of 32)
@@ -533,7 +560,94 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
     }
     __syncthreads();  // the next item is in s_item[k ^ 1]; s_red / s_tab may be rewritten
   }
-  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+  if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// --------------------------------------------------------------------------
+// The same fused amax + quantize with the two kinds of work interleaved:
+// item (p, c) of the sequence takes the amax of chunk c of entry p (if p <
+// batch) and quantizes chunk c of entry p - L (if p >= L), chunks of kIChunk
+// blocks.  The amax chunk is started into L2 by a bulk prefetch at the
+// item's start and reduced after the quantize work, so its memory latency
+// hides behind that work instead of holding a CTA slot on its own.  Each
+// warp folds its amax into the entry's word and counts in (8 per item); the
+// quantize part waits (bounded) until all 8 * nc count-ins of its entry are
+// in.  The same no-deadlock argument as k_q1x16_fused holds: an item waits
+// only on items earlier in the sequence.
+#ifndef FOS_FUSED_ICHUNK
+#define FOS_FUSED_ICHUNK 1536
+#endif
+#ifndef FOS_FUSED_ILAG
+#define FOS_FUSED_ILAG 3
+#endif
+constexpr uint32_t kIChunk = FOS_FUSED_ICHUNK;
+
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE>
+__global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_K1_MIN_BLOCKS)
+    k_q1x16_fused2(const QuantArgs a, int batch, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue) {
+  __shared__ float4 s_tab[128];
+  __shared__ float s_St;
+  __shared__ uint32_t s_item[2];
+  const uint32_t mask16 = RHT ? rht_sign_mask(a.seed) : 0u;
+  const uint32_t nc = (a.nblk + kIChunk - 1) / kIChunk;
+  const int L = FOS_FUSED_ILAG;
+  const uint32_t total = (uint32_t)(batch + L) * nc;
+  const unsigned long long pol_keep = l2_policy_evict_last();   // amax reads: kept for the quantize
+  const unsigned long long pol_done = l2_policy_evict_first();  // quantize reads: last use
+  const uint32_t lane = threadIdx.x & 31;
+  uint32_t bad = 0;
+  int tab_entry = -1;
+
+  if (threadIdx.x == 0) s_item[0] = atomicAdd(queue, 1u);
+  __syncthreads();
+  for (int k = 0;; k ^= 1) {
+    const uint32_t i = s_item[k];
+    if (i >= total) break;
+    if (threadIdx.x == 0) s_item[k ^ 1] = atomicAdd(queue, 1u);  // claim the next one now
+    const int p = (int)(i / nc);
+    const uint32_t c = i - (uint32_t)p * nc;
+    const uint32_t lo = c * kIChunk, hi = min(lo + kIChunk, a.nblk);
+    const bool has_amax = p < batch;
+    if (DENSE && has_amax && threadIdx.x < 32) {  // the amax chunk into L2 now, 16 KB per lane
+      const uint32_t nbytes = (hi - lo) * 32u, off = lane * 16384u;
+      if (off < nbytes)
+        prefetch_l2(a.x + (long long)p * a.x_bs + (long long)lo * 16 + off / 2, min(16384u, nbytes - off),
+                    pol_keep);
+    }
+    const int q = p - L;
+    if (q >= 0) {
+      if (q != tab_entry) {
+        if (threadIdx.x == 0) {
+          wait_at_least(done_a + q, nc * (kThreads / 32), a.status, a.spin_limit);
+          const float A = __uint_as_float(__ldcg(amax_ws + q));
+          s_St = __fdiv_rn(A, F46 ? 1792.0f : 2688.0f);
+        }
+        __syncthreads();
+        build_scale_table4(s_tab, s_St);
+        __syncthreads();
+        tab_entry = q;
+      }
+      const float St = s_St;
+      const TScale ts = make_tscale(St);
+      if (!FAKE && c == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[q] = St;
+      rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, q, lo, hi, s_tab, ts, mask16, bad, pol_done);
+    }
+    if (has_amax) {
+      uint32_t m = slice_amax_bits<RHT, DENSE>(a, p, lo, hi, mask16, pol_keep);
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (lane == 0) {
+        if (m >= 0x7f800000u) {
+          if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+        } else if (m) {
+          atomicMax(amax_ws + p, m);
+        }
+        __threadfence();
+        if (p != a.stall_entry) atomicAdd(done_a + p, 1u);
+      }
+    }
+    __syncthreads();  // the next item is in s_item[k ^ 1]; s_tab may be rewritten
+  }
+  if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
 // --------------------------------------------------------------------------
@@ -555,7 +669,7 @@ __global__ void __launch_bounds__(kThreads) k_mxfp4(const QuantArgs a) {
     for (int k = 0; k < 4; ++k) w4[k] = __ldg(p + k);
     const uint4 lo[2] = {w4[0], w4[1]}, hi[2] = {w4[2], w4[3]};
     const uint32_t am = max(amax_bits_bf16(lo), amax_bits_bf16(hi));
-    bad |= am >= 0x7f800000u;
+    bad = max(bad, am);
     const uint32_t ex = max(am >> 23, 2u);          // biased exponent, >= 2
     const uint32_t scale = ex - 2u;                 // E + 127 with E = ex - 129
     const float inv = __uint_as_float((256u - ex) << 23);  // 2^-E
@@ -582,7 +696,7 @@ __global__ void __launch_bounds__(kThreads) k_mxfp4(const QuantArgs a) {
     else     so = (long long)b * a.row.scales_bs + (long long)row * a.row.scales_ld + cb;
     a.row.scales[so] = (uint8_t)scale;
   }
-  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+  if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
 // --------------------------------------------------------------------------
@@ -664,7 +778,7 @@ __global__ void __launch_bounds__(kThreads) k_fake_mx(const QuantArgs a) {
     for (int k = 0; k < 4; ++k) w4[k] = __ldg(p + k);
     const uint4 lo[2] = {w4[0], w4[1]}, hi[2] = {w4[2], w4[3]};
     const uint32_t am = max(amax_bits_bf16(lo), amax_bits_bf16(hi));
-    bad |= am >= 0x7f800000u;
+    bad = max(bad, am);
     const uint32_t ex = max(am >> 23, 2u);                     // biased exponent, >= 2
     const float inv = __uint_as_float((256u - ex) << 23);      // 2^-E, E = ex - 129
     const uint32_t sc = ex - 2u;                               // E + 127
@@ -697,7 +811,7 @@ __global__ void __launch_bounds__(kThreads) k_fake_mx(const QuantArgs a) {
       yp[2 * part + 1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
   }
-  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+  if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
 }  // namespace
@@ -754,11 +868,21 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 // and cached; 0 = not yet known, -1 = the kernel cannot be resident.
 static constexpr int kMaxDevices = 64;
 
+// 1: amax and quantize as separate queue items (k_q1x16_fused); 2: each item
+// does both (k_q1x16_fused2)
+#ifndef FOS_FUSED_MODE
+#define FOS_FUSED_MODE 1
+#endif
+
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE = false>
 static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_ws, uint32_t* done_a,
                                   uint32_t* queue, cudaStream_t st) {
   static std::atomic<int> grid_of[kMaxDevices];
+#if FOS_FUSED_MODE == 2
+  auto kern = k_q1x16_fused2<F46, SR, RHT, SWZ, DENSE, FAKE>;
+#else
   auto kern = k_q1x16_fused<F46, SR, RHT, SWZ, DENSE, FAKE>;
+#endif
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
   int grid = grid_of[dev].load(std::memory_order_relaxed);

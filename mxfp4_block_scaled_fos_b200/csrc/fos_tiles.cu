@@ -502,6 +502,147 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_DUALW_MIN_BLOCKS) k_dua
 }
 
 // --------------------------------------------------------------------------
+// 16x16 2D block scaling, one row per lane.  grid (CTAs, batch); every warp
+// takes units of 2 horizontally adjacent tiles (tile row tr, tile columns
+// 2u, 2u+1), 16 lanes per tile, lane r of a tile holding its row r as one
+// block of 8 split pairs -- the per-block arithmetic of the rowwise
+// quantizer.  The tile amax and the tree over the 16 row error sums (rows
+// (2i, 2i+1) first, then pairs of those: the R6 order) are 16-lane xor
+// shuffles.  For the transposed copy the even lanes zip their row with the
+// next (row 2i in the low nibbles, 2i+1 in the high) and the tile goes
+// through this warp's shared buffer (8 row pairs x 16 bytes), from which
+// lane j of the first 8 takes columns 2j and 2j+1.  No CTA barrier in the
+// loop; choice bits go into zeroed bitmaps with atomics.
+constexpr int kTrStride = 144;   // bytes between the tiles' rows in the per-warp
+                                 // transpose buffers: 9 x 16, so that reads of
+                                 // different tiles fall into distinct banks
+#ifndef FOS_2DR_MIN_BLOCKS
+#define FOS_2DR_MIN_BLOCKS 5
+#endif
+
+template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
+__global__ void __launch_bounds__(kThreads, SR ? 3 : FOS_2DR_MIN_BLOCKS) k_2d_row(const QuantArgs a, FastDiv ntc2) {
+  __shared__ __align__(16) float4 s_tab[128];
+  __shared__ __align__(16) uint8_t s_tr[kThreads / 32][2 * kTrStride];
+  const int b = blockIdx.y;
+  const float St = tensor_scale_of(a, b, F46);
+  build_scale_table4(s_tab, St);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
+    if (COL && a.col.tensor_scale) a.col.tensor_scale[b] = St;
+  }
+  __syncthreads();
+  const TScale ts = make_tscale(St);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = lane >> 4, r = lane & 15;
+  const uint32_t ntr = a.rows / 16, ntc = a.cols / 16;
+  const uint32_t nunits = ntr * ntc2.d;
+  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
+  const float nz = a.neg_zero;
+  uint8_t* trb = s_tr[warp] + h * kTrStride;
+  uint32_t badmax = 0;
+  for (uint32_t u = blockIdx.x * (kThreads / 32) + warp; u < nunits; u += gridDim.x * (kThreads / 32)) {
+    const uint32_t trow = fdiv(u, ntc2), tq = u - trow * ntc2.d;
+    const uint32_t tc = tq * 2 + h;
+    const bool valid = tc < ntc;  // uniform over the 16 lanes of a tile
+    const long long row = (long long)trow * 16 + r;
+    uint4 w[2];
+    if (valid) {
+      const uint4* px = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs + row * a.ld + (long long)tc * 16);
+      w[0] = __ldg(px);
+      w[1] = __ldg(px + 1);
+    } else {
+      w[0] = w[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    const uint32_t W8[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+    float2 P[8];
+    unpack_split(W8, P);
+    uint32_t m = amax_bits_bf16(w);
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
+    badmax = max(badmax, m);
+    uint32_t s6, s4;
+    cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
+    const float4 t6 = s_tab[s6];
+    const Cand1 c6 = candidate1_t<F46>(P, t6, nz);
+    uint32_t codes[2] = {c6.c[0], c6.c[1]};
+    uint32_t sc = s6;
+    float inv = t6.x;
+    bool pick = false;
+    if (F46) {
+      const float4 t4 = s_tab[s4];
+      const Cand1 c4 = candidate1_t<true>(P, t4, nz);
+      float e6 = c6.err, e4 = c4.err;  // this row's sums; then the tree over rows
+#pragma unroll
+      for (int sh = 1; sh < 16; sh *= 2) {
+        e6 = __fadd_rn(e6, __shfl_xor_sync(0xffffffffu, e6, sh));
+        e4 = __fadd_rn(e4, __shfl_xor_sync(0xffffffffu, e4, sh));
+      }
+      pick = e4 < e6;  // strictly lower wins; ties keep 6
+      if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.x; }
+    }
+    if (SR) sr_block1(P, inv, sr_bytes16(a.seed, gbase + row * a.cols + (long long)tc * 16), codes);
+    if (ROW && valid) {
+      store_codes8(a.row, b, row, (long long)tc * 8, codes[0], codes[1]);
+      a.row.scales[scale_off<SWZ>(a.row, b, row, tc)] = (uint8_t)sc;
+    }
+    if (COL) {
+      // the next row's codes, then byte c of an even lane = column c of rows
+      // (r, r+1)
+      const uint32_t n0 = __shfl_down_sync(0xffffffffu, codes[0], 1);
+      const uint32_t n1 = __shfl_down_sync(0xffffffffu, codes[1], 1);
+      if ((r & 1) == 0) {
+        const unsigned long long lo = zip_nibbles(codes[0], n0), hi = zip_nibbles(codes[1], n1);
+        *reinterpret_cast<uint4*>(trb + (r >> 1) * 16) =
+            make_uint4((uint32_t)lo, (uint32_t)(lo >> 32), (uint32_t)hi, (uint32_t)(hi >> 32));
+      }
+      __syncwarp();
+      if (r < 8) {  // lane r of the first 8: columns 2r, 2r+1, one byte per row pair
+        uint32_t v[8];
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii) v[ii] = *reinterpret_cast<const uint16_t*>(trb + ii * 16 + 2 * r);
+        const uint32_t t01 = __byte_perm(v[0], v[1], 0x5140), t23 = __byte_perm(v[2], v[3], 0x5140);
+        const uint32_t t45 = __byte_perm(v[4], v[5], 0x5140), t67 = __byte_perm(v[6], v[7], 0x5140);
+        if (valid) {
+          const long long c0 = (long long)tc * 16 + 2 * r;
+          store_codes8(a.col, b, c0, (long long)trow * 8, __byte_perm(t01, t23, 0x5410),
+                       __byte_perm(t45, t67, 0x5410));
+          store_codes8(a.col, b, c0 + 1, (long long)trow * 8, __byte_perm(t01, t23, 0x7632),
+                       __byte_perm(t45, t67, 0x7632));
+        }
+      }
+      if (valid) a.col.scales[scale_off<SWZ>(a.col, b, (long long)tc * 16 + r, trow)] = (uint8_t)sc;
+      __syncwarp();
+    }
+    if (F46 && ((ROW && a.row.choice) || (COL && a.col.choice))) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, pick && valid && r == 0);
+      if (lane == 0 && bal) {
+        const uint32_t v2 = (bal & 1u) | ((bal >> 15) & 2u);
+        if (ROW && a.row.choice) {  // 2 consecutive tiles of tile row trow
+          const unsigned long long bit = ((unsigned long long)b * ntr + trow) * ntc + (unsigned long long)tq * 2;
+          unsigned int* wp = reinterpret_cast<unsigned int*>(a.row.choice) + (bit >> 5);
+          const unsigned long long vv = (unsigned long long)v2 << (bit & 31);
+          if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
+          if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
+        }
+        if (COL && a.col.choice) {  // tile (trow, tc) is tile (tc, trow) of x^T
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            if (!((v2 >> gg) & 1u)) continue;
+            const unsigned long long bit = ((unsigned long long)b * ntc + tq * 2 + gg) * ntr + trow;
+            atomicOr(reinterpret_cast<unsigned int*>(a.col.choice) + (bit >> 5), 1u << (bit & 31));
+          }
+        }
+      }
+    }
+  }
+  badmax = __reduce_max_sync(0xffffffffu, badmax);
+  if (lane == 0 && badmax >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+}
+
+// --------------------------------------------------------------------------
 // 16x16 2D block scaling, warp-based.  grid (CTAs, batch); every warp takes
 // units of 4 horizontally adjacent tiles (tile row tr, tile columns 4u ..
 // 4u+3), 8 lanes per tile, lane i of a tile holding its rows 2i and 2i+1 as
@@ -510,9 +651,6 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_DUALW_MIN_BLOCKS) k_dua
 // shuffles; the transposed copy is zipped into bytes (rows 2i, 2i+1 of a
 // column) and transposed through this warp's own shared buffer, so the loop
 // has no CTA barrier.  Choice bits go into zeroed bitmaps with atomics.
-constexpr int kTrStride = 144;   // bytes between the 8-lane groups' rows in the
-                                 // transpose buffer: 9 x 16, so that the 4
-                                 // groups' reads fall into distinct banks
 #ifndef FOS_2DW_MIN_BLOCKS
 #define FOS_2DW_MIN_BLOCKS 3
 #endif
@@ -839,7 +977,13 @@ cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, b
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz, bool want_row,
                           bool want_col, cudaStream_t st) {
   const bool f46 = fmt == 0;
-#if FOS_2D_WARP
+#if FOS_2D_WARP == 2
+  const uint32_t ntc2 = (uint32_t)((a.cols / 16 + 1) / 2);
+  const uint32_t units = (uint32_t)(a.rows / 16) * ntc2;
+  const FastDiv fd = make_fastdiv(ntc2);
+  const dim3 g(min((units + kThreads / 32 - 1) / (kThreads / 32), 148u * 10u), (unsigned)batch);
+#define FOS_L(F, S, W, R, C) k_2d_row<F, S, W, R, C><<<g, kThreads, 0, st>>>(a, fd)
+#elif FOS_2D_WARP
   const uint32_t ntc4 = (uint32_t)((a.cols / 16 + 3) / 4);
   const uint32_t units = (uint32_t)(a.rows / 16) * ntc4;
   const FastDiv fd = make_fastdiv(ntc4);
