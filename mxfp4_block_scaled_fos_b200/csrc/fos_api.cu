@@ -228,22 +228,13 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
   // bitmaps whose words are shared between CTAs are built with atomics on a
   // zeroed buffer.
   if (opt->blk == FOS_BLOCK_16X16) {
-#if FOS_2D_WARP
-    // the warp-based kernel sets every bit with an atomic on a zeroed bitmap
-    a.row.choice_aligned = a.col.choice_aligned = 0;
-#else
     // rowwise: a CTA writes whole bytes (8 tile columns of one tile row);
     // transposed copy: whole 32-bit words (32 tile rows of one tile column)
     a.row.choice_aligned = (cols / 16) % 8 == 0;
     a.col.choice_aligned = (rows / 16) % 32 == 0;
-#endif
   } else if (colwise) {
-#if FOS_DUAL_WARP
-    a.row.choice_aligned = a.col.choice_aligned = 0;  // atomics on zeroed bitmaps
-#else
-    a.row.choice_aligned = (cols / 16) % 8 == 0;
-    a.col.choice_aligned = (rows / 16) % 32 == 0;
-#endif
+    // the warp-based kernel sets every bit with an atomic on a zeroed bitmap
+    a.row.choice_aligned = a.col.choice_aligned = 0;
   }
   const int64_t nb_row = opt->blk == FOS_BLOCK_16X16 ? batch * (rows / 16) * (cols / 16)
                                                      : batch * rows * (cols / 16);

@@ -63,10 +63,15 @@ __device__ __forceinline__ uint32_t hmax_abs2(uint32_t a, uint32_t b) {
   return d;
 }
 
+// max |x| of each bf16 half over 8 bf16x2 words (sign bits meaningless).
+__device__ __forceinline__ uint32_t hmax_abs_words(const uint4 (&w)[2]) {
+  return hmax_abs2(hmax_abs2(hmax_abs2(w[0].x, w[0].y), hmax_abs2(w[0].z, w[0].w)),
+                   hmax_abs2(hmax_abs2(w[1].x, w[1].y), hmax_abs2(w[1].z, w[1].w)));
+}
+
 // max |x| of 8 bf16x2 words, as binary32 bits (NaN/Inf give >= 0x7f800000).
 __device__ __forceinline__ uint32_t amax_bits_bf16(const uint4 (&w)[2]) {
-  uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(w[0].x, w[0].y), hmax_abs2(w[0].z, w[0].w)),
-                         hmax_abs2(hmax_abs2(w[1].x, w[1].y), hmax_abs2(w[1].z, w[1].w)));
+  uint32_t m = hmax_abs_words(w);
   m &= 0x7fff7fffu;
   return max(m & 0xffffu, m >> 16) << 16;
 }
@@ -450,12 +455,17 @@ __device__ __forceinline__ void build_scale_table(float2* tab, float St) {
 
 // The same table as (inv, inv, -E, -E) per code: the two packed operands of
 // the candidate step (candidate1_t) in one 16-byte load.
-__device__ __forceinline__ void build_scale_table4(float4* tab, float St) {
-  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+// Entries t, t + nt, ... are written by this thread.
+__device__ __forceinline__ void build_scale_table4(float4* tab, float St, int t, int nt) {
+  for (int c = t; c < 128; c += nt) {
     const float E = __fmul_rn(e4m3_to_f32((uint32_t)c), St);
     const float inv = (E == 0.0f) ? 0.0f : fminf(__frcp_rn(E), kFltMax);
     tab[c] = make_float4(inv, inv, -E, -E);
   }
+}
+
+__device__ __forceinline__ void build_scale_table4(float4* tab, float St) {
+  build_scale_table4(tab, St, (int)threadIdx.x, (int)blockDim.x);
 }
 
 }  // namespace fos

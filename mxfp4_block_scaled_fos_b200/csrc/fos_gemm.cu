@@ -16,7 +16,7 @@
 //   warp 0     TMA producer: per 256-wide K step, the A and B code tiles
 //              (128 rows x 128 bytes each, 128-byte swizzle) as 2D tensor
 //              copies and the four 512-byte scale atoms of each as one
-//              2 KB bulk copy, into a 4-stage shared-memory ring;
+//              2 KB bulk copy, into a 6-stage shared-memory ring;
 //   warp 1     allocates the tensor memory; one thread copies the stage's
 //              scale atoms into tensor memory (tcgen05.cp 32x128b.warpx4)
 //              and issues the four K=64 tcgen05.mma of the stage

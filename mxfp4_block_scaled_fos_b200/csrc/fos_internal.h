@@ -8,17 +8,6 @@
 #include "fos.h"
 #include "fos_device.cuh"
 
-// 16x16 tiles (fos_tiles.cu): 2 = one row per lane (k_2d_row), 1 = two rows
-// per lane (k_2d_warp), 0 = the shared-memory strip kernel (k_2d16x16)
-#ifndef FOS_2D_WARP
-#define FOS_2D_WARP 0
-#endif
-// 1: rowwise + colwise 1x16 by the warp-based kernel (k_dual_warp);
-// 0: the strip kernel (k_dual1x16)
-#ifndef FOS_DUAL_WARP
-#define FOS_DUAL_WARP 1
-#endif
-
 namespace fos {
 
 // One output orientation as the kernels see it.

@@ -23,11 +23,22 @@ namespace fos {
 namespace {
 
 constexpr int kThreads = 256;
-// resident CTAs per SM the rowwise quantizer is compiled for (register cap)
+// Resident CTAs per SM the rowwise quantizer (k_q1x16) is compiled for (the
+// register cap).  Its dense loop loads the next group's block one iteration
+// ahead (FOS_K1_PREFETCH), which needs the registers of 4 CTAs per SM: 0.595
+// ms against 0.618 ms (5 CTAs, no prefetch) on the 128-expert 4/6 batch.
 #ifndef FOS_K1_MIN_BLOCKS
-#define FOS_K1_MIN_BLOCKS 5
+#define FOS_K1_MIN_BLOCKS 4
 #endif
-// the same for the stochastic-rounding and Hadamard variants (more registers)
+#ifndef FOS_K1_PREFETCH
+#define FOS_K1_PREFETCH 1
+#endif
+// the fused amax + quantize kernel: 5 CTAs per SM, no prefetch (its amax
+// items want the CTAs; 0.729 ms against 0.747 ms with 4 CTAs and prefetch)
+#ifndef FOS_FUSED_MIN_BLOCKS
+#define FOS_FUSED_MIN_BLOCKS 5
+#endif
+// the stochastic-rounding and Hadamard variants of both (more registers)
 #ifndef FOS_K1_MIN_BLOCKS_HEAVY
 #define FOS_K1_MIN_BLOCKS_HEAVY 4
 #endif
@@ -195,7 +206,7 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float4* s_tab
 // past c1 recomputes block c1 - 1 and stores nothing).  With choice bits the
 // bitmap words must belong to one warp each (blocks per entry % 64 == 0,
 // c0 % 32 == 0).
-template <bool F46, bool SR, bool RHT, int FAST, int NT = kThreads, bool FAKE = false>
+template <bool F46, bool SR, bool RHT, int FAST, int NT = kThreads, bool FAKE = false, bool PF = false>
 __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
                                               const float4* s_tab, const TScale& ts, uint32_t mask16,
                                               uint32_t& bad, unsigned long long pol) {
@@ -209,12 +220,20 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
   const long long g0 = SR ? a.elem_offset + (long long)b * a.x_bs : 0;
   const float nz = a.neg_zero;
   const unsigned long long seed = a.seed;
-  uint32_t g = c0 + 32 * (threadIdx.x >> 5);  // uniform per warp
+  uint32_t g = c0 + 32 * (NT == 32 ? 0u : (threadIdx.x >> 5));  // uniform per warp
+  uint4 wn[2];  // PF: the next group's block, loaded one iteration ahead
+  if (PF && g + 32 <= c1) ld_block256_hint(xb + (size_t)(g + lane) * 16, pol, wn);
 #pragma unroll 1
   for (; g + 32 <= c1; g += NT) {
     const uint32_t j = g + lane;
     uint4 w[2];
-    ld_block256_hint(xb + (size_t)j * 16, pol, w);
+    if (PF) {
+      w[0] = wn[0];
+      w[1] = wn[1];
+      if (g + NT + 32 <= c1) ld_block256_hint(xb + (size_t)(j + NT) * 16, pol, wn);
+    } else {
+      ld_block256_hint(xb + (size_t)j * 16, pol, w);
+    }
     uint32_t codes[2], sc;
     bool pick;
     rowwise_block<F46, SR, RHT, FAST>(w, s_tab, ts, mask16, nz, seed, g0 + (long long)j * 16, bad, codes,
@@ -255,21 +274,21 @@ __device__ __forceinline__ void rowwise_dense(const QuantArgs& a, int b, uint32_
   }
 }
 
-// Quantize blocks [c0, c1) of batch entry b with this CTA: lane l of warp w
-// takes block g + l for g = c0 + 32w, c0 + 32w + 256, ...  c0 must be a
-// multiple of 32 so that each 32-bit word of the choice bitmap belongs to one
-// warp.
-template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, int NT = kThreads, bool FAKE = false>
+// Quantize blocks [c0, c1) of batch entry b with a group of NT threads (the
+// CTA, or with NT = 32 one warp): lane l of warp w takes block g + l for
+// g = c0 + 32w, c0 + 32w + NT, ...  c0 must be a multiple of 32 so that each
+// 32-bit word of the choice bitmap belongs to one warp.
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, int NT = kThreads, bool FAKE = false, bool PF = false>
 __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_t c0, uint32_t c1,
                                               const float4* s_tab, const TScale& ts, uint32_t mask16,
                                               uint32_t& bad, unsigned long long pol) {
   if (DENSE) {
-    if (ts.fast) rowwise_dense<F46, SR, RHT, 1, NT, FAKE>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
-    else         rowwise_dense<F46, SR, RHT, 0, NT, FAKE>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    if (ts.fast) rowwise_dense<F46, SR, RHT, 1, NT, FAKE, PF>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
+    else         rowwise_dense<F46, SR, RHT, 0, NT, FAKE, PF>(a, b, c0, c1, s_tab, ts, mask16, bad, pol);
     return;
   }
   const int lane = threadIdx.x & 31;
-  for (uint32_t g = c0 + 32 * (threadIdx.x >> 5); g < c1; g += NT) {  // uniform per warp
+  for (uint32_t g = c0 + 32 * (NT == 32 ? 0u : (threadIdx.x >> 5)); g < c1; g += NT) {  // uniform per warp
     const uint32_t j = g + lane;
     const bool valid = j < c1;
     uint4 w[2];
@@ -355,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
                   l2_policy_evict_first());
   }
   uint32_t bad = 0;
-  rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, b, c0, c1, s_tab, ts, mask16, bad,
+  rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE, FOS_K1_PREFETCH != 0>(a, b, c0, c1, s_tab, ts, mask16, bad,
                                                           DENSE ? l2_policy_evict_first() : 0ull);
   if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
@@ -366,22 +385,22 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 // queue.  The queue is a fixed sequence of items: phase p holds the amax
 // chunks of entry p (if p < batch) followed by the quantize chunks of entry
 // p - L (L = min(lag, batch)).  CTAs claim items in sequence order with one
-// atomic counter, claiming the next item while they work on the current one.
-// An amax item reduces its chunk and counts in on done_a[entry]; a quantize
-// item first waits until every amax chunk of its entry has counted in, then
-// quantizes its chunk with that entry's S_t.  Every item an item waits on
-// precedes it in the sequence and was claimed by a running CTA that never
-// waits on a later item, so the queue needs no co-residency and cannot
-// deadlock; the wait is bounded anyway (about a second, then
+// atomic counter.  An amax item reduces its chunk and counts in on done_a[entry]; a
+// quantize item first waits until every amax chunk of its entry has counted
+// in, then quantizes its chunk with that entry's S_t.  Every item an item
+// waits on precedes it in the sequence and was claimed by a running CTA
+// that never waits on a later item, so the queue needs no co-residency and
+// cannot deadlock; the wait is bounded anyway (about a second, then
 // FOS_STATUS_TIMEOUT).  Memory-bound amax chunks and compute-bound quantize
 // chunks run side by side on every SM, and with the L + 1 entries in flight
 // smaller than L2 (and the amax reads marked evict-last) the quantize reads
 // hit L2, so HBM sees the input about once.
-// Lag in entries between an entry's amax and its quantize items, and the
-// quantize item size: measured best on the 128 x 2880 x 2880 expert batch
-// (4/6: 1536 blocks, lag 3; 6-only: 1536 blocks, lag 2).
+// Lag in entries between an entry's amax and its quantize items, and the item
+// sizes in blocks: measured on the 128 x 2880 x 2880 expert batch (lag 2,
+// claims at item end: 0.738 ms for 4/6 against 0.781 ms for lag 3 with
+// claim-ahead; 2048-block quantize items 0.729 ms).
 #ifndef FOS_FUSED_LAG_46
-#define FOS_FUSED_LAG_46 3
+#define FOS_FUSED_LAG_46 2
 #endif
 #ifndef FOS_FUSED_LAG_6
 #define FOS_FUSED_LAG_6 2
@@ -392,16 +411,24 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 #ifndef FOS_FUSED_ACHUNK
 #define FOS_FUSED_ACHUNK 4096
 #endif
-#ifndef FOS_FUSED_QCHUNK
-#define FOS_FUSED_QCHUNK 1536
+#ifndef FOS_FUSED_QCHUNK_46
+#define FOS_FUSED_QCHUNK_46 2048
 #endif
-// 1: the CTA that claims an amax item starts a bulk L2 prefetch of its chunk
-// at claim time, so that the item itself reads from L2
-#ifndef FOS_FUSED_PREFETCH
-#define FOS_FUSED_PREFETCH 0
+#ifndef FOS_FUSED_QCHUNK_6
+#define FOS_FUSED_QCHUNK_6 1536
+#endif
+// 1: a CTA claims its next item when it starts an item (the claim's latency
+// hides behind the item, but twice as many items are in flight, so an entry's
+// quantize items reach the queue head while its amax items are still being
+// reduced unless the lag grows); 0: when it ends one
+#ifndef FOS_FUSED_CLAIM_AHEAD
+#define FOS_FUSED_CLAIM_AHEAD 0
 #endif
 constexpr uint32_t kAChunk = FOS_FUSED_ACHUNK;  // blocks per amax item
-constexpr uint32_t kQChunk = FOS_FUSED_QCHUNK;  // blocks per quantize item (multiple of 32)
+// blocks per quantize item
+template <bool F46>
+constexpr uint32_t qchunk() { return F46 ? FOS_FUSED_QCHUNK_46 : FOS_FUSED_QCHUNK_6; }
+static_assert(qchunk<true>() % 32 == 0 && qchunk<false>() % 32 == 0, "quantize items hold whole choice words");
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
@@ -409,8 +436,8 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   return v;
 }
 
-// Bounded wait until *p >= target (thread 0 of the CTA calls it): at most
-// `limit` polls, then FOS_STATUS_TIMEOUT and return.
+// Bounded wait until *p >= target (one thread calls it): at most `limit`
+// polls, then FOS_STATUS_TIMEOUT and return.
 __device__ __forceinline__ void wait_at_least(const uint32_t* p, uint32_t target, uint32_t* status,
                                               uint32_t limit) {
   uint32_t it = 0;
@@ -423,17 +450,40 @@ __device__ __forceinline__ void wait_at_least(const uint32_t* p, uint32_t target
   }
 }
 
-// max |x| (of the RHT of x) over blocks [lo, hi) of entry b, U loads in
-// flight per thread.
-template <bool RHT, bool DENSE>
+// max |x| (of the RHT of x) over blocks [lo, hi) of entry b by a group of NT
+// threads (t = this thread's index in the group), U loads in flight per
+// thread.  Dense input without the transform keeps a running max of |x| over
+// bf16 pairs (8 packed max per block) and converts it once at the end.
+template <bool RHT, bool DENSE, int NT = kThreads>
 __device__ __forceinline__ uint32_t slice_amax_bits(const QuantArgs& a, int b, uint32_t lo, uint32_t hi,
-                                                    uint32_t mask16, unsigned long long pol) {
+                                                    uint32_t mask16, unsigned long long pol, uint32_t t) {
   constexpr int U = FOS_FUSED_AMAX_UNROLL;
+  if (DENSE && !RHT) {
+    const uint16_t* xb = a.x + (long long)b * a.x_bs;
+    uint32_t m2 = 0;  // the sign bits of this word carry no meaning (xorsign form)
+    uint32_t j = lo + t;
+#pragma unroll 1
+    for (; j + (U - 1) * NT < hi; j += U * NT) {
+      uint4 w[U][2];
+#pragma unroll
+      for (int u = 0; u < U; ++u) ld_block256_hint(xb + (size_t)(j + u * NT) * 16, pol, w[u]);
+#pragma unroll
+      for (int u = 0; u < U; ++u) m2 = hmax_abs2(m2, hmax_abs_words(w[u]));
+    }
+#pragma unroll 1
+    for (; j < hi; j += NT) {
+      uint4 w[2];
+      ld_block256_hint(xb + (size_t)j * 16, pol, w);
+      m2 = hmax_abs2(m2, hmax_abs_words(w));
+    }
+    m2 &= 0x7fff7fffu;
+    return max(m2 & 0xffffu, m2 >> 16) << 16;
+  }
   uint32_t m = 0;
-  for (uint32_t j0 = lo + threadIdx.x; j0 < hi; j0 += U * kThreads) {
+  for (uint32_t j0 = lo + t; j0 < hi; j0 += U * NT) {
     uint4 w[U][2];
 #pragma unroll
-    for (int u = 0; u < U; ++u) k1_load<DENSE>(a, b, j0 + u * kThreads, j0 + u * kThreads < hi, w[u], pol);
+    for (int u = 0; u < U; ++u) k1_load<DENSE>(a, b, j0 + u * NT, j0 + u * NT < hi, w[u], pol);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (RHT) {
@@ -458,6 +508,15 @@ __device__ __forceinline__ uint32_t slice_amax_bits(const QuantArgs& a, int b, u
   return m;
 }
 
+// The item sequence of one launch (computed on the host).
+struct FusedPlan {
+  uint32_t na, nq;         // amax and quantize items per entry
+  uint32_t head, mid;      // items of phases [0, L) and of phases [L, batch)
+  uint32_t total;          // batch * (na + nq) < 2^31
+  int L;
+  FastDiv f_na, f_nq, f_ph;  // division by na, nq and na + nq
+};
+
 struct FusedItem {
   bool amax;        // amax item (else quantize item)
   int entry;
@@ -465,65 +524,64 @@ struct FusedItem {
 };
 
 // Position i of the item sequence (i < total) -> item.
-__device__ __forceinline__ FusedItem fused_item(uint32_t i, int batch, int L, uint32_t na, uint32_t nq) {
+__device__ __forceinline__ FusedItem fused_item(uint32_t i, int batch, const FusedPlan& p) {
   FusedItem it;
-  const uint32_t head = (uint32_t)L * na;                 // phases 0 .. L-1: amax only
-  const uint32_t mid = (uint32_t)(batch - L) * (na + nq);  // phases L .. batch-1: amax + quantize
-  if (i < head) {
-    it.amax = true; it.entry = (int)(i / na); it.chunk = i % na;
-  } else if (i - head < mid) {
-    const uint32_t r = (i - head) % (na + nq);
-    const int p = L + (int)((i - head) / (na + nq));
-    if (r < na) { it.amax = true; it.entry = p; it.chunk = r; }
-    else        { it.amax = false; it.entry = p - L; it.chunk = r - na; }
+  if (i < p.head) {                                        // phases 0 .. L-1: amax only
+    const uint32_t e = fdiv(i, p.f_na);
+    it.amax = true; it.entry = (int)e; it.chunk = i - e * p.na;
+  } else if (i - p.head < p.mid) {                         // phases L .. batch-1
+    const uint32_t r0 = i - p.head, ph = fdiv(r0, p.f_ph);
+    const uint32_t r = r0 - ph * (p.na + p.nq);
+    const int e = p.L + (int)ph;
+    if (r < p.na) { it.amax = true; it.entry = e; it.chunk = r; }
+    else          { it.amax = false; it.entry = e - p.L; it.chunk = r - p.na; }
   } else {                                                 // phases batch .. batch+L-1
-    const uint32_t r = i - head - mid;
-    it.amax = false; it.entry = batch - L + (int)(r / nq); it.chunk = r % nq;
+    const uint32_t r = i - p.head - p.mid, e = fdiv(r, p.f_nq);
+    it.amax = false; it.entry = batch - p.L + (int)e; it.chunk = r - e * p.nq;
   }
   return it;
 }
 
+// An amax item's result m (max |x| bits of the chunk) into the entry's word,
+// then the count-in (release) on done_a[entry]; one thread calls it.
+__device__ __forceinline__ void amax_count_in(const QuantArgs& a, uint32_t* amax_ws, uint32_t* done_a, int e,
+                                              uint32_t m) {
+  if (m >= 0x7f800000u) {
+    if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+  } else if (m) {
+    atomicMax(amax_ws + e, m);
+  }
+  __threadfence();
+  if (e != a.stall_entry) atomicAdd(done_a + e, 1u);
+}
+
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE>
-__global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_K1_MIN_BLOCKS)
-    k_q1x16_fused(const QuantArgs a, int batch, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue) {
+__global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_FUSED_MIN_BLOCKS)
+    k_q1x16_fused(const QuantArgs a, int batch, const FusedPlan p, uint32_t* amax_ws, uint32_t* done_a,
+                  uint32_t* queue) {
   __shared__ float4 s_tab[128];
   __shared__ uint32_t s_red[kThreads / 32];
   __shared__ float s_St;
   __shared__ uint32_t s_item[2];
   const uint32_t mask16 = RHT ? rht_sign_mask(a.seed) : 0u;
-  const uint32_t na = (a.nblk + kAChunk - 1) / kAChunk;
-  const uint32_t nq = (a.nblk + kQChunk - 1) / kQChunk;
-  const int L = min(F46 ? FOS_FUSED_LAG_46 : FOS_FUSED_LAG_6, batch);
-  const uint32_t total = (uint32_t)batch * (na + nq);
   const unsigned long long pol_keep = l2_policy_evict_last();   // amax reads: keep for quantize
   const unsigned long long pol_done = l2_policy_evict_first();  // quantize reads: last use
   uint32_t bad = 0;
   int tab_entry = -1;   // entry whose scale table s_tab holds
+  TScale ts{0.0f, 0.0f, false};
 
   if (threadIdx.x == 0) s_item[0] = atomicAdd(queue, 1u);
   __syncthreads();
   for (int k = 0;; k ^= 1) {
     const uint32_t i = s_item[k];
-    if (i >= total) break;
-    if (threadIdx.x == 0) {  // claim the next item now
-      const uint32_t nx = atomicAdd(queue, 1u);
-      s_item[k ^ 1] = nx;
-#if FOS_FUSED_PREFETCH
-      if (DENSE && nx < total) {  // an amax chunk is read from HBM: start it into L2 now
-        const FusedItem ni = fused_item(nx, batch, L, na, nq);
-        if (ni.amax) {
-          const uint32_t lo = ni.chunk * kAChunk, hi = min(lo + kAChunk, a.nblk);
-          const char* base = reinterpret_cast<const char*>(a.x + (long long)ni.entry * a.x_bs + (long long)lo * 16);
-          for (uint32_t off = 0; off < (hi - lo) * 32u; off += 32768u)
-            prefetch_l2(base + off, min(32768u, (hi - lo) * 32u - off), pol_keep);
-        }
-      }
+    if (i >= p.total) break;
+#if FOS_FUSED_CLAIM_AHEAD
+    if (threadIdx.x == 0) s_item[k ^ 1] = atomicAdd(queue, 1u);  // claim the next item now
 #endif
-    }
-    const FusedItem it = fused_item(i, batch, L, na, nq);
+    const FusedItem it = fused_item(i, batch, p);
     if (it.amax) {
       const uint32_t lo = it.chunk * kAChunk, hi = min(lo + kAChunk, a.nblk);
-      uint32_t m = slice_amax_bits<RHT, DENSE>(a, it.entry, lo, hi, mask16, pol_keep);
+      uint32_t m = slice_amax_bits<RHT, DENSE>(a, it.entry, lo, hi, mask16, pol_keep, threadIdx.x);
       m = __reduce_max_sync(0xffffffffu, m);
       if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
       __syncthreads();
@@ -531,121 +589,30 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
         uint32_t v = 0;
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) v = max(v, s_red[w]);
-        if (v >= 0x7f800000u) {
-          if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
-        } else if (v) {
-          atomicMax(amax_ws + it.entry, v);
-        }
-        __threadfence();
-        if (it.entry != a.stall_entry) atomicAdd(done_a + it.entry, 1u);
+        amax_count_in(a, amax_ws, done_a, it.entry, v);
       }
     } else {
       if (it.entry != tab_entry) {
         if (threadIdx.x == 0) {
-          wait_at_least(done_a + it.entry, na, a.status, a.spin_limit);
+          wait_at_least(done_a + it.entry, p.na, a.status, a.spin_limit);
           const float A = __uint_as_float(__ldcg(amax_ws + it.entry));
           s_St = __fdiv_rn(A, F46 ? 1792.0f : 2688.0f);
         }
         __syncthreads();
-        build_scale_table4(s_tab, s_St);
+        ts = make_tscale(s_St);
+        build_scale_table4(s_tab, ts.St);
         __syncthreads();
         tab_entry = it.entry;
       }
-      const float St = s_St;
-      const TScale ts = make_tscale(St);
-      if (it.chunk == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[it.entry] = St;
-      const uint32_t lo = it.chunk * kQChunk, hi = min(lo + kQChunk, a.nblk);
+      if (it.chunk == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[it.entry] = ts.St;
+      const uint32_t lo = it.chunk * qchunk<F46>(), hi = min(lo + qchunk<F46>(), a.nblk);
       rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, it.entry, lo, hi, s_tab, ts, mask16, bad,
                                                               pol_done);
     }
-    __syncthreads();  // the next item is in s_item[k ^ 1]; s_red / s_tab may be rewritten
-  }
-  if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
-}
-
-// --------------------------------------------------------------------------
-// The same fused amax + quantize with the two kinds of work interleaved:
-// item (p, c) of the sequence takes the amax of chunk c of entry p (if p <
-// batch) and quantizes chunk c of entry p - L (if p >= L), chunks of kIChunk
-// blocks.  The amax chunk is started into L2 by a bulk prefetch at the
-// item's start and reduced after the quantize work, so its memory latency
-// hides behind that work instead of holding a CTA slot on its own.  Each
-// warp folds its amax into the entry's word and counts in (8 per item); the
-// quantize part waits (bounded) until all 8 * nc count-ins of its entry are
-// in.  The same no-deadlock argument as k_q1x16_fused holds: an item waits
-// only on items earlier in the sequence.
-#ifndef FOS_FUSED_ICHUNK
-#define FOS_FUSED_ICHUNK 1536
+#if !FOS_FUSED_CLAIM_AHEAD
+    if (threadIdx.x == 0) s_item[k ^ 1] = atomicAdd(queue, 1u);
 #endif
-#ifndef FOS_FUSED_ILAG
-#define FOS_FUSED_ILAG 3
-#endif
-constexpr uint32_t kIChunk = FOS_FUSED_ICHUNK;
-
-template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE>
-__global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_K1_MIN_BLOCKS)
-    k_q1x16_fused2(const QuantArgs a, int batch, uint32_t* amax_ws, uint32_t* done_a, uint32_t* queue) {
-  __shared__ float4 s_tab[128];
-  __shared__ float s_St;
-  __shared__ uint32_t s_item[2];
-  const uint32_t mask16 = RHT ? rht_sign_mask(a.seed) : 0u;
-  const uint32_t nc = (a.nblk + kIChunk - 1) / kIChunk;
-  const int L = FOS_FUSED_ILAG;
-  const uint32_t total = (uint32_t)(batch + L) * nc;
-  const unsigned long long pol_keep = l2_policy_evict_last();   // amax reads: kept for the quantize
-  const unsigned long long pol_done = l2_policy_evict_first();  // quantize reads: last use
-  const uint32_t lane = threadIdx.x & 31;
-  uint32_t bad = 0;
-  int tab_entry = -1;
-
-  if (threadIdx.x == 0) s_item[0] = atomicAdd(queue, 1u);
-  __syncthreads();
-  for (int k = 0;; k ^= 1) {
-    const uint32_t i = s_item[k];
-    if (i >= total) break;
-    if (threadIdx.x == 0) s_item[k ^ 1] = atomicAdd(queue, 1u);  // claim the next one now
-    const int p = (int)(i / nc);
-    const uint32_t c = i - (uint32_t)p * nc;
-    const uint32_t lo = c * kIChunk, hi = min(lo + kIChunk, a.nblk);
-    const bool has_amax = p < batch;
-    if (DENSE && has_amax && threadIdx.x < 32) {  // the amax chunk into L2 now, 16 KB per lane
-      const uint32_t nbytes = (hi - lo) * 32u, off = lane * 16384u;
-      if (off < nbytes)
-        prefetch_l2(a.x + (long long)p * a.x_bs + (long long)lo * 16 + off / 2, min(16384u, nbytes - off),
-                    pol_keep);
-    }
-    const int q = p - L;
-    if (q >= 0) {
-      if (q != tab_entry) {
-        if (threadIdx.x == 0) {
-          wait_at_least(done_a + q, nc * (kThreads / 32), a.status, a.spin_limit);
-          const float A = __uint_as_float(__ldcg(amax_ws + q));
-          s_St = __fdiv_rn(A, F46 ? 1792.0f : 2688.0f);
-        }
-        __syncthreads();
-        build_scale_table4(s_tab, s_St);
-        __syncthreads();
-        tab_entry = q;
-      }
-      const float St = s_St;
-      const TScale ts = make_tscale(St);
-      if (!FAKE && c == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[q] = St;
-      rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, q, lo, hi, s_tab, ts, mask16, bad, pol_done);
-    }
-    if (has_amax) {
-      uint32_t m = slice_amax_bits<RHT, DENSE>(a, p, lo, hi, mask16, pol_keep);
-      m = __reduce_max_sync(0xffffffffu, m);
-      if (lane == 0) {
-        if (m >= 0x7f800000u) {
-          if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
-        } else if (m) {
-          atomicMax(amax_ws + p, m);
-        }
-        __threadfence();
-        if (p != a.stall_entry) atomicAdd(done_a + p, 1u);
-      }
-    }
-    __syncthreads();  // the next item is in s_item[k ^ 1]; s_tab may be rewritten
+    __syncthreads();  // the next item is in s_item[k ^ 1]; s_red / s_tab / s_St may be rewritten
   }
   if (bad >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
@@ -868,21 +835,32 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 // and cached; 0 = not yet known, -1 = the kernel cannot be resident.
 static constexpr int kMaxDevices = 64;
 
-// 1: amax and quantize as separate queue items (k_q1x16_fused); 2: each item
-// does both (k_q1x16_fused2)
-#ifndef FOS_FUSED_MODE
-#define FOS_FUSED_MODE 1
-#endif
+// The item sequence for nblk blocks per entry; false when the item count does
+// not fit the 31-bit positions of the queue.
+static bool make_plan(FusedPlan& p, uint32_t nblk, int batch, uint32_t achunk, uint32_t qchunk, int lag) {
+  if (nblk == 0 || batch < 1) return false;
+  p.na = (nblk + achunk - 1) / achunk;
+  p.nq = (nblk + qchunk - 1) / qchunk;
+  p.L = lag < batch ? lag : batch;
+  const unsigned long long total = (unsigned long long)batch * (p.na + p.nq);
+  if (total >= (1ull << 31)) return false;
+  p.total = (uint32_t)total;
+  p.head = (uint32_t)p.L * p.na;
+  p.mid = (uint32_t)(batch - p.L) * (p.na + p.nq);
+  p.f_na = make_fastdiv(p.na);
+  p.f_nq = make_fastdiv(p.nq);
+  p.f_ph = make_fastdiv(p.na + p.nq);
+  return true;
+}
 
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE = false>
 static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_ws, uint32_t* done_a,
                                   uint32_t* queue, cudaStream_t st) {
   static std::atomic<int> grid_of[kMaxDevices];
-#if FOS_FUSED_MODE == 2
-  auto kern = k_q1x16_fused2<F46, SR, RHT, SWZ, DENSE, FAKE>;
-#else
   auto kern = k_q1x16_fused<F46, SR, RHT, SWZ, DENSE, FAKE>;
-#endif
+  FusedPlan plan;
+  if (!make_plan(plan, a.nblk, batch, kAChunk, qchunk<F46>(), F46 ? FOS_FUSED_LAG_46 : FOS_FUSED_LAG_6))
+    return cudaErrorNotSupported;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
   int grid = grid_of[dev].load(std::memory_order_relaxed);
@@ -895,7 +873,7 @@ static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_
     grid_of[dev].store(grid, std::memory_order_relaxed);
   }
   if (grid < 1) return cudaErrorNotSupported;
-  kern<<<grid, kThreads, 0, st>>>(a, batch, amax_ws, done_a, queue);
+  kern<<<grid, kThreads, 0, st>>>(a, batch, plan, amax_ws, done_a, queue);
   return cudaGetLastError();
 }
 

@@ -5,14 +5,18 @@
 //   * 16x16 2D block scaling (same section): one scale and one 4/6 choice per
 //     16x16 tile, written row-major and as its exact transpose.
 //
-// A CTA of 256 threads walks a strip of up to 8 sub-tiles of 64 rows x 128
-// columns (16 KB of bf16) down the tensor.  Each sub-tile is staged in shared
-// memory with 16-byte chunks XOR-swizzled by row so that the row-major reads,
-// the column reads and the 16x16 reads are all free of bank conflicts; the
-// next sub-tile's global loads are issued before the current one is
-// processed.  Stochastic-rounding bytes are drawn once per 16 source elements
-// (one Philox call per rowwise block) and shared by both orientations
-// through shared memory.
+// 1x16 rowwise + colwise (k_dual_warp): every warp takes units of 4
+// adjacent 16x16 tiles, loaded straight from global memory, and transposes
+// them through its own shared buffer; no CTA barrier in the loop.
+// 16x16 (k_2d16x16): a CTA of 256 threads walks a strip of up to 8 sub-tiles
+// of 64 rows x 128 columns (16 KB of bf16) down the tensor.  Each sub-tile is
+// staged in shared memory with 16-byte chunks XOR-swizzled by row so that the
+// row-major reads, the column reads and the 16x16 reads are all free of bank
+// conflicts; the next sub-tile's global loads are issued before the current
+// one is processed.
+// Stochastic-rounding bytes are drawn once per 16 source elements (one Philox
+// call per rowwise block) and shared by both orientations through shared
+// memory.
 #include "fos_core.cuh"
 
 namespace fos {
@@ -23,17 +27,9 @@ constexpr int kThreads = 256;
 constexpr int kSubRows = 64;
 constexpr int kSubCols = 128;
 constexpr int kStrip = 8;  // sub-tiles per CTA strip (512 rows)
-#ifndef FOS_DUAL_MIN_BLOCKS
-#define FOS_DUAL_MIN_BLOCKS 2
-#endif
 #ifndef FOS_2D_MIN_BLOCKS
 #define FOS_2D_MIN_BLOCKS 3
 #endif
-
-struct TileGeom {
-  int rows, cols;     // tensor
-  int r_strip0, c0;   // strip origin
-};
 
 // smem byte offset of the 16-byte chunk c16 of row r under swizzle f(r).
 template <int SHIFT>
@@ -146,185 +142,6 @@ __device__ __forceinline__ PairResult<F46> quant_pair4(const float2 (&P)[16], ui
     if (r.pb) { r.cb[0] = c4.cb[0]; r.cb[1] = c4.cb[1]; r.sb = s4b; r.invb = t4b.x; }
   }
   return r;
-}
-
-// --------------------------------------------------------------------------
-// 1x16 rowwise + colwise.  grid (ceil(cols/128), ceil(rows/512), batch).
-template <bool F46, bool SR, bool SWZ, bool ROW>
-__global__ void __launch_bounds__(kThreads, FOS_DUAL_MIN_BLOCKS) k_dual1x16(const QuantArgs a) {
-  __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
-  __shared__ __align__(16) uint4 s_rnd[SR ? kSubRows * 8 : 1];
-  __shared__ float2 s_tab[128];
-  __shared__ uint32_t s_rbits[kSubRows];
-  __shared__ uint32_t s_cbits[kSubCols];
-
-  const int b = blockIdx.z;
-  const int c0 = blockIdx.x * kSubCols;
-  const int rs0 = blockIdx.y * (kSubRows * kStrip);
-  const float St = tensor_scale_of(a, b, F46);
-  build_scale_table(s_tab, St);
-  const TScale ts = make_tscale(St);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
-    if (a.col.tensor_scale) a.col.tensor_scale[b] = St;
-  }
-  if (threadIdx.x < kSubCols) s_cbits[threadIdx.x] = 0;
-  if (threadIdx.x < kSubRows) s_rbits[threadIdx.x] = 0;
-
-  const int t = threadIdx.x;
-  // rowwise role: row rr, block pair pp (blocks 2pp, 2pp+1 of the 8 in a row)
-  const int rr = t & 63, pp = t >> 6;
-  // colwise role: column pair cq (cols 2cq, 2cq+1), row group gq (16 rows)
-  const int cq = t & 63, gq = t >> 6;
-  const long long nbc = a.cols / 16;   // rowwise blocks per row
-  const long long nrg = a.rows / 16;   // colwise blocks per column
-  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
-  uint32_t bad = 0;
-  uint32_t cbits_a = 0, cbits_b = 0;   // colwise picks of this thread's 2 columns
-
-  uint4 reg[4];
-  load_sub(a, b, rs0, c0, reg);
-  for (int k = 0; k < kStrip; ++k) {
-    const int r0 = rs0 + k * kSubRows;
-    if (r0 >= a.rows) break;
-    __syncthreads();
-    store_sub<0>(s_tile, reg);
-    __syncthreads();
-    if (k + 1 < kStrip && r0 + kSubRows < a.rows) load_sub(a, b, r0 + kSubRows, c0, reg);
-
-    // ---------------- rowwise pass (also draws the SR bytes) ----------------
-    {
-      const int gr = r0 + rr;
-      const int bc = c0 / 16 + 2 * pp;   // global block column of block A
-      const bool va = gr < a.rows && bc < nbc;
-      const bool vb = gr < a.rows && bc + 1 < nbc;
-      if (SR) {
-        uint4 ra = make_uint4(0, 0, 0, 0), rb = ra;
-        if (va) ra = sr_bytes16(a.seed, gbase + (long long)gr * a.cols + bc * 16);
-        if (vb) rb = sr_bytes16(a.seed, gbase + (long long)gr * a.cols + (bc + 1) * 16);
-        s_rnd[rr * 8 + 2 * pp] = ra;
-        s_rnd[rr * 8 + 2 * pp + 1] = rb;
-      }
-      if (ROW && va) {
-        uint4 wa[2], wb[2];
-        wa[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp));
-        wa[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp + 1));
-        wb[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp + 2));
-        wb[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<0>(rr, 4 * pp + 3));
-        float2 P[16];
-        unpack_pairs(wa, wb, P);
-        const uint32_t ma = amax_bits_bf16(wa), mb = amax_bits_bf16(wb);
-        bad |= max(ma, mb) >= 0x7f800000u;
-        PairResult<F46> q = quant_pair<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
-        if (SR) {
-          sr_block(P, 0, q.inva, s_rnd[rr * 8 + 2 * pp], q.ca);
-          sr_block(P, 1, q.invb, s_rnd[rr * 8 + 2 * pp + 1], q.cb);
-        }
-        store_codes8(a.row, b, gr, bc * 8, q.ca[0], q.ca[1]);
-        a.row.scales[scale_off<SWZ>(a.row, b, gr, bc)] = (uint8_t)q.sa;
-        if (vb) {
-          store_codes8(a.row, b, gr, (bc + 1) * 8, q.cb[0], q.cb[1]);
-          a.row.scales[scale_off<SWZ>(a.row, b, gr, bc + 1)] = (uint8_t)q.sb;
-        }
-        if (F46 && a.row.choice && (q.pa | q.pb))
-          atomicOr(&s_rbits[rr], (q.pa << (2 * pp)) | ((vb ? q.pb : 0u) << (2 * pp + 1)));
-      }
-    }
-    if (SR) __syncthreads();  // SR bytes visible to the colwise pass
-
-    // ---------------- colwise pass ----------------
-    {
-      const int gc = c0 + 2 * cq;
-      const int grow = r0 + 16 * gq;
-      if (gc < a.cols && grow < a.rows) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int r = 16 * gq + i;
-          w[i] = *reinterpret_cast<const uint32_t*>(s_tile + chunk_off<0>(r, cq >> 2) + (cq & 3) * 4);
-        }
-        float2 P[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) P[i] = make_float2(bf_lo(w[i]), bf_hi(w[i]));
-        uint32_t h[8];   // max |x| of both columns: a tree of packed bf16 maxima
-#pragma unroll
-        for (int i = 0; i < 8; ++i) h[i] = hmax_abs2(w[2 * i], w[2 * i + 1]);
-        const uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(h[0], h[1]), hmax_abs2(h[2], h[3])),
-                                     hmax_abs2(hmax_abs2(h[4], h[5]), hmax_abs2(h[6], h[7]))) &
-                           0x7fff7fffu;
-        const uint32_t ma = (m & 0xffffu) << 16, mb = m & 0xffff0000u;
-        bad |= max(ma, mb) >= 0x7f800000u;
-        PairResult<F46> q = quant_pair<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
-        if (SR) {
-          uint32_t ba[16], bb[16];
-          const uint8_t* rb = reinterpret_cast<const uint8_t*>(s_rnd);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int r = 16 * gq + i;
-            const uint32_t two = *reinterpret_cast<const uint16_t*>(rb + r * 128 + (cq >> 3) * 16 +
-                                                                    2 * (cq & 7));
-            ba[i] = two & 0xffu;
-            bb[i] = two >> 8;
-          }
-          sr_block_bytes(P, 0, q.inva, ba, q.ca);
-          sr_block_bytes(P, 1, q.invb, bb, q.cb);
-        }
-        const long long rg = grow / 16;
-        store_codes8(a.col, b, gc, rg * 8, q.ca[0], q.ca[1]);
-        store_codes8(a.col, b, gc + 1, rg * 8, q.cb[0], q.cb[1]);
-        a.col.scales[scale_off<SWZ>(a.col, b, gc, rg)] = (uint8_t)q.sa;
-        a.col.scales[scale_off<SWZ>(a.col, b, gc + 1, rg)] = (uint8_t)q.sb;
-        cbits_a |= q.pa << (4 * k + gq);
-        cbits_b |= q.pb << (4 * k + gq);
-      }
-    }
-
-    // rowwise choice bits of this sub-tile: 8 bits per row
-    if (ROW && F46 && a.row.choice) {
-      __syncthreads();
-      if (t < kSubRows) {
-        const uint32_t v = s_rbits[t];
-        s_rbits[t] = 0;
-        const int gr = r0 + t;
-        if (gr < a.rows) {
-          const unsigned long long bit = ((unsigned long long)b * a.rows + gr) * nbc + c0 / 16;
-          if (a.row.choice_aligned) {
-            a.row.choice[bit >> 3] = (uint8_t)v;
-          } else if (v) {
-            unsigned int* wp = reinterpret_cast<unsigned int*>(a.row.choice) + (bit >> 5);
-            const int sh = (int)(bit & 31);
-            const unsigned long long vv = (unsigned long long)v << sh;
-            if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
-            if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
-          }
-        }
-      }
-    }
-  }
-
-  // colwise choice bits of the strip: 32 row groups per column
-  if (F46 && a.col.choice) {
-    if (cbits_a) atomicOr(&s_cbits[2 * cq], cbits_a);
-    if (cbits_b) atomicOr(&s_cbits[2 * cq + 1], cbits_b);
-    __syncthreads();
-    if (t < kSubCols) {
-      const int gc = c0 + t;
-      if (gc < a.cols) {
-        const uint32_t v = s_cbits[t];
-        const unsigned long long bit = ((unsigned long long)b * a.cols + gc) * nrg + rs0 / 16;
-        unsigned int* base = reinterpret_cast<unsigned int*>(a.col.choice);
-        if (a.col.choice_aligned) {
-          base[bit >> 5] = v;
-        } else if (v) {
-          const int sh = (int)(bit & 31);
-          const unsigned long long vv = (unsigned long long)v << sh;
-          if ((uint32_t)vv) atomicOr(base + (bit >> 5), (uint32_t)vv);
-          if ((uint32_t)(vv >> 32)) atomicOr(base + (bit >> 5) + 1, (uint32_t)(vv >> 32));
-        }
-      }
-    }
-  }
-  if (bad && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
 }
 
 // Nibbles of a (8) into the low halves of 8 bytes, b into the high halves:
@@ -494,281 +311,6 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_DUALW_MIN_BLOCKS) k_dua
         const unsigned long long c0 = (unsigned long long)tc * 16 + 2 * i;
         if (pca) or_bits(a.col.choice, ((unsigned long long)b * a.cols + c0) * ntr + trow, 1u);
         if (pcb) or_bits(a.col.choice, ((unsigned long long)b * a.cols + c0 + 1) * ntr + trow, 1u);
-      }
-    }
-  }
-  badmax = __reduce_max_sync(0xffffffffu, badmax);
-  if (lane == 0 && badmax >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
-}
-
-// --------------------------------------------------------------------------
-// 16x16 2D block scaling, one row per lane.  grid (CTAs, batch); every warp
-// takes units of 2 horizontally adjacent tiles (tile row tr, tile columns
-// 2u, 2u+1), 16 lanes per tile, lane r of a tile holding its row r as one
-// block of 8 split pairs -- the per-block arithmetic of the rowwise
-// quantizer.  The tile amax and the tree over the 16 row error sums (rows
-// (2i, 2i+1) first, then pairs of those: the R6 order) are 16-lane xor
-// shuffles.  For the transposed copy the even lanes zip their row with the
-// next (row 2i in the low nibbles, 2i+1 in the high) and the tile goes
-// through this warp's shared buffer (8 row pairs x 16 bytes), from which
-// lane j of the first 8 takes columns 2j and 2j+1.  No CTA barrier in the
-// loop; choice bits go into zeroed bitmaps with atomics.
-constexpr int kTrStride = 144;   // bytes between the tiles' rows in the per-warp
-                                 // transpose buffers: 9 x 16, so that reads of
-                                 // different tiles fall into distinct banks
-#ifndef FOS_2DR_MIN_BLOCKS
-#define FOS_2DR_MIN_BLOCKS 5
-#endif
-
-template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
-__global__ void __launch_bounds__(kThreads, SR ? 3 : FOS_2DR_MIN_BLOCKS) k_2d_row(const QuantArgs a, FastDiv ntc2) {
-  __shared__ __align__(16) float4 s_tab[128];
-  __shared__ __align__(16) uint8_t s_tr[kThreads / 32][2 * kTrStride];
-  const int b = blockIdx.y;
-  const float St = tensor_scale_of(a, b, F46);
-  build_scale_table4(s_tab, St);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
-    if (COL && a.col.tensor_scale) a.col.tensor_scale[b] = St;
-  }
-  __syncthreads();
-  const TScale ts = make_tscale(St);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int h = lane >> 4, r = lane & 15;
-  const uint32_t ntr = a.rows / 16, ntc = a.cols / 16;
-  const uint32_t nunits = ntr * ntc2.d;
-  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
-  const float nz = a.neg_zero;
-  uint8_t* trb = s_tr[warp] + h * kTrStride;
-  uint32_t badmax = 0;
-  for (uint32_t u = blockIdx.x * (kThreads / 32) + warp; u < nunits; u += gridDim.x * (kThreads / 32)) {
-    const uint32_t trow = fdiv(u, ntc2), tq = u - trow * ntc2.d;
-    const uint32_t tc = tq * 2 + h;
-    const bool valid = tc < ntc;  // uniform over the 16 lanes of a tile
-    const long long row = (long long)trow * 16 + r;
-    uint4 w[2];
-    if (valid) {
-      const uint4* px = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs + row * a.ld + (long long)tc * 16);
-      w[0] = __ldg(px);
-      w[1] = __ldg(px + 1);
-    } else {
-      w[0] = w[1] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    const uint32_t W8[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
-    float2 P[8];
-    unpack_split(W8, P);
-    uint32_t m = amax_bits_bf16(w);
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
-    badmax = max(badmax, m);
-    uint32_t s6, s4;
-    cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
-    const float4 t6 = s_tab[s6];
-    const Cand1 c6 = candidate1_t<F46>(P, t6, nz);
-    uint32_t codes[2] = {c6.c[0], c6.c[1]};
-    uint32_t sc = s6;
-    float inv = t6.x;
-    bool pick = false;
-    if (F46) {
-      const float4 t4 = s_tab[s4];
-      const Cand1 c4 = candidate1_t<true>(P, t4, nz);
-      float e6 = c6.err, e4 = c4.err;  // this row's sums; then the tree over rows
-#pragma unroll
-      for (int sh = 1; sh < 16; sh *= 2) {
-        e6 = __fadd_rn(e6, __shfl_xor_sync(0xffffffffu, e6, sh));
-        e4 = __fadd_rn(e4, __shfl_xor_sync(0xffffffffu, e4, sh));
-      }
-      pick = e4 < e6;  // strictly lower wins; ties keep 6
-      if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.x; }
-    }
-    if (SR) sr_block1(P, inv, sr_bytes16(a.seed, gbase + row * a.cols + (long long)tc * 16), codes);
-    if (ROW && valid) {
-      store_codes8(a.row, b, row, (long long)tc * 8, codes[0], codes[1]);
-      a.row.scales[scale_off<SWZ>(a.row, b, row, tc)] = (uint8_t)sc;
-    }
-    if (COL) {
-      // the next row's codes, then byte c of an even lane = column c of rows
-      // (r, r+1)
-      const uint32_t n0 = __shfl_down_sync(0xffffffffu, codes[0], 1);
-      const uint32_t n1 = __shfl_down_sync(0xffffffffu, codes[1], 1);
-      if ((r & 1) == 0) {
-        const unsigned long long lo = zip_nibbles(codes[0], n0), hi = zip_nibbles(codes[1], n1);
-        *reinterpret_cast<uint4*>(trb + (r >> 1) * 16) =
-            make_uint4((uint32_t)lo, (uint32_t)(lo >> 32), (uint32_t)hi, (uint32_t)(hi >> 32));
-      }
-      __syncwarp();
-      if (r < 8) {  // lane r of the first 8: columns 2r, 2r+1, one byte per row pair
-        uint32_t v[8];
-#pragma unroll
-        for (int ii = 0; ii < 8; ++ii) v[ii] = *reinterpret_cast<const uint16_t*>(trb + ii * 16 + 2 * r);
-        const uint32_t t01 = __byte_perm(v[0], v[1], 0x5140), t23 = __byte_perm(v[2], v[3], 0x5140);
-        const uint32_t t45 = __byte_perm(v[4], v[5], 0x5140), t67 = __byte_perm(v[6], v[7], 0x5140);
-        if (valid) {
-          const long long c0 = (long long)tc * 16 + 2 * r;
-          store_codes8(a.col, b, c0, (long long)trow * 8, __byte_perm(t01, t23, 0x5410),
-                       __byte_perm(t45, t67, 0x5410));
-          store_codes8(a.col, b, c0 + 1, (long long)trow * 8, __byte_perm(t01, t23, 0x7632),
-                       __byte_perm(t45, t67, 0x7632));
-        }
-      }
-      if (valid) a.col.scales[scale_off<SWZ>(a.col, b, (long long)tc * 16 + r, trow)] = (uint8_t)sc;
-      __syncwarp();
-    }
-    if (F46 && ((ROW && a.row.choice) || (COL && a.col.choice))) {
-      const uint32_t bal = __ballot_sync(0xffffffffu, pick && valid && r == 0);
-      if (lane == 0 && bal) {
-        const uint32_t v2 = (bal & 1u) | ((bal >> 15) & 2u);
-        if (ROW && a.row.choice) {  // 2 consecutive tiles of tile row trow
-          const unsigned long long bit = ((unsigned long long)b * ntr + trow) * ntc + (unsigned long long)tq * 2;
-          unsigned int* wp = reinterpret_cast<unsigned int*>(a.row.choice) + (bit >> 5);
-          const unsigned long long vv = (unsigned long long)v2 << (bit & 31);
-          if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
-          if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
-        }
-        if (COL && a.col.choice) {  // tile (trow, tc) is tile (tc, trow) of x^T
-#pragma unroll
-          for (int gg = 0; gg < 2; ++gg) {
-            if (!((v2 >> gg) & 1u)) continue;
-            const unsigned long long bit = ((unsigned long long)b * ntc + tq * 2 + gg) * ntr + trow;
-            atomicOr(reinterpret_cast<unsigned int*>(a.col.choice) + (bit >> 5), 1u << (bit & 31));
-          }
-        }
-      }
-    }
-  }
-  badmax = __reduce_max_sync(0xffffffffu, badmax);
-  if (lane == 0 && badmax >= 0x7f800000u && a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
-}
-
-// --------------------------------------------------------------------------
-// 16x16 2D block scaling, warp-based.  grid (CTAs, batch); every warp takes
-// units of 4 horizontally adjacent tiles (tile row tr, tile columns 4u ..
-// 4u+3), 8 lanes per tile, lane i of a tile holding its rows 2i and 2i+1 as
-// the pair (A, B), loaded straight from global memory (32 bytes per row).
-// The tile amax and the tree over the 16 row error sums are 8-lane xor
-// shuffles; the transposed copy is zipped into bytes (rows 2i, 2i+1 of a
-// column) and transposed through this warp's own shared buffer, so the loop
-// has no CTA barrier.  Choice bits go into zeroed bitmaps with atomics.
-#ifndef FOS_2DW_MIN_BLOCKS
-#define FOS_2DW_MIN_BLOCKS 3
-#endif
-
-template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
-__global__ void __launch_bounds__(kThreads, FOS_2DW_MIN_BLOCKS) k_2d_warp(const QuantArgs a, FastDiv ntc4) {
-  __shared__ __align__(16) float4 s_tab[128];
-  __shared__ __align__(16) uint8_t s_tr[kThreads / 32][4 * kTrStride];
-  const int b = blockIdx.y;
-  const float St = tensor_scale_of(a, b, F46);
-  build_scale_table4(s_tab, St);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
-    if (COL && a.col.tensor_scale) a.col.tensor_scale[b] = St;
-  }
-  __syncthreads();
-  const TScale ts = make_tscale(St);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 3, i = lane & 7;
-  const uint32_t ntr = a.rows / 16, ntc = a.cols / 16;
-  const uint32_t nunits = ntr * ntc4.d;
-  const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
-  uint8_t* trb = s_tr[warp];
-  uint32_t badmax = 0;
-  for (uint32_t u = blockIdx.x * (kThreads / 32) + warp; u < nunits; u += gridDim.x * (kThreads / 32)) {
-    const uint32_t trow = fdiv(u, ntc4), tq = u - trow * ntc4.d;
-    const uint32_t tc = tq * 4 + g;
-    const bool valid = tc < ntc;  // uniform over the 8 lanes of a tile
-    const long long r0 = (long long)trow * 16 + 2 * i;
-    uint4 wa[2], wb[2];
-    if (valid) {
-      const uint4* pa = reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs + r0 * a.ld + (long long)tc * 16);
-      const uint4* pb = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(pa) + a.ld);
-      wa[0] = __ldg(pa); wa[1] = __ldg(pa + 1);
-      wb[0] = __ldg(pb); wb[1] = __ldg(pb + 1);
-    } else {
-      wa[0] = wa[1] = wb[0] = wb[1] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    float2 P[16];
-    unpack_pairs(wa, wb, P);
-    uint32_t m = max(amax_bits_bf16(wa), amax_bits_bf16(wb));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    badmax = max(badmax, m);
-    uint32_t s6, s4;
-    cand_scales<F46>(__uint_as_float(m), ts, s6, s4);
-    const float4 t6 = s_tab[s6];
-    const Cand c6 = candidate<F46>(P, make_float2(t6.x, t6.y), make_float2(t6.z, t6.w), a.neg_zero);
-    uint32_t ca[2] = {c6.ca[0], c6.ca[1]}, cb[2] = {c6.cb[0], c6.cb[1]};
-    uint32_t sc = s6;
-    float inv = t6.x;
-    bool pick = false;
-    if (F46) {
-      const float4 t4 = s_tab[s4];
-      const Cand c4 = candidate<true>(P, make_float2(t4.x, t4.y), make_float2(t4.z, t4.w), a.neg_zero);
-      // tree over the 16 row sums: rows (2i, 2i+1) here, then pairs of lanes
-      float e6 = __fadd_rn(c6.err.x, c6.err.y), e4 = __fadd_rn(c4.err.x, c4.err.y);
-#pragma unroll
-      for (int sh = 1; sh < 8; sh *= 2) {
-        e6 = __fadd_rn(e6, __shfl_xor_sync(0xffffffffu, e6, sh));
-        e4 = __fadd_rn(e4, __shfl_xor_sync(0xffffffffu, e4, sh));
-      }
-      pick = e4 < e6;  // strictly lower wins; ties keep 6
-      if (pick) { ca[0] = c4.ca[0]; ca[1] = c4.ca[1]; cb[0] = c4.cb[0]; cb[1] = c4.cb[1]; sc = s4; inv = t4.x; }
-    }
-    if (SR) {
-      sr_block(P, 0, inv, sr_bytes16(a.seed, gbase + r0 * a.cols + (long long)tc * 16), ca);
-      sr_block(P, 1, inv, sr_bytes16(a.seed, gbase + (r0 + 1) * a.cols + (long long)tc * 16), cb);
-    }
-    if (ROW && valid) {
-      store_codes8(a.row, b, r0, (long long)tc * 8, ca[0], ca[1]);
-      store_codes8(a.row, b, r0 + 1, (long long)tc * 8, cb[0], cb[1]);
-      a.row.scales[scale_off<SWZ>(a.row, b, r0, tc)] = (uint8_t)sc;
-      a.row.scales[scale_off<SWZ>(a.row, b, r0 + 1, tc)] = (uint8_t)sc;
-    }
-    if (COL) {
-      // byte c of lane i: column c of rows 2i (low nibble) and 2i+1 (high)
-      const unsigned long long lo = zip_nibbles(ca[0], cb[0]), hi = zip_nibbles(ca[1], cb[1]);
-      *reinterpret_cast<uint4*>(trb + g * kTrStride + i * 16) =
-          make_uint4((uint32_t)lo, (uint32_t)(lo >> 32), (uint32_t)hi, (uint32_t)(hi >> 32));
-      __syncwarp();
-      // lane i now takes columns 2i and 2i+1 of its tile: 8 bytes each, one
-      // per row pair
-      uint32_t v[8];
-#pragma unroll
-      for (int ii = 0; ii < 8; ++ii) v[ii] = *reinterpret_cast<const uint16_t*>(trb + g * kTrStride + ii * 16 + 2 * i);
-      __syncwarp();
-      const uint32_t t01 = __byte_perm(v[0], v[1], 0x5140), t23 = __byte_perm(v[2], v[3], 0x5140);
-      const uint32_t t45 = __byte_perm(v[4], v[5], 0x5140), t67 = __byte_perm(v[6], v[7], 0x5140);
-      if (valid) {
-        const long long c0 = (long long)tc * 16 + 2 * i;
-        store_codes8(a.col, b, c0, (long long)trow * 8, __byte_perm(t01, t23, 0x5410), __byte_perm(t45, t67, 0x5410));
-        store_codes8(a.col, b, c0 + 1, (long long)trow * 8, __byte_perm(t01, t23, 0x7632),
-                     __byte_perm(t45, t67, 0x7632));
-        a.col.scales[scale_off<SWZ>(a.col, b, c0, trow)] = (uint8_t)sc;
-        a.col.scales[scale_off<SWZ>(a.col, b, c0 + 1, trow)] = (uint8_t)sc;
-      }
-    }
-    if (F46 && ((ROW && a.row.choice) || (COL && a.col.choice))) {
-      const uint32_t bal = __ballot_sync(0xffffffffu, pick && valid && i == 0);
-      if (lane == 0 && bal) {
-        const uint32_t v4 = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u);
-        if (ROW && a.row.choice) {  // 4 consecutive tiles of tile row trow
-          const unsigned long long bit = ((unsigned long long)b * ntr + trow) * ntc + (unsigned long long)tq * 4;
-          unsigned int* wp = reinterpret_cast<unsigned int*>(a.row.choice) + (bit >> 5);
-          const unsigned long long vv = (unsigned long long)v4 << (bit & 31);
-          if ((uint32_t)vv) atomicOr(wp, (uint32_t)vv);
-          if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
-        }
-        if (COL && a.col.choice) {  // tile (trow, tc) is tile (tc, trow) of x^T
-#pragma unroll
-          for (int gg = 0; gg < 4; ++gg) {
-            if (!((v4 >> gg) & 1u)) continue;
-            const unsigned long long bit = ((unsigned long long)b * ntc + tq * 4 + gg) * ntr + trow;
-            atomicOr(reinterpret_cast<unsigned int*>(a.col.choice) + (bit >> 5), 1u << (bit & 31));
-          }
-        }
       }
     }
   }
@@ -951,17 +493,11 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
 cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
                               bool want_row, cudaStream_t st) {
   const bool f46 = fmt == 0;
-#if FOS_DUAL_WARP
   const uint32_t ntc4 = (uint32_t)((a.cols / 16 + 3) / 4);
   const uint32_t units = (uint32_t)(a.rows / 16) * ntc4;
   const FastDiv fd = make_fastdiv(ntc4);
   const dim3 g(min((units + kThreads / 32 - 1) / (kThreads / 32), 148u * 8u), (unsigned)batch);
 #define FOS_L(F, S, W, R) k_dual_warp<F, S, W, R><<<g, kThreads, 0, st>>>(a, fd)
-#else
-  const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * kStrip - 1) / (kSubRows * kStrip),
-               (unsigned)batch);
-#define FOS_L(F, S, W, R) k_dual1x16<F, S, W, R><<<g, kThreads, 0, st>>>(a)
-#endif
 #define FOS_R(F, S, W) do { if (want_row) FOS_L(F, S, W, true); else FOS_L(F, S, W, false); } while (0)
 #define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)
 #define FOS_S(F) do { if (sr) FOS_W(F, true); else FOS_W(F, false); } while (0)
@@ -977,23 +513,9 @@ cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, b
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz, bool want_row,
                           bool want_col, cudaStream_t st) {
   const bool f46 = fmt == 0;
-#if FOS_2D_WARP == 2
-  const uint32_t ntc2 = (uint32_t)((a.cols / 16 + 1) / 2);
-  const uint32_t units = (uint32_t)(a.rows / 16) * ntc2;
-  const FastDiv fd = make_fastdiv(ntc2);
-  const dim3 g(min((units + kThreads / 32 - 1) / (kThreads / 32), 148u * 10u), (unsigned)batch);
-#define FOS_L(F, S, W, R, C) k_2d_row<F, S, W, R, C><<<g, kThreads, 0, st>>>(a, fd)
-#elif FOS_2D_WARP
-  const uint32_t ntc4 = (uint32_t)((a.cols / 16 + 3) / 4);
-  const uint32_t units = (uint32_t)(a.rows / 16) * ntc4;
-  const FastDiv fd = make_fastdiv(ntc4);
-  const dim3 g(min((units + kThreads / 32 - 1) / (kThreads / 32), 148u * 8u), (unsigned)batch);
-#define FOS_L(F, S, W, R, C) k_2d_warp<F, S, W, R, C><<<g, kThreads, 0, st>>>(a, fd)
-#else
   const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * kStrip - 1) / (kSubRows * kStrip),
                (unsigned)batch);
 #define FOS_L(F, S, W, R, C) k_2d16x16<F, S, W, R, C><<<g, kThreads, 0, st>>>(a)
-#endif
 #define FOS_C(F, S, W, R) do { if (want_col) FOS_L(F, S, W, R, true); else FOS_L(F, S, W, R, false); } while (0)
 #define FOS_R(F, S, W) do { if (want_row) FOS_C(F, S, W, true); else FOS_C(F, S, W, false); } while (0)
 #define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)
