@@ -46,12 +46,13 @@ int fosck_div_tscale_random(unsigned long long seed, unsigned long long n,
                             unsigned long long* counts, void* stream);
 
 /* Every binary32 v in [0, 16] and +inf with every byte 0..255: the E2M1 code
- * of the integer form of the stochastic-rounding rule against the float
- * form.  counts[0] += mismatching pairs of codes. */
+ * of the integer form and of the pair (ceiling) form of the
+ * stochastic-rounding rule against the float form.  counts[0] += mismatching
+ * codes. */
 int fosck_sr_forms(unsigned long long* counts, void* stream);
 
 /* out[i] = E2M1 magnitude code of the stochastic rounding of v[i] with byte
- * bytes[i] (form 0: float form, 1: integer form), i < n. */
+ * bytes[i] (form 0: float form, 1: integer form, 2: pair form), i < n. */
 int fosck_sr_codes(const float* v, const uint8_t* bytes, long long n, int form, uint8_t* out,
                    void* stream);
 

@@ -143,7 +143,8 @@ __global__ void k_div_tscale_random(unsigned long long seed, unsigned long long 
 
 // ------------------------------------------------------------ SR
 // Every binary32 v in [0, 16] and +inf, with every byte: the E2M1 code of
-// the integer-form rule vs the float-form rule.
+// the integer-form rule and of the pair (ceiling) form vs the float-form
+// rule.
 __global__ void k_sr_forms(unsigned long long* counts) {
   unsigned long long bad = 0;
   const unsigned long long n = 0x41800001ull + 1;  // 0 .. 16.0, then +inf
@@ -155,7 +156,9 @@ __global__ void k_sr_forms(unsigned long long* counts) {
       const uint32_t c1 = e2m1x8(sr_e2m1_mag(v, byte), sr_e2m1_mag(v, byte + 1), 0, 0, 0, 0, 0, 0);
       const uint32_t c2 =
           e2m1x8(sr_e2m1_mag_bits(v, byte), sr_e2m1_mag_bits(v, byte + 1), 0, 0, 0, 0, 0, 0);
-      bad += (c1 != c2);
+      const float2 q = sr_e2m1_mag2(make_float2(v, v), sr_thr_bits(byte), sr_thr_bits(byte + 1));
+      const uint32_t c3 = e2m1x8(q.x, q.y, 0, 0, 0, 0, 0, 0);
+      bad += (c1 != c2) + (c1 != c3);
     }
   }
   if (bad) atomicAdd(counts, bad);
@@ -164,7 +167,8 @@ __global__ void k_sr_forms(unsigned long long* counts) {
 __global__ void k_sr_codes(const float* v, const uint8_t* bytes, long long n, int form, uint8_t* out) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
-    const float m = form ? sr_e2m1_mag_bits(v[i], bytes[i]) : sr_e2m1_mag(v[i], bytes[i]);
+    const float m = form == 2 ? sr_e2m1_mag2(make_float2(v[i], 0.0f), sr_thr_bits(bytes[i]), sr_thr_bits(0)).x
+                    : form ? sr_e2m1_mag_bits(v[i], bytes[i]) : sr_e2m1_mag(v[i], bytes[i]);
     out[i] = (uint8_t)(e2m1x8(m, 0, 0, 0, 0, 0, 0, 0) & 0xfu);
   }
 }

@@ -249,12 +249,16 @@ __device__ __forceinline__ Cand1 candidate1(const float2 (&P)[8], float inv, flo
 // B: which = 1) with 16 Philox bytes.
 __device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float inv, uint4 rnd,
                                          uint32_t (&out)[2]) {
+  const float2 inv2 = make_float2(inv, inv);
   float q[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float w = which ? P[i].y : P[i].x;
-    const float m = sr_e2m1_mag_bits(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
-    q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
+  for (int m = 0; m < 8; ++m) {  // elements 2m, 2m+1: bytes of word m / 2
+    const float w0 = which ? P[2 * m].y : P[2 * m].x, w1 = which ? P[2 * m + 1].y : P[2 * m + 1].x;
+    const uint32_t word = (m < 2) ? rnd.x : (m < 4) ? rnd.y : (m < 6) ? rnd.z : rnd.w;
+    const float2 r = sr_e2m1_mag2(mul2(make_float2(fabsf(w0), fabsf(w1)), inv2),
+                                  sr_thr_bits_of(word, (2 * m) & 3), sr_thr_bits_of(word, (2 * m + 1) & 3));
+    q[2 * m] = __uint_as_float(__float_as_uint(r.x) | (__float_as_uint(w0) & 0x80000000u));
+    q[2 * m + 1] = __uint_as_float(__float_as_uint(r.y) | (__float_as_uint(w1) & 0x80000000u));
   }
   out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
   out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
@@ -262,12 +266,16 @@ __device__ __forceinline__ void sr_block(const float2 (&P)[16], int which, float
 
 // Stochastic rounding of one block held as 8 split pairs.
 __device__ __forceinline__ void sr_block1(const float2 (&P)[8], float inv, uint4 rnd, uint32_t (&out)[2]) {
+  const float2 inv2 = make_float2(inv, inv);
   float q[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float w = (i < 8) ? P[i].x : P[i - 8].y;
-    const float m = sr_e2m1_mag(__fmul_rn(fabsf(w), inv), byte_of(rnd, i));
-    q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
+  for (int k = 0; k < 8; ++k) {  // P[k] = elements (k, k + 8): bytes k and k + 8
+    const float2 w = P[k];
+    const float2 r = sr_e2m1_mag2(mul2(make_float2(fabsf(w.x), fabsf(w.y)), inv2),
+                                  sr_thr_bits_of(k < 4 ? rnd.x : rnd.y, k & 3),
+                                  sr_thr_bits_of(k < 4 ? rnd.z : rnd.w, k & 3));
+    q[k] = __uint_as_float(__float_as_uint(r.x) | (__float_as_uint(w.x) & 0x80000000u));
+    q[k + 8] = __uint_as_float(__float_as_uint(r.y) | (__float_as_uint(w.y) & 0x80000000u));
   }
   out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
   out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);

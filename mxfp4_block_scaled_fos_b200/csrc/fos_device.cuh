@@ -187,11 +187,6 @@ __device__ __forceinline__ uint4 sr_bytes16(unsigned long long seed, long long g
                        seed_key(seed));
 }
 
-__device__ __forceinline__ uint32_t byte_of(uint4 r, int j) {
-  const uint32_t w = (j < 4) ? r.x : (j < 8) ? r.y : (j < 12) ? r.z : r.w;
-  return (w >> (8 * (j & 3))) & 0xffu;
-}
-
 // 16-bit mask of the random Hadamard signs: bit i set -> element i negated.
 __device__ __forceinline__ uint32_t rht_sign_mask(unsigned long long seed) {
   return philox4x32_10(make_uint4(0u, 0u, 1u, 0u), seed_key(seed)).x & 0xffffu;
@@ -234,6 +229,36 @@ __device__ __forceinline__ float sr_e2m1_mag_bits(float v, uint32_t byte) {
   const float tf = __fsub_rn(__uint_as_float(0x4B000000u | (2u * byte + 1u)), 8388608.0f);
   const uint32_t qs = (__fmul_rn(v, 1024.0f) > tf) ? 0x3F000000u : 0u;
   return __uint_as_float(bits >= 0x3F000000u ? qn : qs);
+}
+
+// The same rule for a pair of magnitudes, as a ceiling.  With step the grid
+// spacing at v (0.5 below 2, then 2^(e-1) for v in [2^e, 2^(e+1))), u = v /
+// step (exact: a power of two) and r = (2*byte+1)/512, the result is step *
+// ceil(u - r): ceil(u - r) = floor(u) + 1 exactly when frac(u) > r.  u - r
+// is exact (both are multiples of the smaller of ulp(u) and 2^-9, and where
+// the difference would need more than 24 bits it is negative, and any
+// rounding keeps it in (-1, 0)), so one fma forms it from v.  Values >= 6
+// come out as 6 or more and are clamped; +inf gives NaN at the fma, which
+// the clamp (fminf) turns into 6; a -0 ceiling becomes +0 through the +0
+// addend of the last fma.  R0, R1 carry the thresholds as the binary32 bits
+// of 2^14 + (2*byte+1)/512 (sr_thr_bits): subtracting from 2^14 is exact.
+__device__ __forceinline__ uint32_t sr_thr_bits(uint32_t byte) { return (byte << 1) | 0x46800001u; }
+
+// byte j (0..3) of w as sr_thr_bits
+__device__ __forceinline__ uint32_t sr_thr_bits_of(uint32_t w, int j) {
+  return ((j ? (w >> (8 * j - 1)) : (w << 1)) & 0x1feu) | 0x46800001u;
+}
+
+__device__ __forceinline__ float2 sr_e2m1_mag2(float2 v, uint32_t R0, uint32_t R1) {
+  const float2 rneg = sub2(make_float2(16384.0f, 16384.0f), make_float2(__uint_as_float(R0), __uint_as_float(R1)));
+  const int s0 = max((int)(__float_as_uint(v.x) & 0x7f800000u) - 0x00800000, 0x3f000000);
+  const int s1 = max((int)(__float_as_uint(v.y) & 0x7f800000u) - 0x00800000, 0x3f000000);
+  const float2 inv_step = make_float2(__uint_as_float(0x7f000000u - (uint32_t)s0),
+                                      __uint_as_float(0x7f000000u - (uint32_t)s1));
+  const float2 t = fma2(v, inv_step, rneg);
+  const float2 c = make_float2(ceilf(t.x), ceilf(t.y));
+  const float2 q = fma2(c, make_float2(__int_as_float(s0), __int_as_float(s1)), make_float2(0.0f, 0.0f));
+  return make_float2(fminf(q.x, 6.0f), fminf(q.y, 6.0f));
 }
 
 // ---------------------------------------------------------------- indexing

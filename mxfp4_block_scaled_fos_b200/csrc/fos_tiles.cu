@@ -78,12 +78,15 @@ __device__ __forceinline__ void store_codes8(const OutDesc& o, int b, long long 
 // Stochastic rounding of one block of a pair with explicit per-element bytes.
 __device__ __forceinline__ void sr_block_bytes(const float2 (&P)[16], int which, float inv,
                                                const uint32_t (&bytes)[16], uint32_t (&out)[2]) {
+  const float2 inv2 = make_float2(inv, inv);
   float q[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float w = which ? P[i].y : P[i].x;
-    const float m = sr_e2m1_mag_bits(__fmul_rn(fabsf(w), inv), bytes[i]);
-    q[i] = __uint_as_float(__float_as_uint(m) | (__float_as_uint(w) & 0x80000000u));
+  for (int m = 0; m < 8; ++m) {
+    const float w0 = which ? P[2 * m].y : P[2 * m].x, w1 = which ? P[2 * m + 1].y : P[2 * m + 1].x;
+    const float2 r = sr_e2m1_mag2(mul2(make_float2(fabsf(w0), fabsf(w1)), inv2), sr_thr_bits(bytes[2 * m]),
+                                  sr_thr_bits(bytes[2 * m + 1]));
+    q[2 * m] = __uint_as_float(__float_as_uint(r.x) | (__float_as_uint(w0) & 0x80000000u));
+    q[2 * m + 1] = __uint_as_float(__float_as_uint(r.y) | (__float_as_uint(w1) & 0x80000000u));
   }
   out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
   out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);

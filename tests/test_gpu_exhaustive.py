@@ -94,7 +94,7 @@ def test_div_tscale_random_binary32_pairs():
     assert c.tolist() == [0, 0], "a/S_t shortcut: %d code mismatches, %d quotient mismatches" % tuple(c.tolist())
 
 
-def test_sr_integer_form_equals_float_form_everywhere():
+def test_sr_integer_and_pair_forms_equal_float_form_everywhere():
     c = _counts(1)
     _run("fosck_sr_forms", _p(c))
     assert c.item() == 0, "SR forms differ on %d (v, byte) pairs" % c.item()
@@ -126,7 +126,7 @@ def test_sr_rule_matches_oracle():
     want = oracle.e2m1_sr(vv, bb)
     tv = torch.from_numpy(vv).to(dev)
     tb = torch.from_numpy(bb).to(dev)
-    for form in (0, 1):
+    for form in (0, 1, 2):
         out = torch.empty(vv.size, dtype=torch.uint8, device=dev)
         _run("fosck_sr_codes", _p(tv), _p(tb), vv.size, form, _p(out))
         got = out.cpu().numpy()
