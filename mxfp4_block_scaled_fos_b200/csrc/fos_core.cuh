@@ -415,6 +415,49 @@ __device__ __forceinline__ Cand1 candidate1_t(const float2 (&P)[8], const float4
   return r;
 }
 
+// The 4/6 (or 6-only) step of one block in split form (P[k] = elements k,
+// k + 8) with block amax bits m: codes, scale byte, whether the 4 candidate
+// was kept (strictly lower error; ties keep 6) and the kept candidate's
+// 1/E for a stochastic re-rounding.
+template <bool F46, int FAST = -1>
+__device__ __forceinline__ void block_step(const float2 (&P)[8], uint32_t m, const float4* s_tab,
+                                           const TScale& ts, float nz, uint32_t (&codes)[2], uint32_t& sc,
+                                           bool& pick, float& inv) {
+  uint32_t s6, s4;
+  cand_scales<F46, FAST>(__uint_as_float(m), ts, s6, s4);
+  const float4 t6 = s_tab[s6];
+  const Cand1 c6 = candidate1_t<F46>(P, t6, nz);
+  codes[0] = c6.c[0];
+  codes[1] = c6.c[1];
+  sc = s6;
+  inv = t6.x;
+  pick = false;
+  if (F46) {
+    const float4 t4 = s_tab[s4];
+    const Cand1 c4 = candidate1_t<true>(P, t4, nz);
+    pick = c4.err < c6.err;
+    if (pick) { codes[0] = c4.c[0]; codes[1] = c4.c[1]; sc = s4; inv = t4.x; }
+  }
+}
+
+// Stochastic re-rounding of a split-form block with the bytes of its
+// elements read from shared memory: element k's byte at bp[k * stride].
+__device__ __forceinline__ void sr_block1_smem(const float2 (&P)[8], float inv, const uint8_t* bp, int stride,
+                                               uint32_t (&out)[2]) {
+  const float2 inv2 = make_float2(inv, inv);
+  float q[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float2 w = P[k];
+    const float2 r = sr_e2m1_mag2(mul2(make_float2(fabsf(w.x), fabsf(w.y)), inv2), sr_thr_bits(bp[k * stride]),
+                                  sr_thr_bits(bp[(k + 8) * stride]));
+    q[k] = __uint_as_float(__float_as_uint(r.x) | (__float_as_uint(w.x) & 0x80000000u));
+    q[k + 8] = __uint_as_float(__float_as_uint(r.y) | (__float_as_uint(w.y) & 0x80000000u));
+  }
+  out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+  out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+}
+
 // Fake quantization of one block: the kept codes back to bf16 with the
 // dequantization rule y = bf16_RNE((q * float(s)) * S_t) (the first product
 // is exact), 16 values = 32 bytes to y.

@@ -75,23 +75,6 @@ __device__ __forceinline__ void store_codes8(const OutDesc& o, int b, long long 
       make_uint2(w0, w1);
 }
 
-// Stochastic rounding of one block of a pair with explicit per-element bytes.
-__device__ __forceinline__ void sr_block_bytes(const float2 (&P)[16], int which, float inv,
-                                               const uint32_t (&bytes)[16], uint32_t (&out)[2]) {
-  const float2 inv2 = make_float2(inv, inv);
-  float q[16];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const float w0 = which ? P[2 * m].y : P[2 * m].x, w1 = which ? P[2 * m + 1].y : P[2 * m + 1].x;
-    const float2 r = sr_e2m1_mag2(mul2(make_float2(fabsf(w0), fabsf(w1)), inv2), sr_thr_bits(bytes[2 * m]),
-                                  sr_thr_bits(bytes[2 * m + 1]));
-    q[2 * m] = __uint_as_float(__float_as_uint(r.x) | (__float_as_uint(w0) & 0x80000000u));
-    q[2 * m + 1] = __uint_as_float(__float_as_uint(r.y) | (__float_as_uint(w1) & 0x80000000u));
-  }
-  out[0] = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-  out[1] = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-}
-
 // Quantize the pair P (blocks A, B) with per-block amax bits (ma, mb):
 // returns codes, scale bytes and picks (SR re-rounding done by the caller).
 template <bool F46>
@@ -124,29 +107,6 @@ __device__ __forceinline__ PairResult<F46> quant_pair(const float2 (&P)[16], uin
   return r;
 }
 
-// quant_pair with the (inv, inv, -E, -E) table of build_scale_table4.
-template <bool F46>
-__device__ __forceinline__ PairResult<F46> quant_pair4(const float2 (&P)[16], uint32_t ma, uint32_t mb,
-                                                       const TScale& St, const float4* tab, float nz) {
-  PairResult<F46> r;
-  uint32_t s6a, s4a, s6b, s4b;
-  cand_scales<F46>(__uint_as_float(ma), St, s6a, s4a);
-  cand_scales<F46>(__uint_as_float(mb), St, s6b, s4b);
-  const float4 t6a = tab[s6a], t6b = tab[s6b];
-  const Cand c6 = candidate<F46>(P, make_float2(t6a.x, t6b.x), make_float2(t6a.z, t6b.z), nz);
-  r.ca[0] = c6.ca[0]; r.ca[1] = c6.ca[1]; r.cb[0] = c6.cb[0]; r.cb[1] = c6.cb[1];
-  r.sa = s6a; r.sb = s6b; r.inva = t6a.x; r.invb = t6b.x; r.pa = 0; r.pb = 0;
-  if (F46) {
-    const float4 t4a = tab[s4a], t4b = tab[s4b];
-    const Cand c4 = candidate<true>(P, make_float2(t4a.x, t4b.x), make_float2(t4a.z, t4b.z), nz);
-    r.pa = c4.err.x < c6.err.x;
-    r.pb = c4.err.y < c6.err.y;
-    if (r.pa) { r.ca[0] = c4.ca[0]; r.ca[1] = c4.ca[1]; r.sa = s4a; r.inva = t4a.x; }
-    if (r.pb) { r.cb[0] = c4.cb[0]; r.cb[1] = c4.cb[1]; r.sb = s4b; r.invb = t4b.x; }
-  }
-  return r;
-}
-
 // Nibbles of a (8) into the low halves of 8 bytes, b into the high halves:
 // byte k = a_k | b_k << 4.
 __device__ __forceinline__ unsigned long long zip_nibbles(uint32_t a, uint32_t b) {
@@ -162,10 +122,11 @@ __device__ __forceinline__ unsigned long long zip_nibbles(uint32_t a, uint32_t b
 // --------------------------------------------------------------------------
 // 1x16 rowwise + colwise from one read, warp-based.  grid (CTAs, batch);
 // every warp takes units of 4 horizontally adjacent 16x16 tiles, 8 lanes per
-// tile.  Lane i of a tile first holds the tile's rows 2i and 2i+1 as a pair
-// of rowwise blocks; the tile then goes through this warp's shared buffer so
-// that lane j holds its columns 2j and 2j+1 as a pair of colwise blocks.
-// With stochastic rounding the Philox bytes of each rowwise block (one call
+// tile.  Lane i of a tile first quantizes the tile's rows 2i and 2i+1 (one
+// rowwise block each); the tile then goes through this warp's shared buffer
+// so that lane j quantizes its columns 2j and 2j+1 (one colwise block each).
+// Blocks go one at a time through the rowwise quantizer's per-block step,
+// which keeps the kernel at 3 CTAs per SM with stochastic rounding.  With stochastic rounding the Philox bytes of each rowwise block (one call
 // per 16 consecutive elements) take the same way, so both orientations use
 // the byte of the same source element.  Choice bits go into zeroed bitmaps
 // with atomics.  No CTA barrier in the loop.
@@ -174,6 +135,9 @@ constexpr int kDwGroup = 16 * 32 + 32;   // bytes per tile in the buffer: 16 row
                                          // reads fall into distinct banks
 #ifndef FOS_DUALW_MIN_BLOCKS
 #define FOS_DUALW_MIN_BLOCKS 3
+#endif
+#ifndef FOS_DUALW_MIN_BLOCKS_SR
+#define FOS_DUALW_MIN_BLOCKS_SR 3
 #endif
 
 // 4 bits at lanes i, 8+i, 16+i, 24+i of a ballot -> bits 0..3
@@ -190,8 +154,31 @@ __device__ __forceinline__ void or_bits(uint8_t* bitmap, unsigned long long bit,
   if ((uint32_t)(vv >> 32)) atomicOr(wp + 1, (uint32_t)(vv >> 32));
 }
 
+// One rowwise block of the dual kernel: row R of the tile at tile column
+// tc, words w, Philox bytes rnd of its 16 elements.  Returns the 4/6 pick.
+template <bool F46, bool SR, bool SWZ>
+__device__ __forceinline__ uint32_t dual_row_block(const QuantArgs& a, int b, const uint4 (&w)[2], uint4 rnd,
+                                                   long long R, uint32_t tc, bool valid, const float4* s_tab,
+                                                   const TScale& ts, uint32_t& badmax) {
+  const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+  float2 P[8];
+  unpack_split(W, P);
+  const uint32_t m = amax_bits_bf16(w);
+  badmax = max(badmax, m);
+  uint32_t codes[2], sc;
+  bool pick;
+  float inv;
+  block_step<F46>(P, m, s_tab, ts, a.neg_zero, codes, sc, pick, inv);
+  if (SR) sr_block1(P, inv, rnd, codes);
+  if (valid) {
+    store_codes8(a.row, b, R, (long long)tc * 8, codes[0], codes[1]);
+    a.row.scales[scale_off<SWZ>(a.row, b, R, tc)] = (uint8_t)sc;
+  }
+  return pick && valid;
+}
+
 template <bool F46, bool SR, bool SWZ, bool ROW>
-__global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_DUALW_MIN_BLOCKS) k_dual_warp(const QuantArgs a, FastDiv ntc4) {
+__global__ void __launch_bounds__(kThreads, SR ? FOS_DUALW_MIN_BLOCKS_SR : FOS_DUALW_MIN_BLOCKS) k_dual_warp(const QuantArgs a, FastDiv ntc4) {
   __shared__ __align__(16) float4 s_tab[128];
   __shared__ __align__(16) uint8_t s_x[kThreads / 32][4 * kDwGroup];
   __shared__ __align__(16) uint8_t s_r[SR ? kThreads / 32 : 1][SR ? 4 * 256 : 16];
@@ -238,65 +225,44 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_DUALW_MIN_BLOCKS) k_dua
       reinterpret_cast<uint4*>(rbuf)[2 * i] = ra;
       reinterpret_cast<uint4*>(rbuf)[2 * i + 1] = rb;
     }
-    // ---------------- rowwise: blocks (row 2i) and (row 2i+1) as a pair
+    // ---------------- rowwise: row 2i, then row 2i+1, one block each
     uint32_t pra = 0, prb = 0;
     if (ROW) {
-      float2 P[16];
-      unpack_pairs(wa, wb, P);
-      const uint32_t ma = amax_bits_bf16(wa), mb = amax_bits_bf16(wb);
-      badmax = max(badmax, max(ma, mb));
-      PairResult<F46> q = quant_pair4<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
-      if (SR) {
-        sr_block(P, 0, q.inva, ra, q.ca);
-        sr_block(P, 1, q.invb, rb, q.cb);
-      }
-      if (valid) {
-        store_codes8(a.row, b, r0, (long long)tc * 8, q.ca[0], q.ca[1]);
-        store_codes8(a.row, b, r0 + 1, (long long)tc * 8, q.cb[0], q.cb[1]);
-        a.row.scales[scale_off<SWZ>(a.row, b, r0, tc)] = (uint8_t)q.sa;
-        a.row.scales[scale_off<SWZ>(a.row, b, r0 + 1, tc)] = (uint8_t)q.sb;
-      }
-      pra = q.pa && valid;
-      prb = q.pb && valid;
+      pra = dual_row_block<F46, SR, SWZ>(a, b, wa, ra, r0, tc, valid, s_tab, ts, badmax);
+      prb = dual_row_block<F46, SR, SWZ>(a, b, wb, rb, r0 + 1, tc, valid, s_tab, ts, badmax);
     }
     __syncwarp();
-    // ---------------- colwise: columns 2i and 2i+1 of the tile as a pair
+    // ---------------- colwise: column 2i, then column 2i+1 of the tile
     uint32_t pca = 0, pcb = 0;
     {
-      uint32_t w[16];
+      uint32_t w[16];  // row r of the tile's columns 2i (low half) and 2i+1 (high half)
 #pragma unroll
       for (int r = 0; r < 16; ++r) w[r] = *reinterpret_cast<const uint32_t*>(xb + r * 32 + 4 * i);
-      float2 P[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) P[r] = make_float2(bf_lo(w[r]), bf_hi(w[r]));
       uint32_t h[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) h[k] = hmax_abs2(w[2 * k], w[2 * k + 1]);
       const uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(h[0], h[1]), hmax_abs2(h[2], h[3])),
                                    hmax_abs2(hmax_abs2(h[4], h[5]), hmax_abs2(h[6], h[7]))) & 0x7fff7fffu;
-      const uint32_t ma = (m & 0xffffu) << 16, mb = m & 0xffff0000u;
-      badmax = max(badmax, max(ma, mb));
-      PairResult<F46> q = quant_pair4<F46>(P, ma, mb, ts, s_tab, a.neg_zero);
-      if (SR) {
-        uint32_t ba[16], bb[16];
+      const uint32_t mc[2] = {(m & 0xffffu) << 16, m & 0xffff0000u};
+      badmax = max(badmax, max(mc[0], mc[1]));
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const uint32_t two = *reinterpret_cast<const uint16_t*>(rbuf + r * 16 + 2 * i);
-          ba[r] = two & 0xffu;
-          bb[r] = two >> 8;
+      for (int hc = 0; hc < 2; ++hc) {
+        float2 P[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          P[k] = hc ? make_float2(bf_hi(w[k]), bf_hi(w[k + 8])) : make_float2(bf_lo(w[k]), bf_lo(w[k + 8]));
+        uint32_t codes[2], sc;
+        bool pick;
+        float inv;
+        block_step<F46>(P, mc[hc], s_tab, ts, a.neg_zero, codes, sc, pick, inv);
+        if (SR) sr_block1_smem(P, inv, rbuf + 2 * i + hc, 16, codes);
+        const long long c = (long long)tc * 16 + 2 * i + hc;
+        if (valid) {
+          store_codes8(a.col, b, c, (long long)trow * 8, codes[0], codes[1]);
+          a.col.scales[scale_off<SWZ>(a.col, b, c, trow)] = (uint8_t)sc;
         }
-        sr_block_bytes(P, 0, q.inva, ba, q.ca);
-        sr_block_bytes(P, 1, q.invb, bb, q.cb);
+        (hc ? pcb : pca) = pick && valid;
       }
-      if (valid) {
-        const long long c0 = (long long)tc * 16 + 2 * i;
-        store_codes8(a.col, b, c0, (long long)trow * 8, q.ca[0], q.ca[1]);
-        store_codes8(a.col, b, c0 + 1, (long long)trow * 8, q.cb[0], q.cb[1]);
-        a.col.scales[scale_off<SWZ>(a.col, b, c0, trow)] = (uint8_t)q.sa;
-        a.col.scales[scale_off<SWZ>(a.col, b, c0 + 1, trow)] = (uint8_t)q.sb;
-      }
-      pca = q.pa && valid;
-      pcb = q.pb && valid;
     }
     __syncwarp();  // the buffers are rewritten by the next unit
     if (F46) {
