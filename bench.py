@@ -191,15 +191,22 @@ def time_loop(fn, steps, warmup, world, stream):
 TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def source_hash() -> str:
-    """SHA-256 over the CUDA sources, to tell whether a profile is current."""
-    import glob
+# The sources each profiled kernel is built from: a profile stays current
+# while these files are unchanged.
+KERNEL_SOURCES = {
+    "k_q1x16_fused_moe_experts": ["csrc/fos_rowwise.cu", "csrc/fos_core.cuh", "csrc/fos_device.cuh",
+                                  "csrc/fos_internal.h"],
+}
+
+
+def source_hash(kernel: str = "k_q1x16_fused_moe_experts") -> str:
+    """SHA-256 over the sources `kernel` is built from (and the public header),
+    to tell whether its profile is current."""
     import hashlib
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "mxfp4_block_scaled_fos_b200", "csrc")
-    for fn in sorted(glob.glob(os.path.join(csrc, "*"))):
-        if not os.path.isfile(fn):
-            continue
+    pkg = os.path.join(ROOT, "mxfp4_block_scaled_fos_b200")
+    files = [os.path.join(pkg, f) for f in KERNEL_SOURCES[kernel]] + [os.path.join(ROOT, "include", "fos.h")]
+    for fn in files:
         with open(fn, "rb") as f:
             h.update(os.path.basename(fn).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
@@ -212,7 +219,7 @@ def profiled_traffic(kernel, elems):
     try:
         with open(TRAFFIC_JSON) as f:
             d = json.load(f)[kernel]
-        if d.get("source_sha256") != source_hash():
+        if d.get("source_sha256") != source_hash(kernel):
             return None
         return int(float(d["dram_bytes_per_element"]) * elems)
     except (OSError, KeyError, ValueError, TypeError):
