@@ -212,6 +212,27 @@ def source_hash(kernel: str = "k_q1x16_fused_moe_experts") -> str:
     return h.hexdigest()[:16]
 
 
+def issue_bound(kernel, elems, ms, sm_mhz, sms=148):
+    """The issue-slot roofline of `kernel` for a launch over `elems` elements
+    taking `ms`: warp instructions per element from its ncu capture
+    (profiles/traffic.json, smsp__inst_executed.sum over the captured
+    elements), against 4 warp schedulers per SM each issuing one warp
+    instruction per cycle at the sampled SM clock.  None if the sources
+    changed since the capture."""
+    try:
+        with open(TRAFFIC_JSON) as f:
+            d = json.load(f)[kernel]
+        if d.get("source_sha256") != source_hash(kernel):
+            return None
+        wi = float(d["warp_instructions_per_element"]) * elems
+    except (OSError, KeyError, ValueError, TypeError):
+        return None
+    slots_per_s = sms * 4 * sm_mhz * 1e6
+    min_ms = wi / slots_per_s * 1e3
+    return {"warp_instructions_per_launch": int(wi), "issue_slots_per_s": slots_per_s,
+            "min_ms": round(min_ms, 4), "frac": round(min_ms / ms, 4)}
+
+
 def profiled_traffic(kernel, elems):
     """DRAM bytes per launch of `kernel` from profiles/traffic.json (its ncu
     capture's dram__bytes_read.sum + dram__bytes_write.sum per element,
@@ -344,6 +365,10 @@ def run_fos(args, world, rank):
         "clocks": clocks,
         "modes": extra,
     }
+    issue = issue_bound("k_q1x16_fused_moe_experts", elems, ms_per_step,
+                        clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0)
+    if issue is not None:
+        out["roofline"]["issue"] = issue
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_cpu = max(4, min(E, host_cores()))
         xs = workloads.bits(x[:n_cpu])
