@@ -495,6 +495,34 @@ def measure_modes(args, world, x, dev, stream, peak):
     except Exception as e:
         res["gemm_error"] = repr(e)
     torch.cuda.empty_cache()
+    # a quantized Linear layer, 8192 tokens x 4096 -> 4096: the forward GEMM,
+    # then dgrad and wgrad, with every operand quantized inside the step
+    # (x 1x16 rowwise and along M, dy with SR in both orientations); the 2D
+    # weight quantization is done once, outside the step
+    try:
+        peak_tf, peak_src = fp4_peak_tflops()
+        M_, N_, K_ = 8192, 4096, 4096
+        xl = workloads.activation_outliers(M_, K_, device=dev)
+        wl = workloads.weight_normal(N_, K_, device=dev)
+        dyl = workloads.gradient_student_t(M_, N_, device=dev)
+        qw = F.quantize_weight(wl)
+
+        def layer_step():
+            F.linear_forward(xl, qw)
+            F.linear_backward(dyl, xl, qw, seed=7)
+
+        ms = time_loop(layer_step, n, 3, world, stream) / n
+        tf = 3 * 2.0 * M_ * N_ * K_ / (ms * 1e-3) / 1e12
+        res["linear_layer_fwd_bwd"] = {"ms": round(ms, 4), "TFLOP_s": round(tf, 1),
+                                       "frac": round(tf / peak_tf, 4), "peak_TFLOP_s": peak_tf,
+                                       "peak_source": peak_src, "shape": [M_, N_, K_],
+                                       "note": "3 GEMMs (forward, dgrad, wgrad) + the quantization of "
+                                               "x (both orientations) and dy (SR, both orientations) per "
+                                               "step; f32 gradients, bf16 y"}
+        del xl, wl, dyl, qw
+    except Exception as e:
+        res["linear_error"] = repr(e)
+    torch.cuda.empty_cache()
     return res
 
 
