@@ -11,21 +11,28 @@
 // Hugging Face transformers doc "Four Over Six", introduction (the codes
 // feed FP4 GEMMs on Blackwell).
 //
-// Persistent: one CTA per SM walks 128 x 128 tiles of D (grouped by 8 tile
-// rows for L2 reuse of B) with 6 warps:
+// Persistent: one CTA per SM walks 128 x 256 tiles of D (128 x 128 when N
+// is not a multiple of 256), grouped by 8 tile rows for L2 reuse of B, with
+// 6 warps:
 //   warp 0     TMA producer: per 256-wide K step, the A and B code tiles
 //              (128 rows x 128 bytes each, 128-byte swizzle) as 2D tensor
 //              copies and the four 512-byte scale atoms of each as one
-//              2 KB bulk copy, into a 6-stage shared-memory ring;
+//              2 KB bulk copy per 128 rows, into a 4-stage (6 for 128 x 128)
+//              shared-memory ring;
 //   warp 1     allocates the tensor memory; one thread copies the stage's
 //              scale atoms into tensor memory (tcgen05.cp 32x128b.warpx4)
 //              and issues the four K=64 tcgen05.mma of the stage
 //              (kind::mxf4nvf4, block16, f32 accumulator in tensor memory);
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp its
 //              32-lane quarter), scale by S_tA * S_tB, store bf16 or f32.
-// The accumulator is double-buffered in tensor memory (2 x 128 columns), so
-// the epilogue of one tile runs while the MMAs of the next one are issued;
-// the shared-memory ring and its barriers run on across tiles.
+// Every tcgen05.mma (and every scale copy) holds the tensor pipe for about
+// the same time whatever its N, so the 256-wide tile does twice the work per
+// instruction: 8192^3 in 0.387 ms against 0.571 ms with 128 x 128 tiles.
+// Its accumulator takes 256 of the 512 tensor-memory columns and the scale
+// buffers most of the rest, so it is single-buffered: the epilogue releases
+// it as soon as its last columns are in registers.  128 x 128 tiles keep two
+// accumulators, so that a tile's epilogue runs while the next one's MMAs are
+// issued.  The shared-memory ring and its barriers run on across tiles.
 // Every mbarrier wait is bounded: after the limit the kernel sets
 // FOS_STATUS_TIMEOUT, stops issuing work, waits (bounded) for its own copies
 // in flight, frees its tensor memory and returns.
@@ -41,27 +48,47 @@ namespace fos {
 
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 256;      // BK in FP4 elements (128 bytes)
-constexpr int kStages = 6;
+constexpr int BM = 128, BK = 256;                // BK in FP4 elements (128 bytes)
 constexpr int kTileA = BM * BK / 2;              // 16384 bytes
-constexpr int kTileB = BN * BK / 2;              // 16384 bytes
-constexpr int kSFTile = 2048;                    // 4 atoms of 128 rows x 4 scales
-constexpr uint32_t kStageTx = kTileA + kTileB + 2 * kSFTile;
+constexpr int kSFRowTile = 2048;                 // one 128-row tile's 4 scale atoms per K step
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;              // 2 accumulators of 128 + scale buffers 64
-constexpr uint32_t kColSFA = 256, kColSFB = 288; // + 16 * (k step & 1)
+constexpr uint32_t kTmemCols = 512;
 constexpr int kGroupM = 8;                       // tile rows per group of the tile order
 constexpr uint32_t kWaitLimit = 1u << 22;        // polls of one mbarrier wait
 
-// dynamic shared memory layout (from a 1024-byte aligned base)
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kStages * kTileA;
-constexpr int kOffSFA = kOffB + kStages * kTileB;
-constexpr int kOffSFB = kOffSFA + kStages * kSFTile;
-constexpr int kOffBar = kOffSFB + kStages * kSFTile;   // full[S], empty[S], acc_full[2], acc_empty[2]
-constexpr int kOffTmem = kOffBar + (2 * kStages + 4) * 8;
-constexpr int kOffFlag = kOffTmem + 8;
-constexpr int kSmemBytes = kOffFlag + 8 + 1024;        // + alignment slack
+// The tile shape BM x BN of one CTA and what follows from it.  BN = 256
+// gives each tcgen05.mma twice the work of BN = 128 for the same issue cost
+// (measured: an N = 256 MMA takes as long as an N = 128 one here), at the
+// price of one accumulator buffer instead of two: 256 tensor-memory columns
+// of accumulator leave room only for the scale buffers.
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = BN == 128 ? 6 : 4;
+  static constexpr int kTileB = BN * BK / 2;
+  static constexpr int kSFB = (BN / 128) * kSFRowTile;   // B scales per stage
+  static constexpr uint32_t kStageTx = kTileA + kTileB + kSFRowTile + kSFB;
+  static constexpr int kAcc = BN == 128 ? 2 : 1;         // accumulator buffers (kAcc * BN <= 256 columns)
+  // tensor memory: accumulators from column 0; A scales 256 + 16 * (k step &
+  // 1) (4 columns per K-64 group); B scales 288 + (BN / 8) * (k step & 1)
+  // (BN / 32 columns per K-64 group: 4 per 128 rows)
+  static constexpr uint32_t kColSFA = 256, kColSFB = 288;
+  static constexpr uint32_t kSFBGroup = BN / 32;
+  // dynamic shared memory layout (from a 1024-byte aligned base)
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kTileA;
+  static constexpr int kOffSFA = kOffB + kStages * kTileB;
+  static constexpr int kOffSFB = kOffSFA + kStages * kSFRowTile;
+  static constexpr int kOffBar = kOffSFB + kStages * kSFB;  // full[S], empty[S], acc_full[2], acc_empty[2]
+  static constexpr int kOffTmem = kOffBar + (2 * kStages + 4) * 8;
+  static constexpr int kOffFlag = kOffTmem + 8;
+  static constexpr int kSmemBytes = kOffFlag + 8 + 1024;    // + alignment slack
+  // instruction descriptor: kind::mxf4nvf4, A and B E2M1, K-major, UE4M3
+  // scales, M = 128, N = BN, K = 64 per instruction
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                     ((uint32_t)(BM >> 4) << 24);
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kColSFB + 2 * (BN / 8) <= kTmemCols && kAcc * BN <= 256, "tensor memory");
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -114,17 +141,13 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
          ((uint64_t)1 << 46);
 }
 
-// Instruction descriptor: kind::mxf4nvf4, A and B E2M1, K-major, UE4M3
-// scales, M = 128, N = 128, K = 64 per instruction.
-constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-
-__device__ __forceinline__ void umma(uint32_t tmem_c, uint64_t da, uint64_t db, uint32_t tsfa, uint32_t tsfb,
-                                     uint32_t accumulate) {
+__device__ __forceinline__ void umma(uint32_t tmem_c, uint64_t da, uint64_t db, uint32_t idesc, uint32_t tsfa,
+                                     uint32_t tsfb, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-      :: "r"(tmem_c), "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate), "r"(tsfa), "r"(tsfb) : "memory");
+      :: "r"(tmem_c), "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb) : "memory");
 }
 
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
@@ -160,22 +183,25 @@ __device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int& tm, in
   tn = r / gm;
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_nvfp4(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const GemmArgs g) {
+  using C = Cfg<BN>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + kOffBar, bar_empty = bar_full + 8 * kStages;
-  const uint32_t bar_accf = bar_empty + 8 * kStages, bar_acce = bar_accf + 16;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
-  volatile uint32_t* fail = reinterpret_cast<volatile uint32_t*>(smem + kOffFlag);
+  const uint32_t bar_full = sbase + C::kOffBar, bar_empty = bar_full + 8 * S;
+  const uint32_t bar_accf = bar_empty + 8 * S, bar_acce = bar_accf + 16;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
+  volatile uint32_t* fail = reinterpret_cast<volatile uint32_t*>(smem + C::kOffFlag);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ksteps = g.K / BK;
   const int ntm = g.M / BM, ntn = g.N / BN, ntiles = ntm * ntn;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
@@ -188,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 1) {  // tensor memory for the accumulators and the scale buffers
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 :: "r"(sbase + kOffTmem), "r"(kTmemCols) : "memory");
+                 :: "r"(sbase + C::kOffTmem), "r"(kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -204,48 +230,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tm, tn;
         tile_coords(t, ntm, ntn, tm, tn);
         for (int kt = 0; kt < ksteps; ++kt, ++it) {
-          const int s = it % kStages;
-          if (it >= kStages && !mbar_wait(bar_empty + 8 * s, ((it / kStages) - 1) & 1)) { *fail = 1; break; }
+          const int s = it % S;
+          if (it >= S && !mbar_wait(bar_empty + 8 * s, ((it / S) - 1) & 1)) { *fail = 1; break; }
           const uint32_t fb = bar_full + 8 * s;
-          mbar_expect_tx(fb, kStageTx);
-          tma_load_2d(sbase + kOffA + s * kTileA, &map_a, kt * (BK / 2), tm * BM, fb);
-          tma_load_2d(sbase + kOffB + s * kTileB, &map_b, kt * (BK / 2), tn * BN, fb);
-          // the 4 scale atoms of rows [128 tile, +128) and scale columns [16 kt, +16)
-          bulk_load(sbase + kOffSFA + s * kSFTile, g.sfa + ((long long)tm * g.sf_col_tiles + 4 * kt) * 512,
-                    kSFTile, fb);
-          bulk_load(sbase + kOffSFB + s * kSFTile, g.sfb + ((long long)tn * g.sf_col_tiles + 4 * kt) * 512,
-                    kSFTile, fb);
+          mbar_expect_tx(fb, C::kStageTx);
+          tma_load_2d(sbase + C::kOffA + s * kTileA, &map_a, kt * (BK / 2), tm * BM, fb);
+          tma_load_2d(sbase + C::kOffB + s * C::kTileB, &map_b, kt * (BK / 2), tn * BN, fb);
+          // the 4 scale atoms of each 128-row tile, scale columns [16 kt, +16)
+          bulk_load(sbase + C::kOffSFA + s * kSFRowTile, g.sfa + ((long long)tm * g.sf_col_tiles + 4 * kt) * 512,
+                    kSFRowTile, fb);
+#pragma unroll
+          for (int h = 0; h < BN / 128; ++h)
+            bulk_load(sbase + C::kOffSFB + s * C::kSFB + h * kSFRowTile,
+                      g.sfb + ((long long)(tn * (BN / 128) + h) * g.sf_col_tiles + 4 * kt) * 512, kSFRowTile, fb);
         }
       }
       // before leaving, every copy this thread started must have landed
-      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j)
-        if (!mbar_wait(bar_full + 8 * (j % kStages), (j / kStages) & 1)) *fail = 1;
+      for (int j = (it > S ? it - S : 0); j < it; ++j)
+        if (!mbar_wait(bar_full + 8 * (j % S), (j / S) & 1)) *fail = 1;
     }
   } else if (warp == 1) {
     if (lane == 0) {
       int it = 0, lt = 0;
       for (int t = blockIdx.x; t < ntiles && !*fail; t += gridDim.x, ++lt) {
-        const int acc = lt & 1;
-        // the epilogue must have drained this accumulator (tile lt - 2)
-        if (lt >= 2 && !mbar_wait(bar_acce + 8 * acc, ((lt >> 1) - 1) & 1)) { *fail = 1; break; }
+        const int acc = lt % C::kAcc;
+        // the epilogue must have drained this accumulator (tile lt - kAcc)
+        if (lt >= C::kAcc && !mbar_wait(bar_acce + 8 * acc, ((lt / C::kAcc) - 1) & 1)) { *fail = 1; break; }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t tacc = tmem + (uint32_t)(acc * BN);
         for (int kt = 0; kt < ksteps; ++kt, ++it) {
-          const int s = it % kStages;
-          if (*fail || !mbar_wait(bar_full + 8 * s, (it / kStages) & 1)) { *fail = 1; break; }
+          const int s = it % S;
+          if (*fail || !mbar_wait(bar_full + 8 * s, (it / S) & 1)) { *fail = 1; break; }
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          const uint32_t buf = 16u * (it & 1);
+          const uint32_t sfa = tmem + C::kColSFA + 16u * (it & 1);
+          const uint32_t sfb = tmem + C::kColSFB + 4u * C::kSFBGroup * (it & 1);
+          // scale atom j of each 128-row tile h -> 4 columns (K-64 group j);
+          // B's groups hold BN / 32 columns, its row tiles 4 columns apart
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            tmem_cp_sf(tmem + kColSFA + buf + 4 * j, desc_sf(sbase + kOffSFA + s * kSFTile + 512 * j));
-            tmem_cp_sf(tmem + kColSFB + buf + 4 * j, desc_sf(sbase + kOffSFB + s * kSFTile + 512 * j));
+            tmem_cp_sf(sfa + 4 * j, desc_sf(sbase + C::kOffSFA + s * kSFRowTile + 512 * j));
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h)
+              tmem_cp_sf(sfb + C::kSFBGroup * j + 4 * h,
+                         desc_sf(sbase + C::kOffSFB + s * C::kSFB + h * kSFRowTile + 512 * j));
           }
-          const uint64_t da = desc_sw128(sbase + kOffA + s * kTileA);
-          const uint64_t db = desc_sw128(sbase + kOffB + s * kTileB);
+          const uint64_t da = desc_sw128(sbase + C::kOffA + s * kTileA);
+          const uint64_t db = desc_sw128(sbase + C::kOffB + s * C::kTileB);
 #pragma unroll
           for (int j = 0; j < 4; ++j)  // K = 64 (32 bytes) per instruction
-            umma(tacc, da + 2 * j, db + 2 * j, tmem + kColSFA + buf + 4 * j, tmem + kColSFB + buf + 4 * j,
-                 (kt | j) != 0);
+            umma(tacc, da + 2 * j, db + 2 * j, C::kIdesc, sfa + 4 * j, sfb + C::kSFBGroup * j, (kt | j) != 0);
           umma_commit(bar_empty + 8 * s);  // the stage's smem is free once these MMAs are done
         }
         umma_commit(bar_accf + 8 * acc);  // this tile's accumulator is complete
@@ -257,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float alpha = __fmul_rn(g.sta[0], g.stb[0]);
     int lt = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
-      const int acc = lt & 1;
-      const bool ok = mbar_wait(bar_accf + 8 * acc, (lt >> 1) & 1);
+      const int acc = lt % C::kAcc;
+      const bool ok = mbar_wait(bar_accf + 8 * acc, (lt / C::kAcc) & 1);
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       if (!ok) *fail = 1;
       if (!ok || *fail) break;
@@ -278,6 +311,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
             : "r"(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN + c0)));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (c0 + 32 == BN) {
+          // the last columns are in registers: the MMA warp may reuse the
+          // accumulator while they are converted and stored
+          asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar_acce + 8 * acc) : "memory");
+        }
         const long long col = (long long)tn * BN + c0;
         if (g.f32_out) {
           float4* dp = reinterpret_cast<float4*>(static_cast<float*>(g.d) + row * g.ldd + col);
@@ -302,10 +342,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // this warp is done reading the accumulator: the MMA warp may reuse it
-      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar_acce + 8 * acc) : "memory");
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -335,33 +371,49 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D map over packed codes [rows][ld bytes]: boxes of 128 bytes x 128 rows,
-// 128-byte swizzle.
-bool make_code_map(CUtensorMap* m, const void* codes, long long rows, long long kbytes, long long ld) {
+// 2D map over packed codes [rows][ld bytes]: boxes of 128 bytes x box_rows
+// rows, 128-byte swizzle.
+bool make_code_map(CUtensorMap* m, const void* codes, long long rows, long long kbytes, long long ld,
+                   cuuint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)ld};
-  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t box[2] = {128, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, void* d,
-                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st) {
+template <int BN>
+cudaError_t launch_bn(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, const GemmArgs& g,
+                      cudaStream_t st) {
   CUtensorMap ma, mb;
-  if (!make_code_map(&ma, a->codes, M, K / 2, a->codes_ld) || !make_code_map(&mb, b->codes, N, K / 2, b->codes_ld))
+  if (!make_code_map(&ma, a->codes, M, K / 2, a->codes_ld, BM) ||
+      !make_code_map(&mb, b->codes, N, K / 2, b->codes_ld, BN))
     return cudaErrorNotSupported;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(k_gemm_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    attr_err = cudaFuncSetAttribute(k_gemm_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg<BN>::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return cudaErrorNotSupported;
+  const int ntiles = (M / BM) * (N / BN);
+  k_gemm_nvfp4<BN><<<dim3(ntiles < sms ? ntiles : sms), kThreads, Cfg<BN>::kSmemBytes, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// 128 x 256 tiles when N allows them, else 128 x 128.
+cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, void* d,
+                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st) {
   GemmArgs g;
   g.sfa = a->scales;
   g.sfb = b->scales;
@@ -375,13 +427,7 @@ cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M,
   g.f32_out = f32_out;
   g.sf_col_tiles = K / 64;
   g.status = status;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
-      cudaSuccess)
-    return cudaErrorNotSupported;
-  const int ntiles = (M / BM) * (N / BN);
-  k_gemm_nvfp4<<<dim3(ntiles < sms ? ntiles : sms), kThreads, kSmemBytes, st>>>(ma, mb, g);
-  return cudaGetLastError();
+  return N % 256 == 0 ? launch_bn<256>(a, b, M, N, K, g, st) : launch_bn<128>(a, b, M, N, K, g, st);
 }
 
 }  // namespace fos
