@@ -490,7 +490,7 @@ def measure_modes(args, world, x, dev, stream, peak):
             res["gemm_nvfp4_%d" % n_] = {"ms": round(ms, 4), "TFLOP_s": round(tf, 1),
                                          "frac": round(tf / peak_tf, 4), "peak_TFLOP_s": peak_tf,
                                          "peak_source": peak_src, "shape": [n_, n_, n_],
-                                         "note": "bf16 out, 128x128 tiles, kind::mxf4nvf4"}
+                                         "note": "bf16 out, 128x256 tiles, kind::mxf4nvf4"}
             del xa, xb, qa, qb, d_
     except Exception as e:
         res["gemm_error"] = repr(e)

@@ -383,12 +383,16 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
         a.row.scales[scale_off<SWZ>(a.row, b, grA + 1, gtc)] = (uint8_t)s;
       }
       if (COL) {
-        // byte for rows (2i, 2i+1) of each of the tile's 16 columns
+        // byte for rows (2i, 2i+1) of each of the tile's 16 columns.  In a
+        // column's 32 bytes the 8-byte group of tile row tr sits at group
+        // tr ^ (tc & 3): the 4 tile columns a warp covers are 512 bytes
+        // apart, which would put their stores in the same banks
         const unsigned long long lo = zip_nibbles(ca[0], cb[0]), hi = zip_nibbles(ca[1], cb[1]);
+        const int gofs = 8 * (tr ^ (tc & 3)) + i;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          s_tc[(16 * tc + c) * 32 + 8 * tr + i] = (uint8_t)(lo >> (8 * c));
-          s_tc[(16 * tc + 8 + c) * 32 + 8 * tr + i] = (uint8_t)(hi >> (8 * c));
+          s_tc[(16 * tc + c) * 32 + gofs] = (uint8_t)(lo >> (8 * c));
+          s_tc[(16 * tc + 8 + c) * 32 + gofs] = (uint8_t)(hi >> (8 * c));
         }
         const long long gcA = (c0 + 16 * tc) + 2 * i;
         a.col.scales[scale_off<SWZ>(a.col, b, gcA, gtr)] = (uint8_t)s;
@@ -406,10 +410,12 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
       const int gc = c0 + col;
       const int grow = r0 + 32 * h;
       if (gc < a.cols && grow < a.rows) {
-        const uint4 v = *reinterpret_cast<const uint4*>(s_tc + col * 32 + 16 * h);
+        const int sw = (col >> 4) & 3;   // the group swizzle of this column's tile column
+        const uint2 v0 = *reinterpret_cast<const uint2*>(s_tc + col * 32 + 8 * ((2 * h) ^ sw));
+        const uint2 v1 = *reinterpret_cast<const uint2*>(s_tc + col * 32 + 8 * ((2 * h + 1) ^ sw));
         const long long byte_col = grow / 2;
-        store_codes8(a.col, b, gc, byte_col, v.x, v.y);
-        if (grow + 16 < a.rows) store_codes8(a.col, b, gc, byte_col + 8, v.z, v.w);
+        store_codes8(a.col, b, gc, byte_col, v0.x, v0.y);
+        if (grow + 16 < a.rows) store_codes8(a.col, b, gc, byte_col + 8, v1.x, v1.y);
       }
     }
     // rowwise copy: one bit per tile in the tile row-major order of x, so a
