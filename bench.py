@@ -502,9 +502,9 @@ def measure_modes(args, world, x, dev, stream, peak):
     try:
         peak_tf, peak_src = fp4_peak_tflops()
         M_, N_, K_ = 8192, 4096, 4096
-        xl = workloads.activation_outliers(M_, K_, device=dev)
-        wl = workloads.weight_normal(N_, K_, device=dev)
-        dyl = workloads.gradient_student_t(M_, N_, device=dev)
+        xl = workloads.activation_outliers(M_, K_, device=dev)[0]
+        wl = workloads.weight_normal(N_, K_, device=dev)[0]
+        dyl = workloads.gradient_student_t(M_, N_, device=dev)[0]
         qw = F.quantize_weight(wl)
 
         def layer_step():

@@ -784,6 +784,8 @@ __global__ void __launch_bounds__(kThreads) k_fake_mx(const QuantArgs a) {
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
+static constexpr int kMaxDevices = 64;
+
 static dim3 grid_for(uint32_t units, uint32_t per_cta, int batch) {
   return dim3((units + per_cta - 1) / per_cta, (unsigned)batch, 1);
 }
@@ -797,13 +799,50 @@ cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_
   return cudaGetLastError();
 }
 
+// Blocks per CTA for `nblk` blocks in each of `batch` entries on `slots`
+// resident CTAs: at most max_units, a multiple of 32 (whole choice words),
+// and spread so that the last wave of CTAs is about as full as the others
+// (e.g. a 2.1 M-block tensor on 592 slots: 1792 blocks per CTA, 1.98 waves,
+// instead of 2048 blocks and 1.73 waves).
+static uint32_t balanced_units(uint32_t nblk, int batch, uint32_t max_units, int slots) {
+  const unsigned long long total = (unsigned long long)nblk * (unsigned long long)batch;
+  const unsigned long long per_wave = (unsigned long long)slots * max_units;
+  const unsigned long long waves = (total + per_wave - 1) / per_wave;
+  unsigned long long u = (total + waves * slots - 1) / (waves * slots);
+  u = (u + 31) / 32 * 32;
+  return (uint32_t)(u < 32 ? 32 : (u > max_units ? max_units : u));
+}
+
+// One k_q1x16 variant, with the work per CTA balanced over the resident
+// slots (SMs x resident CTAs, looked up once per device and variant).
+template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE>
+static cudaError_t launch_k1(const QuantArgs& a, int batch, cudaStream_t st) {
+  static std::atomic<int> slots_of[kMaxDevices];
+  auto kern = k_q1x16<F46, SR, RHT, SWZ, DENSE, FAKE>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
+  int slots = slots_of[dev].load(std::memory_order_relaxed);
+  if (slots == 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess)
+      return cudaErrorNotSupported;
+    slots = sms * (per_sm > 0 ? per_sm : 1);
+    slots_of[dev].store(slots, std::memory_order_relaxed);
+  }
+  QuantArgs b = a;
+  b.units_per_cta = balanced_units(a.nblk, batch, a.units_per_cta, slots);
+  const dim3 g = grid_for(a.nblk, b.units_per_cta, batch);
+  kern<<<g, kThreads, 0, st>>>(b);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr, bool rht,
                                  bool swz, bool dense, cudaStream_t st, bool fake) {
-  const dim3 g = grid_for(a.nblk, a.units_per_cta, batch);
   const bool f46 = fmt == 0;
   if (dense || fake) swz = false;
   if (fake) {
-#define FOS_L(F, S, R, D) k_q1x16<F, S, R, false, D, true><<<g, kThreads, 0, st>>>(a)
+#define FOS_L(F, S, R, D) return launch_k1<F, S, R, false, D, true>(a, batch, st)
 #define FOS_D(F, S, R) do { if (dense) FOS_L(F, S, R, true); else FOS_L(F, S, R, false); } while (0)
 #define FOS_R(F, S) do { if (rht) FOS_D(F, S, true); else FOS_D(F, S, false); } while (0)
 #define FOS_S(F) do { if (sr) FOS_R(F, true); else FOS_R(F, false); } while (0)
@@ -813,9 +852,8 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 #undef FOS_R
 #undef FOS_D
 #undef FOS_L
-    return cudaGetLastError();
   }
-#define FOS_L(F, S, R, W, D) k_q1x16<F, S, R, W, D, false><<<g, kThreads, 0, st>>>(a)
+#define FOS_L(F, S, R, W, D) return launch_k1<F, S, R, W, D, false>(a, batch, st)
 #define FOS_D(F, S, R, W) do { if (dense) FOS_L(F, S, R, W, true); else FOS_L(F, S, R, W, false); } while (0)
 #define FOS_W(F, S, R) do { if (swz) FOS_D(F, S, R, true); else FOS_D(F, S, R, false); } while (0)
 #define FOS_R(F, S) do { if (rht) FOS_W(F, S, true); else FOS_W(F, S, false); } while (0)
@@ -827,13 +865,11 @@ cudaError_t launch_q1x16_rowwise(const QuantArgs& a, int batch, int fmt, bool sr
 #undef FOS_W
 #undef FOS_D
 #undef FOS_L
-  return cudaGetLastError();
 }
 
 // Persistent launch of the fused kernel: one CTA per resident slot.  The
 // grid (SMs x resident CTAs) is looked up once per device and kernel variant
 // and cached; 0 = not yet known, -1 = the kernel cannot be resident.
-static constexpr int kMaxDevices = 64;
 
 // The item sequence for nblk blocks per entry; false when the item count does
 // not fit the 31-bit positions of the queue.
