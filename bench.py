@@ -359,7 +359,22 @@ def run_fos(args, world, rank):
                      "quantize_only_ms": round(tq_ms, 4),
                      "quantize_only_GB_s": round(elems * BYTES_PER_ELEM / (tq_ms * 1e-3) / 1e9, 1),
                      "amax_pass_ms": round(ta_ms, 4),
-                     "peak_source": "%s hbm_gbs (copy, read+write)" % peak_kind},
+                     "peak_source": "%s hbm_gbs (copy, read+write)" % peak_kind,
+                     # the two ways of counting the step's bytes: (i) amax
+                     # supplied, 2.5625 B/element; (ii) amax in the step,
+                     # whose algorithm reads the input twice, 4.5625 B/element
+                     # (this launch reads it about once from DRAM: traffic)
+                     "mode_i_amax_supplied": {
+                         "ms": round(tq_ms, 4),
+                         "GB_s": round(elems * BYTES_PER_ELEM / (tq_ms * 1e-3) / 1e9, 1),
+                         "frac": round(elems * BYTES_PER_ELEM / (tq_ms * 1e-3) / 1e9 / peak, 4),
+                         "frac_of_8tbs_spec": round(elems * BYTES_PER_ELEM / (tq_ms * 1e-3) / 8e12, 4)},
+                     "mode_ii_amax_in_step": {
+                         "ms": round(ms_per_step, 4),
+                         "bytes_per_elem": BYTES_PER_ELEM + 2.0,
+                         "GB_s": round(elems * (BYTES_PER_ELEM + 2.0) / (ms_per_step * 1e-3) / 1e9, 1),
+                         "frac": round(elems * (BYTES_PER_ELEM + 2.0) / (ms_per_step * 1e-3) / 1e9 / peak, 4)},
+                     "frac_of_8tbs_spec": round(achieved / 8000.0, 4)},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": e2e,
         "clocks": clocks,
