@@ -38,6 +38,8 @@ class Opts(ctypes.Structure):
         ("rht", ctypes.c_int32),
         ("seed", ctypes.c_uint64),
         ("elem_offset", ctypes.c_int64),
+        ("rht_col", ctypes.c_int32),
+        ("pad", ctypes.c_int32),
     ]
 
 
@@ -88,7 +90,7 @@ def lib():
             L.or_amax.argtypes = [P, i64, i64, i64, i32, u64, P]
             L.or_quantize.restype = i32
             L.or_quantize.argtypes = [P, i64, i64, i64, ctypes.POINTER(Opts), P,
-                                      P, P, P, P, P, P, P]
+                                      P, P, P, P, P, P, P, P]
             L.or_dequantize.restype = i32
             L.or_dequantize.argtypes = [P, P, P, i64, i64, i64, i32, P]
             L.or_swizzle_offset.restype = i64
@@ -240,11 +242,13 @@ def amax(x_bits: np.ndarray, rht: bool = False, seed: int = 0) -> np.ndarray:
 def quantize(x_bits: np.ndarray, fmt: int = FMT_NVFP4_46, blk: int = BLK_1X16,
              rnd: int = RND_RNE, rht: bool = False, seed: int = 0,
              elem_offset: int = 0, rowwise: bool = True, colwise: bool = False,
-             amax_in: np.ndarray | None = None) -> dict:
+             amax_in: np.ndarray | None = None, rht_col: bool = False) -> dict:
     """Quantize bf16 bits [batch, rows, cols] -> dict of numpy outputs.
 
     Keys: r_codes [b,rows,cols/2], r_scales [b,rows,cols/bs], r_choice (bitmap),
-    c_codes [b,cols,rows/2], c_scales [b,cols,rows/16], c_choice, tensor_scale [b].
+    c_codes [b,cols,rows/2], c_scales [b,cols,rows/16], c_choice, tensor_scale [b],
+    c_tensor_scale [b] (the colwise copy's S_t; differs from tensor_scale only
+    with rht_col, the 16-wide transform of the colwise blocks along rows).
     """
     x = np.ascontiguousarray(x_bits, dtype=np.uint16)
     if x.ndim == 2:
@@ -263,7 +267,8 @@ def quantize(x_bits: np.ndarray, fmt: int = FMT_NVFP4_46, blk: int = BLK_1X16,
         nblk_c = b * c * r // 16 if blk != BLK_16X16 else b * (r // 16) * (c // 16)
         out["c_choice"] = np.zeros((nblk_c + 7) // 8, np.uint8)
     out["tensor_scale"] = np.zeros(b, np.float32)
-    o = Opts(fmt, blk, rnd, int(rht), seed, elem_offset)
+    out["c_tensor_scale"] = np.zeros(b, np.float32)
+    o = Opts(fmt, blk, rnd, int(rht), seed, elem_offset, int(rht_col), 0)
     ain = None
     if amax_in is not None:
         ain = np.ascontiguousarray(amax_in, dtype=np.float32)
@@ -271,7 +276,7 @@ def quantize(x_bits: np.ndarray, fmt: int = FMT_NVFP4_46, blk: int = BLK_1X16,
         _p(x), b, r, c, ctypes.byref(o), _p(ain),
         _p(out.get("r_codes")), _p(out.get("r_scales")), _p(out.get("r_choice")),
         _p(out.get("c_codes")), _p(out.get("c_scales")), _p(out.get("c_choice")),
-        _p(out["tensor_scale"]))
+        _p(out["tensor_scale"]), _p(out["c_tensor_scale"]))
     if st == NONFINITE:
         raise ValueError("oracle: non-finite input")
     if st == UNSUPPORTED:

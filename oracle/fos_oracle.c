@@ -71,6 +71,8 @@ typedef struct {
   int32_t rht;          /* 1 = 16-wide random Hadamard transform along cols */
   uint64_t seed;        /* Philox key for RHT signs and SR draws */
   int64_t elem_offset;  /* global linear index of element [0,0,0] (SR) */
+  int32_t rht_col;      /* 1 = the same transform along rows for the colwise copy */
+  int32_t pad;
 } or_opts;
 
 int or_version(void) { return OR_VERSION; }
@@ -418,6 +420,20 @@ static void set_bit(uint8_t* bits, int64_t b, int v) {
 /* Tensor-level entry points                                            */
 /* ------------------------------------------------------------------ */
 
+/* Amax of |RHT16| over the 16-row column blocks of one entry: the tensor
+ * amax the colwise copy takes when its blocks are transformed along rows. */
+static float amax_cols_rht(const uint16_t* xb, int64_t rows, int64_t cols, uint32_t mask) {
+  float a = 0.0f;
+  for (int64_t c = 0; c < cols; c++)
+    for (int64_t rb = 0; rb < rows / 16; rb++) {
+      float w[16];
+      for (int i = 0; i < 16; i++) w[i] = or_bf16_to_f32(xb[(rb * 16 + i) * cols + c]);
+      if (OR_MUTANT != 20) or_rht16(w, mask);
+      for (int i = 0; i < 16; i++) a = fmaxf(a, fabsf(w[i]));
+    }
+  return a;
+}
+
 /* Per-batch-entry amax of |x| (of the RHT output when rht != 0).
  * Returns OR_NONFINITE if any input is NaN or infinite (R18). */
 int or_amax(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
@@ -451,16 +467,22 @@ int or_amax(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
  *   c_choice bitmap over the colwise copy's blocks (1x16), or over the
  *            transposed copy's 16x16 tiles in its own tile row-major order
  *   tensor_scale [batch]  (NVFP4)
- * amax_in (nullable) gives the per-batch amax instead of computing it. */
+ *   c_tensor_scale [batch] (nullable) the colwise copy's S_t: the same as
+ *            tensor_scale, except with rht_col, where the colwise blocks are
+ *            transformed along rows and take the amax of the transformed
+ *            columns (R21)
+ * amax_in (nullable) gives the per-batch amax instead of computing it (with
+ * rht_col it sets the rowwise S_t only). */
 int or_quantize(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
                 const or_opts* o, const float* amax_in,
                 uint8_t* r_codes, uint8_t* r_scales, uint8_t* r_choice,
                 uint8_t* c_codes, uint8_t* c_scales, uint8_t* c_choice,
-                float* tensor_scale) {
+                float* tensor_scale, float* c_tensor_scale) {
   int mx = o->fmt == OR_FMT_MXFP4;
   if (mx != (o->blk == OR_BLK_1X32)) return OR_UNSUPPORTED;
   if (mx && (o->rnd != OR_RND_RNE || o->rht || c_codes)) return OR_UNSUPPORTED;
   if (o->rht && (o->blk != OR_BLK_1X16 || c_codes)) return OR_UNSUPPORTED;
+  if (o->rht_col && (mx || o->blk != OR_BLK_1X16 || !(c_codes || c_scales))) return OR_UNSUPPORTED;
   int64_t bs = mx ? 32 : 16;
   if (cols % bs) return OR_SHAPE;
   if ((c_codes || o->blk == OR_BLK_16X16) && rows % 16) return OR_SHAPE;
@@ -496,6 +518,8 @@ int or_quantize(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
     }
     float S_t = or_tensor_scale(A, o->fmt);
     if (tensor_scale) tensor_scale[b] = S_t;
+    float S_tc = o->rht_col ? or_tensor_scale(amax_cols_rht(xb, rows, cols, mask), o->fmt) : S_t;
+    if (c_tensor_scale) c_tensor_scale[b] = S_tc;
     int64_t base = o->elem_offset + b * n; /* global index of x[b,0,0] */
 
     if (o->blk == OR_BLK_1X16) {
@@ -518,7 +542,7 @@ int or_quantize(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
             for (int j = 0; j < 16; j++)
               put_nibble(r_codes, (b * rows + r) * cols + cb * 16 + j, codes[j]);
         }
-      if (c_codes || c_scales) /* R12: colwise = independent 1x16 along rows */
+      if (c_codes || c_scales) /* R12: colwise = independent 1x16 along rows; R21: RHT */
         for (int64_t c = 0; c < cols; c++)
           for (int64_t rb = 0; rb < rows / 16; rb++) {
             float w[16];
@@ -529,7 +553,8 @@ int or_quantize(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
               w[i] = or_bf16_to_f32(xb[(rb * 16 + i) * cols + c]);
               g[i] = base + (rb * 16 + i) * cols + c;
             }
-            uint8_t s = nvfp4_block(w, g, 16, S_t, o, codes, &p4);
+            if (o->rht_col) or_rht16(w, mask);
+            uint8_t s = nvfp4_block(w, g, 16, S_tc, o, codes, &p4);
             int64_t blk = (b * cols + c) * (rows / 16) + rb;
             if (c_scales) c_scales[blk] = s;
             set_bit(c_choice, blk, p4);

@@ -26,6 +26,7 @@ MUTANTS = {
     17: "bf16 rounding breaks ties upward instead of to even",
     18: "SR Philox counter is the element index instead of index / 16",
     19: "2D transposed copy's choice bit at the source tile's index",
+    20: "colwise transform: the colwise amax taken before the transform",
 }
 
 PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")

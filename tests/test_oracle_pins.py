@@ -672,6 +672,31 @@ def test_swizzle_is_a_permutation_with_128x4_tiles():
     del lin
 
 
+def test_colwise_rht_is_the_rowwise_rht_of_the_transpose():
+    """R21: with the transform along rows, the colwise copy of x is the
+    rowwise RHT quantization of x^T (without SR, whose draws follow x's
+    element index): codes, scales, choice bits and the colwise S_t, which
+    comes from the transformed columns.  Without the transform the colwise
+    S_t equals the rowwise one."""
+    rng = np.random.default_rng(21)
+    for fmt in (oracle.FMT_NVFP4_46, oracle.FMT_NVFP4_6):
+        for shape in ((1, 32, 48), (2, 48, 64), (1, 96, 16)):
+            x = rng.standard_normal(shape).astype(np.float32)
+            x *= np.exp2(rng.integers(-4, 4, (shape[0], 1, shape[2]))).astype(np.float32)
+            x[..., ::7, :] *= 25.0                       # outlier rows: the transform matters
+            xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+            q = oracle.quantize(xb, fmt=fmt, colwise=True, rht_col=True, seed=5)
+            t = oracle.quantize(np.ascontiguousarray(xb.transpose(0, 2, 1)), fmt=fmt, rht=True, seed=5)
+            assert np.array_equal(q["c_codes"], t["r_codes"])
+            assert np.array_equal(q["c_scales"], t["r_scales"])
+            assert np.array_equal(q["c_choice"], t["r_choice"])
+            assert np.array_equal(q["c_tensor_scale"].view(np.uint32), t["tensor_scale"].view(np.uint32))
+            # the rowwise copy of the same call is untouched by the colwise transform
+            p = oracle.quantize(xb, fmt=fmt, colwise=True, seed=5)
+            assert np.array_equal(q["r_codes"], p["r_codes"])
+            assert np.array_equal(p["c_tensor_scale"].view(np.uint32), p["tensor_scale"].view(np.uint32))
+
+
 def test_threaded_oracle_equals_one_call():
     """The host-core timing helper (row chunks on threads, amax supplied)
     gives the same bytes as one oracle call per entry."""
