@@ -73,6 +73,7 @@ typedef enum fos_round {
 /* fos_options.flags */
 #define FOS_FLAG_RHT16 0x1u          /* 16-wide random Hadamard transform (1x16, rowwise only) */
 #define FOS_FLAG_SCALE_SWIZZLED 0x2u /* scales in the 128x4 tensor-core tile layout */
+#define FOS_FLAG_RHT16_COL 0x4u      /* the same transform along rows for the colwise copy (1x16 NVFP4) */
 
 /* bits OR-ed into *status by the device */
 #define FOS_STATUS_NONFINITE 0x1u /* a NaN or Inf was read; outputs unspecified */
@@ -135,6 +136,15 @@ typedef struct fos_qtensor {
  *  colwise != NULL: blk 1X16 quantizes x^T independently with 16-blocks
  *    along rows (same S_t); blk 16X16 writes the exact transpose of the
  *    rowwise codes and scales.  rows % 16 == 0.
+ *  FOS_FLAG_RHT16_COL (NVFP4, blk 1X16, colwise != NULL): each 16-row
+ *    colwise block is transformed like a rowwise RHT block (the seeded signs
+ *    by position in the block, the 16-point Walsh-Hadamard butterfly, x0.25)
+ *    before it is quantized, and the colwise copy takes its own S_t from the
+ *    amax of the transformed columns (written to colwise->tensor_scale).
+ *    That amax is always computed in the call, so the workspace is needed
+ *    even with amax_in, which then sets the rowwise S_t only.  The rowwise
+ *    copy is not transformed (FOS_FLAG_RHT16 with a colwise copy is
+ *    FOS_ERR_UNSUPPORTED).
  *  FOS_ROUND_SR: the 4/6 choice is made on the RNE candidates, then the kept
  *    candidate is re-rounded stochastically: with v in [lo, hi) on the grid,
  *    round up iff 2*byte+1 < 512*(v-lo)/(hi-lo), byte j = g & 15 of

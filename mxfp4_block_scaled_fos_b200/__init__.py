@@ -5,7 +5,7 @@ ctypes binding that passes torch device buffers and the current stream to it;
 ``linear`` orders its calls into a quantized Linear layer's three GEMMs.
 """
 from .fos import (  # noqa: F401
-    FLAG_RHT16, FLAG_SCALE_SWIZZLED, STATUS_NONFINITE, STATUS_TIMEOUT, FosError, Options,
+    FLAG_RHT16, FLAG_RHT16_COL, FLAG_SCALE_SWIZZLED, STATUS_NONFINITE, STATUS_TIMEOUT, FosError, Options,
     QTensor, amax, dequantize, fake_quantize, gemm_nvfp4, lib, quantize, scales_size, status_string, version,
     workspace_size,
 )

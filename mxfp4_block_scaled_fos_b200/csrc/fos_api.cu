@@ -153,16 +153,18 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
   if (!opt || !x) return FOS_ERR_NULL;
   if (!rowwise && !colwise) return FOS_ERR_NULL;
   if (opt->fmt < 0 || opt->fmt > 2 || opt->blk < 0 || opt->blk > 2 || opt->rnd < 0 ||
-      opt->rnd > 1 || (opt->flags & ~(FOS_FLAG_RHT16 | FOS_FLAG_SCALE_SWIZZLED)))
+      opt->rnd > 1 || (opt->flags & ~(FOS_FLAG_RHT16 | FOS_FLAG_SCALE_SWIZZLED | FOS_FLAG_RHT16_COL)))
     return FOS_ERR_ARG;
   if (batch < 0 || rows < 0 || cols < 0) return FOS_ERR_SHAPE;
   const bool mx = opt->fmt == FOS_FMT_MXFP4;
   const bool rht = (opt->flags & FOS_FLAG_RHT16) != 0;
+  const bool rht_col = (opt->flags & FOS_FLAG_RHT16_COL) != 0;
   const bool swz = (opt->flags & FOS_FLAG_SCALE_SWIZZLED) != 0;
   const bool sr = opt->rnd == FOS_ROUND_SR;
   if (mx != (opt->blk == FOS_BLOCK_1X32)) return FOS_ERR_UNSUPPORTED;
   if (mx && (sr || rht || colwise)) return FOS_ERR_UNSUPPORTED;
   if (rht && (opt->blk != FOS_BLOCK_1X16 || colwise)) return FOS_ERR_UNSUPPORTED;
+  if (rht_col && (mx || opt->blk != FOS_BLOCK_1X16 || !colwise)) return FOS_ERR_UNSUPPORTED;
   const int64_t bs = mx ? 32 : 16;
   if (cols % bs) return FOS_ERR_SHAPE;
   if ((colwise || opt->blk == FOS_BLOCK_16X16) && rows % 16) return FOS_ERR_SHAPE;
@@ -176,7 +178,7 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
   fos_status e;
   if (rowwise && (e = check_out(rowwise, rows, cols, bs, !mx, opt->flags)) != FOS_OK) return e;
   if (colwise && (e = check_out(colwise, cols, rows, 16, !mx, opt->flags)) != FOS_OK) return e;
-  const bool need_ws = !mx && !amax_in;
+  const bool need_ws = !mx && (!amax_in || rht_col);
   if (need_ws) {
     if (!workspace) return FOS_ERR_WORKSPACE;
     if (workspace_bytes < ws_bytes(batch)) return FOS_ERR_WORKSPACE;
@@ -284,7 +286,12 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
   if (opt->blk == FOS_BLOCK_16X16) {
     ce = launch_q16x16(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr, st);
   } else if (colwise) {
-    ce = launch_q1x16_dual(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, st);
+    if (rht_col) {  // the colwise copy's own amax, in the words the fused path uses for its counts
+      if (cudaMemsetAsync(done_ws, 0, 4 * batch, st) != cudaSuccess) return FOS_ERR_CUDA;
+      if (launch_amax_cols_rht(a, (int)batch, done_ws, st) != cudaSuccess) return FOS_ERR_CUDA;
+      a.amax_col_ws = done_ws;
+    }
+    ce = launch_q1x16_dual(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, st, rht_col);
   } else {
     ce = launch_q1x16_rowwise(a, (int)batch, opt->fmt, sr, rht, swz, dense, st);
   }

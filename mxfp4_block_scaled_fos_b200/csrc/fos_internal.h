@@ -34,6 +34,7 @@ struct QuantArgs {
   uint32_t units_per_cta = 0;
   const float* amax_in = nullptr;   // nullable
   const uint32_t* amax_ws = nullptr;
+  const uint32_t* amax_col_ws = nullptr;  // the colwise copy's amax words (colwise transform)
   uint32_t* status = nullptr;       // nullable
   unsigned long long seed = 0;
   long long elem_offset = 0;
@@ -85,7 +86,10 @@ constexpr size_t workspace_bytes_for(long long batch) {
 }
 
 cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
-                              bool want_row, cudaStream_t st);
+                              bool want_row, cudaStream_t st, bool rht_col = false);
+// amax of the 16-row column blocks after the 16-wide transform (the colwise
+// copy's amax with FOS_FLAG_RHT16_COL) into zeroed words amax_col[batch]
+cudaError_t launch_amax_cols_rht(const QuantArgs& a, int batch, uint32_t* amax_col, cudaStream_t st);
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
                           bool want_row, bool want_col, cudaStream_t st);
 cudaError_t launch_mxfp4(const QuantArgs& a, int batch, bool swz, cudaStream_t st);

@@ -50,7 +50,7 @@ fos_status fos_quantize_static(const void* x, int64_t batch, int64_t rows, int64
                                uint32_t* status, void* stream) {
   // only calls that compute the amax use scratch (MXFP4 and calls with
   // amax_in need none): the batch limit applies to those alone
-  const bool needs_scratch = opt && opt->fmt != FOS_FMT_MXFP4 && !amax_in;
+  const bool needs_scratch = opt && opt->fmt != FOS_FMT_MXFP4 && (!amax_in || (opt->flags & FOS_FLAG_RHT16_COL));
   if (needs_scratch && batch > kStaticMaxBatch) return FOS_ERR_WORKSPACE;
   void* scratch = nullptr;
   const fos_status e = scratch_address(&scratch);

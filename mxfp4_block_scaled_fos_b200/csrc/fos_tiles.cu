@@ -177,20 +177,66 @@ __device__ __forceinline__ uint32_t dual_row_block(const QuantArgs& a, int b, co
   return pick && valid;
 }
 
-template <bool F46, bool SR, bool SWZ, bool ROW>
-__global__ void __launch_bounds__(kThreads, SR ? FOS_DUALW_MIN_BLOCKS_SR : FOS_DUALW_MIN_BLOCKS) k_dual_warp(const QuantArgs a, FastDiv ntc4) {
+// Amax of the 16-row column blocks after the 16-wide transform (the colwise
+// copy's tensor amax with FOS_FLAG_RHT16_COL).  One thread per (16-row
+// strip, column pair): 16 32-bit loads (a warp reads 128 contiguous bytes
+// per row), the seeded signs by row, the butterfly on the packed column pair,
+// then a warp max and one atomicMax per warp into amax_col[b] (zeroed).
+__global__ void __launch_bounds__(kThreads) k_amax_cols_rht(const QuantArgs a, uint32_t* amax_col) {
+  const int b = blockIdx.y;
+  const uint32_t mask16 = rht_sign_mask(a.seed);
+  const uint32_t npair = (uint32_t)a.cols / 2, nunits = npair * ((uint32_t)a.rows / 16);
+  const uint16_t* xb = a.x + (long long)b * a.x_bs;
+  uint32_t m = 0;
+  for (uint32_t u = blockIdx.x * kThreads + threadIdx.x; u < nunits; u += gridDim.x * kThreads) {
+    const uint32_t strip = u / npair, cp = u - strip * npair;
+    const uint16_t* p = xb + (long long)strip * 16 * a.ld + 2 * cp;
+    float2 T[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p + (long long)r * a.ld)) ^
+                         (((mask16 >> r) & 1u) ? 0x80008000u : 0u);
+      T[r] = make_float2(bf_lo(w), bf_hi(w));
+    }
+    fwht16_pairs(T);
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      m = max(m, max(__float_as_uint(T[r].x) & 0x7fffffffu, __float_as_uint(T[r].y) & 0x7fffffffu));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0) {
+    if (m >= 0x7f800000u) {
+      if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+    } else if (m) {
+      atomicMax(amax_col + b, m);
+    }
+  }
+}
+
+// RHTC: the colwise blocks are transformed along rows (the 16-wide RHT with
+// the seeded signs by row position) and take their own S_t, from the amax
+// words amax_col_ws of the transformed columns.
+template <bool F46, bool SR, bool SWZ, bool ROW, bool RHTC>
+__global__ void __launch_bounds__(kThreads, RHTC ? 2 : (SR ? FOS_DUALW_MIN_BLOCKS_SR : FOS_DUALW_MIN_BLOCKS))
+    k_dual_warp(const QuantArgs a, FastDiv ntc4) {
   __shared__ __align__(16) float4 s_tab[128];
+  __shared__ __align__(16) float4 s_tabc[RHTC ? 128 : 1];   // the colwise copy's table (RHTC)
   __shared__ __align__(16) uint8_t s_x[kThreads / 32][4 * kDwGroup];
   __shared__ __align__(16) uint8_t s_r[SR ? kThreads / 32 : 1][SR ? 4 * 256 : 16];
   const int b = blockIdx.y;
   const float St = tensor_scale_of(a, b, F46);
+  const float StC = RHTC ? __fdiv_rn(__uint_as_float(a.amax_col_ws[b]), F46 ? 1792.0f : 2688.0f) : St;
   build_scale_table4(s_tab, St);
+  if (RHTC) build_scale_table4(s_tabc, StC);
+  const float4* tab_c = RHTC ? s_tabc : s_tab;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (ROW && a.row.tensor_scale) a.row.tensor_scale[b] = St;
-    if (a.col.tensor_scale) a.col.tensor_scale[b] = St;
+    if (a.col.tensor_scale) a.col.tensor_scale[b] = StC;
   }
   __syncthreads();
   const TScale ts = make_tscale(St);
+  const TScale tsc = RHTC ? make_tscale(StC) : ts;
+  const uint32_t mask16 = RHTC ? rht_sign_mask(a.seed) : 0u;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 3, i = lane & 7;
   const uint32_t ntr = a.rows / 16, ntc = a.cols / 16;
@@ -238,23 +284,43 @@ __global__ void __launch_bounds__(kThreads, SR ? FOS_DUALW_MIN_BLOCKS_SR : FOS_D
       uint32_t w[16];  // row r of the tile's columns 2i (low half) and 2i+1 (high half)
 #pragma unroll
       for (int r = 0; r < 16; ++r) w[r] = *reinterpret_cast<const uint32_t*>(xb + r * 32 + 4 * i);
-      uint32_t h[8];
+      uint32_t mc[2];
+      float2 T[16];   // RHTC: row r of both columns after the transform
+      if (RHTC) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) h[k] = hmax_abs2(w[2 * k], w[2 * k + 1]);
-      const uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(h[0], h[1]), hmax_abs2(h[2], h[3])),
-                                   hmax_abs2(hmax_abs2(h[4], h[5]), hmax_abs2(h[6], h[7]))) & 0x7fff7fffu;
-      const uint32_t mc[2] = {(m & 0xffffu) << 16, m & 0xffff0000u};
+        for (int r = 0; r < 16; ++r) {
+          const uint32_t wr = w[r] ^ (((mask16 >> r) & 1u) ? 0x80008000u : 0u);
+          T[r] = make_float2(bf_lo(wr), bf_hi(wr));
+        }
+        fwht16_pairs(T);
+        mc[0] = mc[1] = 0;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          mc[0] = max(mc[0], __float_as_uint(T[r].x) & 0x7fffffffu);
+          mc[1] = max(mc[1], __float_as_uint(T[r].y) & 0x7fffffffu);
+        }
+      } else {
+        uint32_t h[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) h[k] = hmax_abs2(w[2 * k], w[2 * k + 1]);
+        const uint32_t m = hmax_abs2(hmax_abs2(hmax_abs2(h[0], h[1]), hmax_abs2(h[2], h[3])),
+                                     hmax_abs2(hmax_abs2(h[4], h[5]), hmax_abs2(h[6], h[7]))) & 0x7fff7fffu;
+        mc[0] = (m & 0xffffu) << 16;
+        mc[1] = m & 0xffff0000u;
+      }
       badmax = max(badmax, max(mc[0], mc[1]));
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {
         float2 P[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          P[k] = hc ? make_float2(bf_hi(w[k]), bf_hi(w[k + 8])) : make_float2(bf_lo(w[k]), bf_lo(w[k + 8]));
+        for (int k = 0; k < 8; ++k) {
+          if (RHTC) P[k] = hc ? make_float2(T[k].y, T[k + 8].y) : make_float2(T[k].x, T[k + 8].x);
+          else      P[k] = hc ? make_float2(bf_hi(w[k]), bf_hi(w[k + 8])) : make_float2(bf_lo(w[k]), bf_lo(w[k + 8]));
+        }
         uint32_t codes[2], sc;
         bool pick;
         float inv;
-        block_step<F46>(P, mc[hc], s_tab, ts, a.neg_zero, codes, sc, pick, inv);
+        block_step<F46>(P, mc[hc], tab_c, tsc, a.neg_zero, codes, sc, pick, inv);
         if (SR) sr_block1_smem(P, inv, rbuf + 2 * i + hc, 16, codes);
         const long long c = (long long)tc * 16 + 2 * i + hc;
         if (valid) {
@@ -466,13 +532,14 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
 }  // namespace
 
 cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
-                              bool want_row, cudaStream_t st) {
+                              bool want_row, cudaStream_t st, bool rht_col) {
   const bool f46 = fmt == 0;
   const uint32_t ntc4 = (uint32_t)((a.cols / 16 + 3) / 4);
   const uint32_t units = (uint32_t)(a.rows / 16) * ntc4;
   const FastDiv fd = make_fastdiv(ntc4);
   const dim3 g(min((units + kThreads / 32 - 1) / (kThreads / 32), 148u * 8u), (unsigned)batch);
-#define FOS_L(F, S, W, R) k_dual_warp<F, S, W, R><<<g, kThreads, 0, st>>>(a, fd)
+#define FOS_L(F, S, W, R) do { if (rht_col) k_dual_warp<F, S, W, R, true><<<g, kThreads, 0, st>>>(a, fd); \
+                              else k_dual_warp<F, S, W, R, false><<<g, kThreads, 0, st>>>(a, fd); } while (0)
 #define FOS_R(F, S, W) do { if (want_row) FOS_L(F, S, W, true); else FOS_L(F, S, W, false); } while (0)
 #define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)
 #define FOS_S(F) do { if (sr) FOS_W(F, true); else FOS_W(F, false); } while (0)
@@ -482,6 +549,13 @@ cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, b
 #undef FOS_W
 #undef FOS_R
 #undef FOS_L
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax_cols_rht(const QuantArgs& a, int batch, uint32_t* amax_col, cudaStream_t st) {
+  const uint32_t units = (uint32_t)(a.cols / 2) * (uint32_t)(a.rows / 16);
+  const uint32_t blocks = min((units + kThreads - 1) / kThreads, 148u * 8u);
+  k_amax_cols_rht<<<dim3(blocks, (unsigned)batch), kThreads, 0, st>>>(a, amax_col);
   return cudaGetLastError();
 }
 

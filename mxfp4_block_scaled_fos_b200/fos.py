@@ -25,6 +25,7 @@ BLK = {"1x16": 0, "16x16": 1, "1x32": 2}
 RND = {"rne": 0, "sr": 1}
 FLAG_RHT16 = 0x1
 FLAG_SCALE_SWIZZLED = 0x2
+FLAG_RHT16_COL = 0x4
 STATUS_NONFINITE = 0x1
 STATUS_TIMEOUT = 0x2
 
@@ -170,7 +171,7 @@ def _as3d(x: torch.Tensor) -> torch.Tensor:
 def quantize(x: torch.Tensor, fmt: str = "nvfp4_46", block: Optional[str] = None,
              rounding: str = "rne", rht: bool = False, swizzle: bool = False, seed: int = 0,
              elem_offset: int = 0, rowwise: bool = True, colwise: bool = False,
-             choice: bool = True, amax: Optional[torch.Tensor] = None,
+             choice: bool = True, amax: Optional[torch.Tensor] = None, rht_col: bool = False,
              status: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
              out_row: Optional[QTensor] = None, out_col: Optional[QTensor] = None,
              stream=None):
@@ -186,7 +187,8 @@ def quantize(x: torch.Tensor, fmt: str = "nvfp4_46", block: Optional[str] = None
     batch, rows, cols = x.shape
     ld = x.stride(1)
     block = block or ("1x32" if fmt == "mxfp4" else "1x16")
-    flags = (FLAG_RHT16 if rht else 0) | (FLAG_SCALE_SWIZZLED if swizzle else 0)
+    flags = (FLAG_RHT16 if rht else 0) | (FLAG_SCALE_SWIZZLED if swizzle else 0) | \
+        (FLAG_RHT16_COL if rht_col else 0)
     opts = Options(FMT[fmt], BLK[block], RND[rounding], flags, seed, elem_offset)
     bs = 32 if fmt == "mxfp4" else 16
     if block == "16x16":
@@ -203,7 +205,7 @@ def quantize(x: torch.Tensor, fmt: str = "nvfp4_46", block: Optional[str] = None
     if not colwise:
         out_col = None
     wsz = workspace_size(batch, rows, cols, opts)
-    if workspace is None and amax is None and fmt != "mxfp4":
+    if workspace is None and (amax is None or rht_col) and fmt != "mxfp4":
         workspace = torch.empty(wsz, dtype=torch.uint8, device=x.device)
     r = out_row.c_struct() if out_row is not None else None
     c = out_col.c_struct() if out_col is not None else None

@@ -62,13 +62,14 @@ def zeroed_out(batch, R, C, fmt, block, flags, device, nblocks, choice=True):
 
 def check_quantize(x: torch.Tensor, fmt="nvfp4_46", block=None, rounding="rne", rht=False,
                    swizzle=False, seed=0, elem_offset=0, rowwise=True, colwise=False,
-                   amax=None, x_bits=None):
+                   amax=None, x_bits=None, rht_col=False):
     """Quantize x on the GPU and with the oracle; assert bit equality of
     codes, scales, tensor scales and choice bits.  Returns the GPU outputs."""
     block = block or ("1x32" if fmt == "mxfp4" else "1x16")
     x3 = x if x.dim() == 3 else x.unsqueeze(0)
     batch, R, C = x3.shape
-    flags = (F.FLAG_RHT16 if rht else 0) | (F.FLAG_SCALE_SWIZZLED if swizzle else 0)
+    flags = (F.FLAG_RHT16 if rht else 0) | (F.FLAG_SCALE_SWIZZLED if swizzle else 0) | \
+        (F.FLAG_RHT16_COL if rht_col else 0)
     orow = zeroed_out(batch, R, C, fmt, block, flags, x.device, n_blocks(batch, R, C, block)) \
         if rowwise else None
     ocol = zeroed_out(batch, C, R, fmt, block, flags, x.device,
@@ -77,14 +78,14 @@ def check_quantize(x: torch.Tensor, fmt="nvfp4_46", block=None, rounding="rne", 
     status = torch.zeros(1, dtype=torch.int32, device=x.device)
     F.quantize(x3, fmt=fmt, block=block, rounding=rounding, rht=rht, swizzle=swizzle, seed=seed,
                elem_offset=elem_offset, rowwise=rowwise, colwise=colwise, amax=amax,
-               status=status, out_row=orow, out_col=ocol)
+               status=status, out_row=orow, out_col=ocol, rht_col=rht_col)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     xb = x_bits if x_bits is not None else np_bits(x3.contiguous() if x3.stride(1) != C else x3)
     ain = amax.cpu().numpy() if amax is not None else None
     ref = oracle.quantize(xb, fmt=FMT_O[fmt], blk=BLK_O[block], rnd=RND_O[rounding], rht=rht,
                           seed=seed, elem_offset=elem_offset, rowwise=rowwise, colwise=colwise,
-                          amax_in=ain)
+                          amax_in=ain, rht_col=rht_col)
     for tag, q in (("r", orow), ("c", ocol)):
         if q is None:
             continue
@@ -95,7 +96,8 @@ def check_quantize(x: torch.Tensor, fmt="nvfp4_46", block=None, rounding="rne", 
         assert_bytes_equal(q.scales.cpu().numpy(), sc, tag + "_scales")
         if fmt != "mxfp4":
             assert_bytes_equal(q.tensor_scale.cpu().numpy().view(np.uint32),
-                               ref["tensor_scale"].view(np.uint32), tag + "_tensor_scale")
+                               ref["tensor_scale" if tag == "r" else "c_tensor_scale"].view(np.uint32),
+                               tag + "_tensor_scale")
         if q.choice is not None:
             nb = n_blocks(batch, q.rows, q.cols, block) if block != "16x16" else n_blocks(batch, R, C, block)
             compare_choice(q.choice, ref[tag + "_choice"], nb, tag)

@@ -53,6 +53,35 @@ def test_dual_sr_element_offset():
     check_quantize(x, rounding="sr", seed=17, elem_offset=16 * 12345, colwise=True)
 
 
+@pytest.mark.parametrize("shape", [(1, 16, 16), (2, 80, 272), (1, 528, 400), (3, 1040, 128)])
+@pytest.mark.parametrize("rounding", ["rne", "sr"])
+@pytest.mark.parametrize("fmt", ["nvfp4_46", "nvfp4_6"])
+def test_dual_with_colwise_transform(shape, rounding, fmt):
+    """FOS_FLAG_RHT16_COL: the colwise blocks transformed along rows, with
+    their own S_t (R21); the rowwise copy of the same call untransformed.
+    Outlier rows make the transform change the codes."""
+    dev = require_gpu()
+    x = _rand(shape, shape[1] * 3 + shape[2] + 1, dev, "scaled")
+    x[..., ::9, :] *= 16
+    check_quantize(x, fmt=fmt, rounding=rounding, seed=21, rowwise=True, colwise=True, rht_col=True)
+
+
+def test_colwise_transform_options():
+    dev = require_gpu()
+    x = _rand((2, 96, 160), 12, dev, "scaled")
+    # colwise only, swizzled scales, SR with an element offset
+    check_quantize(x, rowwise=False, colwise=True, rht_col=True, swizzle=True, rounding="sr", seed=4,
+                   elem_offset=16 * 777)
+    # the rowwise amax supplied: the colwise amax is still computed in the call
+    am = F.amax(x)
+    check_quantize(x, rowwise=True, colwise=True, rht_col=True, amax=am)
+    # refused combinations
+    for kw in (dict(rht_col=True), dict(rht_col=True, block="16x16", colwise=True),
+               dict(rht_col=True, rht=True, colwise=True)):
+        with pytest.raises(F.FosError):
+            F.quantize(x, **kw)
+
+
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("rounding", ["rne", "sr"])
 @pytest.mark.parametrize("fmt", ["nvfp4_46", "nvfp4_6"])
