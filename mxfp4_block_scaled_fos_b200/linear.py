@@ -23,9 +23,12 @@ gradients; every tensor quantized with its own per-tensor scale):
                           B = x^T, 1x16 blocks along M
 
 The 2D weight blocks make W and W^T quantize to the same values, so the
-forward and dgrad GEMMs see one weight.  The random Hadamard transform along
-M for the wgrad operands is not offered (the library's transform runs along
-rows only).  Shapes: M and N multiples of 256, K a multiple of 256 (the
+forward and dgrad GEMMs see one weight.  With rht=True the two wgrad
+operands are quantized with the 16-wide random Hadamard transform along M
+(FOS_FLAG_RHT16_COL, the same seeded signs for both): the transform is
+orthogonal and applied to both sides of the reduction, so dW is unchanged
+in exact arithmetic while the outliers of dy and x are spread before
+quantization.  Shapes: M and N multiples of 256, K a multiple of 256 (the
 GEMM's 128-row tiles and 256-wide K steps, in each of the three products).
 """
 from __future__ import annotations
@@ -77,17 +80,20 @@ def linear_forward(x: torch.Tensor, qw: QuantizedWeight, fmt: str = "nvfp4_46",
 
 def linear_backward(dy: torch.Tensor, x: torch.Tensor, qw: QuantizedWeight, seed: int = 0,
                     elem_offset: int = 0, fmt: str = "nvfp4_46", out_dtype=torch.float32,
-                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                    rht: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """(dx [M, K], dW [N, K]) from dy [M, N], the forward input x [M, K] and
     the quantized weight.  dy is quantized once, in both orientations, with
-    stochastic rounding keyed on (seed, elem_offset + element index)."""
+    stochastic rounding keyed on (seed, elem_offset + element index).  rht:
+    the wgrad operands (dy^T, x^T) are transformed along M with the signs of
+    the same key (seed), each with its own S_t."""
     N, K = qw.shape
     if dy.dim() != 2 or x.dim() != 2 or dy.shape[1] != N or x.shape[1] != K or dy.shape[0] != x.shape[0]:
         raise ValueError("dy must be [M, N] and x [M, K] for a weight [N, K]")
     _check("M", dy.shape[0], 256)
     qdy, qdy_t = fos.quantize(dy, fmt=fmt, rounding="sr", seed=seed, elem_offset=elem_offset, swizzle=True,
-                              colwise=True, choice=False, stream=stream)
-    qx_t = fos.quantize(x, fmt=fmt, swizzle=True, rowwise=False, colwise=True, choice=False, stream=stream)[1]
+                              colwise=True, choice=False, rht_col=rht, stream=stream)
+    qx_t = fos.quantize(x, fmt=fmt, swizzle=True, rowwise=False, colwise=True, choice=False, rht_col=rht,
+                        seed=seed, stream=stream)[1]
     dx = fos.gemm_nvfp4(qdy, qw.col, out_dtype=out_dtype, stream=stream)
     dw = fos.gemm_nvfp4(qdy_t, qx_t, out_dtype=out_dtype, stream=stream)
     return dx, dw

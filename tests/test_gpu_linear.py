@@ -57,23 +57,26 @@ def _inputs(M, N, K, dev, seed):
     return (x.to(torch.bfloat16).to(dev), w.to(torch.bfloat16).to(dev), dy.to(torch.bfloat16).to(dev))
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (512, 256, 768), (256, 768, 512)])
-def test_linear_forward_and_backward_match_oracle_operands(M, N, K):
+@pytest.mark.parametrize("M,N,K,rht", [(256, 256, 256, False), (512, 256, 768, False), (256, 768, 512, False),
+                                       (512, 256, 256, True), (256, 512, 768, True)])
+def test_linear_forward_and_backward_match_oracle_operands(M, N, K, rht):
     dev = require_gpu()
     torch.manual_seed(M + N + K)
     x, w, dy = _inputs(M, N, K, dev, M * 7 + N * 3 + K)
     seed = 1234 + M
     qw = F.quantize_weight(w)
     y = F.linear_forward(x, qw, out_dtype=torch.float32)
-    dx, dw = F.linear_backward(dy, x, qw, seed=seed)
+    dx, dw = F.linear_backward(dy, x, qw, seed=seed, rht=rht)
     torch.cuda.synchronize()
 
     xb, wb, gb = np_bits(x)[None], np_bits(w)[None], np_bits(dy)[None]
     ox = oracle.quantize(xb)
     ow = oracle.quantize(wb, blk=oracle.BLK_16X16, colwise=True)
-    og = oracle.quantize(gb, rnd=oracle.RND_SR, seed=seed, colwise=True)
-    oxt = oracle.quantize(xb, rowwise=False, colwise=True)
+    og = oracle.quantize(gb, rnd=oracle.RND_SR, seed=seed, colwise=True, rht_col=rht)
+    oxt = oracle.quantize(xb, rowwise=False, colwise=True, rht_col=rht, seed=seed)
     st_x, st_w, st_g = (float(o["tensor_scale"][0]) for o in (ox, ow, og))
+    # the wgrad operands' own S_t (transformed columns with rht)
+    st_gt, st_xt = float(og["c_tensor_scale"][0]), float(oxt["c_tensor_scale"][0])
     assert qw.row.tensor_scale.item() == st_w and qw.col.tensor_scale.item() == st_w
 
     x_v = _values(ox["r_codes"][0], ox["r_scales"][0])            # [M, K]
@@ -87,7 +90,7 @@ def test_linear_forward_and_backward_match_oracle_operands(M, N, K):
 
     _check(y, *_ref(x_v, st_x, w_v, st_w), "forward y")
     _check(dx, *_ref(g_v, st_g, wt_v, st_w), "dgrad dx")
-    _check(dw, *_ref(gt_v, st_g, xt_v, st_x), "wgrad dW")
+    _check(dw, *_ref(gt_v, st_gt, xt_v, st_xt), "wgrad dW")
 
 
 def test_linear_shape_errors():
