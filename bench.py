@@ -486,6 +486,13 @@ def measure_modes(args, world, x, dev, stream, peak):
         r1 = F.quantize(g, rounding="sr")[0]
         ms = time_loop(lambda: F.quantize(g, rounding="sr", amax=am, out_row=r1), n, 3, world, stream) / n
         rec("gradient_sr_rowwise_kernel", ms, BYTES_PER_ELEM, g.numel(), "amax supplied")
+        rt, ct = F.quantize(g, rounding="sr", colwise=True, rht_col=True)
+        wst = torch.empty(F.workspace_size(1, g.shape[-2], g.shape[-1]), dtype=torch.uint8, device=dev)
+        ms = time_loop(lambda: F.quantize(g, rounding="sr", colwise=True, rht_col=True, amax=am, out_row=rt,
+                                          out_col=ct, workspace=wst), n, 3, world, stream) / n
+        rec("gradient_sr_dual_colwise_rht_step", ms, BYTES_PER_ELEM_DUAL, g.numel(),
+            "rowwise amax supplied; the colwise copy transformed along M with its own amax in the step")
+        del rt, ct, wst
         del g, r, c, r1
     except Exception as e:
         res["gradient_error"] = repr(e)
