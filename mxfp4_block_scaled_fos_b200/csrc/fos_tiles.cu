@@ -453,13 +453,20 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
         // column's 32 bytes the 8-byte group of tile row tr sits at group
         // tr ^ (tc & 3): the 4 tile columns a warp covers are 512 bytes
         // apart, which would put their stores in the same banks
-        const unsigned long long lo = zip_nibbles(ca[0], cb[0]), hi = zip_nibbles(ca[1], cb[1]);
+        // even (E) and odd (O) columns: byte k of word w is column 8 w + 2 k (+ 1),
+        // (row 2i nibble) | (row 2i+1 nibble) << 4
+        const uint32_t E[2] = {(ca[0] & 0x0f0f0f0fu) | ((cb[0] & 0x0f0f0f0fu) << 4),
+                               (ca[1] & 0x0f0f0f0fu) | ((cb[1] & 0x0f0f0f0fu) << 4)};
+        const uint32_t O[2] = {((ca[0] >> 4) & 0x0f0f0f0fu) | (cb[0] & 0xf0f0f0f0u),
+                               ((ca[1] >> 4) & 0x0f0f0f0fu) | (cb[1] & 0xf0f0f0f0u)};
         const int gofs = 8 * (tr ^ (tc & 3)) + i;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          s_tc[(16 * tc + c) * 32 + gofs] = (uint8_t)(lo >> (8 * c));
-          s_tc[(16 * tc + 8 + c) * 32 + gofs] = (uint8_t)(hi >> (8 * c));
-        }
+        for (int w = 0; w < 2; ++w)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            s_tc[(16 * tc + 8 * w + 2 * k) * 32 + gofs] = (uint8_t)(E[w] >> (8 * k));
+            s_tc[(16 * tc + 8 * w + 2 * k + 1) * 32 + gofs] = (uint8_t)(O[w] >> (8 * k));
+          }
         const long long gcA = (c0 + 16 * tc) + 2 * i;
         a.col.scales[scale_off<SWZ>(a.col, b, gcA, gtr)] = (uint8_t)s;
         a.col.scales[scale_off<SWZ>(a.col, b, gcA + 1, gtr)] = (uint8_t)s;
