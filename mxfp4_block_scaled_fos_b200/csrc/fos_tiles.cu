@@ -133,6 +133,9 @@ __device__ __forceinline__ unsigned long long zip_nibbles(uint32_t a, uint32_t b
 constexpr int kDwGroup = 16 * 32 + 32;   // bytes per tile in the buffer: 16 rows of
                                          // 32 bytes, padded so the 4 tiles' column
                                          // reads fall into distinct banks
+constexpr int kDwRGroup = 16 * 16 + 16;  // Philox bytes per tile: 16 rows of 16,
+                                         // padded so that the 4 tiles' colwise byte
+                                         // reads fall into distinct banks
 #ifndef FOS_DUALW_MIN_BLOCKS
 #define FOS_DUALW_MIN_BLOCKS 3
 #endif
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, RHTC ? 2 : (SR ? FOS_DUALW_MIN_BLOCK
   __shared__ __align__(16) float4 s_tab[128];
   __shared__ __align__(16) float4 s_tabc[RHTC ? 128 : 1];   // the colwise copy's table (RHTC)
   __shared__ __align__(16) uint8_t s_x[kThreads / 32][4 * kDwGroup];
-  __shared__ __align__(16) uint8_t s_r[SR ? kThreads / 32 : 1][SR ? 4 * 256 : 16];
+  __shared__ __align__(16) uint8_t s_r[SR ? kThreads / 32 : 1][SR ? 4 * kDwRGroup : 16];
   const int b = blockIdx.y;
   const float St = tensor_scale_of(a, b, F46);
   const float StC = RHTC ? __fdiv_rn(__uint_as_float(a.amax_col_ws[b]), F46 ? 1792.0f : 2688.0f) : St;
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, RHTC ? 2 : (SR ? FOS_DUALW_MIN_BLOCK
   const uint32_t nunits = ntr * ntc4.d;
   const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
   uint8_t* xb = s_x[warp] + g * kDwGroup;
-  uint8_t* rbuf = SR ? s_r[warp] + g * 256 : nullptr;
+  uint8_t* rbuf = SR ? s_r[warp] + g * kDwRGroup : nullptr;
   uint32_t badmax = 0;
   for (uint32_t u = blockIdx.x * (kThreads / 32) + warp; u < nunits; u += gridDim.x * (kThreads / 32)) {
     const uint32_t trow = fdiv(u, ntc4), tq = u - trow * ntc4.d;
