@@ -9,11 +9,9 @@
 // adjacent 16x16 tiles, loaded straight from global memory, and transposes
 // them through its own shared buffer; no CTA barrier in the loop.
 // 16x16 (k_2d16x16): a CTA of 256 threads walks a strip of up to 8 sub-tiles
-// of 64 rows x 128 columns (16 KB of bf16) down the tensor.  Each sub-tile is
-// staged in shared memory with 16-byte chunks XOR-swizzled by row so that the
-// row-major reads, the column reads and the 16x16 reads are all free of bank
-// conflicts; the next sub-tile's global loads are issued before the current
-// one is processed.
+// of 64 rows x 128 columns (16 KB of bf16) down the tensor.  Each thread
+// loads the two tile rows it quantizes straight from global memory, one
+// sub-tile ahead; the transposed codes go through shared memory.
 // Stochastic-rounding bytes are drawn once per 16 source elements (one Philox
 // call per rowwise block) and shared by both orientations through shared
 // memory.
@@ -30,38 +28,6 @@ constexpr int kStrip = 8;  // sub-tiles per CTA strip (512 rows)
 #ifndef FOS_2D_MIN_BLOCKS
 #define FOS_2D_MIN_BLOCKS 3
 #endif
-
-// smem byte offset of the 16-byte chunk c16 of row r under swizzle f(r).
-template <int SHIFT>
-__device__ __forceinline__ uint32_t chunk_off(int r, int c16) {
-  return (uint32_t)(r * 256 + ((c16 ^ ((r >> SHIFT) & 7)) << 4));
-}
-
-// Global -> registers: 4 16-byte chunks per thread of the sub-tile whose
-// first row is r0 (zero beyond the tensor).
-__device__ __forceinline__ void load_sub(const QuantArgs& a, int b, int r0, int c0, uint4 (&reg)[4]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int q = k * kThreads + threadIdx.x;
-    const int row = q >> 4, c16 = q & 15;
-    const int gr = r0 + row, gc = c0 + c16 * 8;
-    if (gr < a.rows && gc < a.cols) {
-      reg[k] = __ldg(reinterpret_cast<const uint4*>(a.x + (long long)b * a.x_bs +
-                                                    (long long)gr * a.ld + gc));
-    } else {
-      reg[k] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-}
-
-template <int SHIFT>
-__device__ __forceinline__ void store_sub(uint8_t* tile, const uint4 (&reg)[4]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int q = k * kThreads + threadIdx.x;
-    *reinterpret_cast<uint4*>(tile + chunk_off<SHIFT>(q >> 4, q & 15)) = reg[k];
-  }
-}
 
 template <bool SWZ>
 __device__ __forceinline__ long long scale_off(const OutDesc& o, int b, long long R, long long c) {
@@ -361,10 +327,12 @@ __global__ void __launch_bounds__(kThreads, RHTC ? 2 : (SR ? FOS_DUALW_MIN_BLOCK
 // In a sub-tile, 8 threads own one 16x16 tile; thread i holds rows 2i, 2i+1
 // as the pair (A, B), so the per-row error trees come out of the pair code
 // and the tree over the 16 row sums is a horizontal add plus three
-// xor-shuffles.
+// xor-shuffles.  Each thread loads its two 32-byte tile rows itself (one
+// 256-bit load each where rows are 32-byte aligned: a warp's load covers 8
+// rows x 128 contiguous bytes), one sub-tile ahead; shared memory only
+// carries the transposed codes.
 template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
 __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x16(const QuantArgs a) {
-  __shared__ __align__(16) uint8_t s_tile[kSubRows * 256];
   __shared__ __align__(16) uint8_t s_tc[COL ? kSubCols * 32 : 16];
   __shared__ float2 s_tab[128];
   __shared__ uint32_t s_bits[kSubRows / 16];   // rowwise picks of a sub-tile: tile row -> 8 tile columns
@@ -390,15 +358,36 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
   const long long gbase = a.elem_offset + (long long)b * a.rows * a.cols;
   uint32_t bad = 0;
 
-  uint4 reg[4];
-  load_sub(a, b, rs0, c0, reg);
+  // rows 2i, 2i+1 of this thread's tile in the sub-tile starting at row r0
+  // (zero for a tile outside the tensor: rows and cols are multiples of 16)
+  const bool al32 = (reinterpret_cast<uintptr_t>(a.x) & 31) == 0 && (a.ld & 15) == 0 && (a.x_bs & 15) == 0;
+  const uint16_t* xb = a.x + (long long)b * a.x_bs;
+  auto load_rows = [&](int r0, uint4 (&ra)[2], uint4 (&rb)[2]) {
+    const long long gr = (long long)r0 + 16 * tr + 2 * i;
+    const int gc = c0 + 16 * tc;
+    if (gr < a.rows && gc < a.cols) {
+      const uint16_t* p = xb + gr * a.ld + gc;
+      if (al32) {
+        ld_block256(p, ra);
+        ld_block256(p + a.ld, rb);
+      } else {
+        ra[0] = __ldg(reinterpret_cast<const uint4*>(p));
+        ra[1] = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+        rb[0] = __ldg(reinterpret_cast<const uint4*>(p + a.ld));
+        rb[1] = __ldg(reinterpret_cast<const uint4*>(p + a.ld) + 1);
+      }
+    } else {
+      ra[0] = ra[1] = rb[0] = rb[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 na[2], nb[2];
+  load_rows(rs0, na, nb);
   for (int k = 0; k < kStrip; ++k) {
     const int r0 = rs0 + k * kSubRows;
     if (r0 >= a.rows) break;
-    __syncthreads();
-    store_sub<1>(s_tile, reg);
-    __syncthreads();
-    if (k + 1 < kStrip && r0 + kSubRows < a.rows) load_sub(a, b, r0 + kSubRows, c0, reg);
+    const uint4 wa[2] = {na[0], na[1]}, wb[2] = {nb[0], nb[1]};
+    if (k + 1 < kStrip && r0 + kSubRows < a.rows) load_rows(r0 + kSubRows, na, nb);
+    __syncthreads();  // the previous sub-tile's readers of s_tc, s_bits and s_cbits are done
 
     const long long gtr = (r0 >> 4) + tr;      // global tile row
     const long long gtc = (c0 >> 4) + tc;      // global tile column
@@ -406,11 +395,6 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
     uint32_t pick = 0;
     if (valid) {
       const int ra = 16 * tr + 2 * i;
-      uint4 wa[2], wb[2];
-      wa[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra, 2 * tc));
-      wa[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra, 2 * tc + 1));
-      wb[0] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra + 1, 2 * tc));
-      wb[1] = *reinterpret_cast<const uint4*>(s_tile + chunk_off<1>(ra + 1, 2 * tc + 1));
       float2 P[16];
       unpack_pairs(wa, wb, P);
       // the 8 lanes of one tile are all valid or all invalid: shuffle among them
