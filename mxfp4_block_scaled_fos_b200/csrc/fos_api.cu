@@ -229,11 +229,14 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
   // Which choice-bit words a CTA owns outright depends on the kernel's tiling;
   // bitmaps whose words are shared between CTAs are built with atomics on a
   // zeroed buffer.
+  int nsub = 0;
   if (opt->blk == FOS_BLOCK_16X16) {
     // rowwise: a CTA writes whole bytes (8 tile columns of one tile row);
     // transposed copy: whole 32-bit words (32 tile rows of one tile column)
+    // when its strips are 8 sub-tiles long
+    nsub = q16x16_strip(rows, cols, batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr);
     a.row.choice_aligned = (cols / 16) % 8 == 0;
-    a.col.choice_aligned = (rows / 16) % 32 == 0;
+    a.col.choice_aligned = (rows / 16) % 32 == 0 && nsub == 8;
   } else if (colwise) {
     // the warp-based kernel sets every bit with an atomic on a zeroed bitmap
     a.row.choice_aligned = a.col.choice_aligned = 0;
@@ -284,7 +287,7 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
   a.units_per_cta = kUnitsQuant;
   if (rowwise_1x16) a.units_per_cta = kBlocksRowwise;
   if (opt->blk == FOS_BLOCK_16X16) {
-    ce = launch_q16x16(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr, st);
+    ce = launch_q16x16(a, (int)batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr, nsub, st);
   } else if (colwise) {
     if (rht_col) {  // the colwise copy's own amax, in the words the fused path uses for its counts
       if (cudaMemsetAsync(done_ws, 0, 4 * batch, st) != cudaSuccess) return FOS_ERR_CUDA;

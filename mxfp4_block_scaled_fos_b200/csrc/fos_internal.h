@@ -90,8 +90,12 @@ cudaError_t launch_q1x16_dual(const QuantArgs& a, int batch, int fmt, bool sr, b
 // amax of the 16-row column blocks after the 16-wide transform (the colwise
 // copy's amax with FOS_FLAG_RHT16_COL) into zeroed words amax_col[batch]
 cudaError_t launch_amax_cols_rht(const QuantArgs& a, int batch, uint32_t* amax_col, cudaStream_t st);
+// sub-tiles (64 rows each) per CTA strip of the 2D kernel, 1..8; only a
+// strip of 8 owns whole words of the transposed copy's choice bitmap
+int q16x16_strip(long long rows, long long cols, long long batch, int fmt, bool sr, bool swz, bool want_row,
+                 bool want_col);
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz,
-                          bool want_row, bool want_col, cudaStream_t st);
+                          bool want_row, bool want_col, int nsub, cudaStream_t st);
 cudaError_t launch_mxfp4(const QuantArgs& a, int batch, bool swz, cudaStream_t st);
 
 struct DequantArgs {

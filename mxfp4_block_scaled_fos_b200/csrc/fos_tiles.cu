@@ -15,6 +15,8 @@
 // Stochastic-rounding bytes are drawn once per 16 source elements (one Philox
 // call per rowwise block) and shared by both orientations through shared
 // memory.
+#include <atomic>
+
 #include "fos_core.cuh"
 
 namespace fos {
@@ -24,7 +26,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kSubRows = 64;
 constexpr int kSubCols = 128;
-constexpr int kStrip = 8;  // sub-tiles per CTA strip (512 rows)
+constexpr int kStrip = 8;  // most sub-tiles per CTA strip (512 rows: one 32-bit word
+                           // of the transposed copy's choice bitmap per tile column)
 #ifndef FOS_2D_MIN_BLOCKS
 #define FOS_2D_MIN_BLOCKS 3
 #endif
@@ -332,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, RHTC ? 2 : (SR ? FOS_DUALW_MIN_BLOCK
 // rows x 128 contiguous bytes), one sub-tile ahead; shared memory only
 // carries the transposed codes.
 template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
-__global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x16(const QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x16(const QuantArgs a, int nsub) {
   __shared__ __align__(16) uint8_t s_tc[COL ? kSubCols * 32 : 16];
   __shared__ float2 s_tab[128];
   __shared__ uint32_t s_bits[kSubRows / 16];   // rowwise picks of a sub-tile: tile row -> 8 tile columns
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
 
   const int b = blockIdx.z;
   const int c0 = blockIdx.x * kSubCols;
-  const int rs0 = blockIdx.y * (kSubRows * kStrip);
+  const int rs0 = blockIdx.y * (kSubRows * nsub);
   const float St = tensor_scale_of(a, b, F46);
   build_scale_table(s_tab, St);
   const TScale ts = make_tscale(St);
@@ -382,11 +385,11 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
   };
   uint4 na[2], nb[2];
   load_rows(rs0, na, nb);
-  for (int k = 0; k < kStrip; ++k) {
+  for (int k = 0; k < nsub; ++k) {
     const int r0 = rs0 + k * kSubRows;
     if (r0 >= a.rows) break;
     const uint4 wa[2] = {na[0], na[1]}, wb[2] = {nb[0], nb[1]};
-    if (k + 1 < kStrip && r0 + kSubRows < a.rows) load_rows(r0 + kSubRows, na, nb);
+    if (k + 1 < nsub && r0 + kSubRows < a.rows) load_rows(r0 + kSubRows, na, nb);
     __syncthreads();  // the previous sub-tile's readers of s_tc, s_bits and s_cbits are done
 
     const long long gtr = (r0 >> 4) + tr;      // global tile row
@@ -553,12 +556,68 @@ cudaError_t launch_amax_cols_rht(const QuantArgs& a, int batch, uint32_t* amax_c
   return cudaGetLastError();
 }
 
+// The 2D kernel variant for these options.
+const void* kernel_2d(bool f46, bool sr, bool swz, bool want_row, bool want_col) {
+  const void* k = nullptr;
+#define FOS_L(F, S, W, R, C) k = reinterpret_cast<const void*>(k_2d16x16<F, S, W, R, C>)
+#define FOS_C(F, S, W, R) do { if (want_col) FOS_L(F, S, W, R, true); else FOS_L(F, S, W, R, false); } while (0)
+#define FOS_R(F, S, W) do { if (want_row) FOS_C(F, S, W, true); else FOS_C(F, S, W, false); } while (0)
+#define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)
+#define FOS_S(F) do { if (sr) FOS_W(F, true); else FOS_W(F, false); } while (0)
+  if (f46) FOS_S(true);
+  else     FOS_S(false);
+#undef FOS_S
+#undef FOS_W
+#undef FOS_R
+#undef FOS_C
+#undef FOS_L
+  return k;
+}
+
+constexpr int kMaxDev = 64;
+
+// Sub-tiles per CTA strip: the n in 1..8 whose grid of column strips x
+// ceil(rows / 64n) x batch CTAs, in rounds of the resident CTA slots, costs
+// the least, counting each CTA as n sub-tiles plus 0.3 for its start-up; the
+// longest strip on ties.  The slots come from the occupancy of the variant,
+// cached per device.
+int q16x16_strip(long long rows, long long cols, long long batch, int fmt, bool sr, bool swz, bool want_row,
+                 bool want_col) {
+  static std::atomic<int> slots_of[kMaxDev][32];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return kStrip;
+  const int v = (fmt == 0) * 16 + sr * 8 + swz * 4 + want_row * 2 + want_col;
+  int slots = slots_of[dev][v].load(std::memory_order_relaxed);
+  if (slots <= 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel_2d(fmt == 0, sr, swz, want_row, want_col),
+                                                      kThreads, 0) != cudaSuccess ||
+        sms <= 0 || per_sm <= 0) {
+      (void)cudaGetLastError();
+      return kStrip;
+    }
+    slots = sms * per_sm;
+    slots_of[dev][v].store(slots, std::memory_order_relaxed);
+  }
+  const long long cts = (cols + kSubCols - 1) / kSubCols * batch;
+  int best = kStrip;
+  long long best_cost = -1;
+  for (int n = kStrip; n >= 1; --n) {
+    const long long ctas = cts * ((rows + kSubRows * n - 1) / (kSubRows * n));
+    const long long cost = (ctas + slots - 1) / slots * (10 * n + 3);
+    if (best_cost < 0 || cost < best_cost) { best = n; best_cost = cost; }
+  }
+  return best;
+}
+
 cudaError_t launch_q16x16(const QuantArgs& a, int batch, int fmt, bool sr, bool swz, bool want_row,
-                          bool want_col, cudaStream_t st) {
+                          bool want_col, int nsub, cudaStream_t st) {
+  if (nsub < 1 || nsub > kStrip) return cudaErrorInvalidValue;
   const bool f46 = fmt == 0;
-  const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * kStrip - 1) / (kSubRows * kStrip),
+  const dim3 g((a.cols + kSubCols - 1) / kSubCols, (a.rows + kSubRows * nsub - 1) / (kSubRows * nsub),
                (unsigned)batch);
-#define FOS_L(F, S, W, R, C) k_2d16x16<F, S, W, R, C><<<g, kThreads, 0, st>>>(a)
+#define FOS_L(F, S, W, R, C) k_2d16x16<F, S, W, R, C><<<g, kThreads, 0, st>>>(a, nsub)
 #define FOS_C(F, S, W, R) do { if (want_col) FOS_L(F, S, W, R, true); else FOS_L(F, S, W, R, false); } while (0)
 #define FOS_R(F, S, W) do { if (want_row) FOS_C(F, S, W, true); else FOS_C(F, S, W, false); } while (0)
 #define FOS_W(F, S) do { if (swz) FOS_R(F, S, true); else FOS_R(F, S, false); } while (0)

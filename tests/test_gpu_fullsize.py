@@ -36,6 +36,7 @@ def test_weight_normal_2d_full():
     assert_bytes_equal(c.scales.cpu().numpy(), ref["c_scales"], "c_scales")
     assert r.tensor_scale.cpu().numpy().view(np.uint32)[0] == ref["tensor_scale"].view(np.uint32)[0]
     compare_choice(r.choice, ref["r_choice"], (14336 // 16) * (4096 // 16), "r")
+    compare_choice(c.choice, ref["c_choice"], (14336 // 16) * (4096 // 16), "c")
 
 
 def test_gradient_student_t_sr_dual_sampled():
