@@ -337,6 +337,11 @@ __global__ void __launch_bounds__(kThreads, RHTC ? 2 : (SR ? FOS_DUALW_MIN_BLOCK
 template <bool F46, bool SR, bool SWZ, bool ROW, bool COL>
 __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x16(const QuantArgs a, int nsub) {
   __shared__ __align__(16) uint8_t s_tc[COL ? kSubCols * 32 : 16];
+  // scale bytes, written out as 4-byte words: the sub-tile's rowwise scales
+  // [64 rows][8 tile columns] and the strip's transposed-copy scales
+  // [128 columns][32 tile rows]
+  __shared__ __align__(16) uint8_t s_rsc[ROW ? kSubRows * 8 : 16];
+  __shared__ __align__(16) uint8_t s_csc[COL ? kSubCols * 32 : 16];
   __shared__ float2 s_tab[128];
   __shared__ uint32_t s_bits[kSubRows / 16];   // rowwise picks of a sub-tile: tile row -> 8 tile columns
   __shared__ uint32_t s_cbits[kSubCols / 16];  // transposed copy: tile column -> 32 tile rows of the strip
@@ -364,6 +369,11 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
   // rows 2i, 2i+1 of this thread's tile in the sub-tile starting at row r0
   // (zero for a tile outside the tensor: rows and cols are multiples of 16)
   const bool al32 = (reinterpret_cast<uintptr_t>(a.x) & 31) == 0 && (a.ld & 15) == 0 && (a.x_bs & 15) == 0;
+  // 4 consecutive scales of a row (4-aligned) form one aligned word; the
+  // transposed codes of 32 rows one aligned 16-byte run
+  const bool rsc_word = (a.row.scales_bs & 3) == 0 && (SWZ || (a.row.scales_ld & 3) == 0);
+  const bool csc_word = (a.col.scales_bs & 3) == 0 && (SWZ || (a.col.scales_ld & 3) == 0);
+  const bool cc16 = (a.col.codes_bs & 15) == 0 && (a.col.codes_ld & 15) == 0;
   const uint16_t* xb = a.x + (long long)b * a.x_bs;
   auto load_rows = [&](int r0, uint4 (&ra)[2], uint4 (&rb)[2]) {
     const long long gr = (long long)r0 + 16 * tr + 2 * i;
@@ -435,8 +445,8 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
       if (ROW) {
         store_codes8(a.row, b, grA, gtc * 8, ca[0], ca[1]);
         store_codes8(a.row, b, grA + 1, gtc * 8, cb[0], cb[1]);
-        a.row.scales[scale_off<SWZ>(a.row, b, grA, gtc)] = (uint8_t)s;
-        a.row.scales[scale_off<SWZ>(a.row, b, grA + 1, gtc)] = (uint8_t)s;
+        s_rsc[ra * 8 + tc] = (uint8_t)s;
+        s_rsc[(ra + 1) * 8 + tc] = (uint8_t)s;
       }
       if (COL) {
         // byte for rows (2i, 2i+1) of each of the tile's 16 columns.  In a
@@ -457,9 +467,8 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
             s_tc[(16 * tc + 8 * w + 2 * k) * 32 + gofs] = (uint8_t)(E[w] >> (8 * k));
             s_tc[(16 * tc + 8 * w + 2 * k + 1) * 32 + gofs] = (uint8_t)(O[w] >> (8 * k));
           }
-        const long long gcA = (c0 + 16 * tc) + 2 * i;
-        a.col.scales[scale_off<SWZ>(a.col, b, gcA, gtr)] = (uint8_t)s;
-        a.col.scales[scale_off<SWZ>(a.col, b, gcA + 1, gtr)] = (uint8_t)s;
+        s_csc[(16 * tc + 2 * i) * 32 + 4 * k + tr] = (uint8_t)s;
+        s_csc[(16 * tc + 2 * i + 1) * 32 + 4 * k + tr] = (uint8_t)s;
       }
       if (F46 && i == 0 && pick) {
         if (ROW && a.row.choice) atomicOr(&s_bits[tr], 1u << tc);
@@ -476,9 +485,28 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
         const int sw = (col >> 4) & 3;   // the group swizzle of this column's tile column
         const uint2 v0 = *reinterpret_cast<const uint2*>(s_tc + col * 32 + 8 * ((2 * h) ^ sw));
         const uint2 v1 = *reinterpret_cast<const uint2*>(s_tc + col * 32 + 8 * ((2 * h + 1) ^ sw));
-        const long long byte_col = grow / 2;
-        store_codes8(a.col, b, gc, byte_col, v0.x, v0.y);
-        if (grow + 16 < a.rows) store_codes8(a.col, b, gc, byte_col + 8, v1.x, v1.y);
+        const long long byte_col = grow / 2;   // a multiple of 16
+        if (grow + 16 < a.rows && cc16) {
+          *reinterpret_cast<uint4*>(a.col.codes + (long long)b * a.col.codes_bs + gc * a.col.codes_ld + byte_col) =
+              make_uint4(v0.x, v0.y, v1.x, v1.y);
+        } else {
+          store_codes8(a.col, b, gc, byte_col, v0.x, v0.y);
+          if (grow + 16 < a.rows) store_codes8(a.col, b, gc, byte_col + 8, v1.x, v1.y);
+        }
+      }
+    }
+    if (ROW && t < kSubRows * 2) {
+      // rowwise scales: row t / 2, tile columns 4 (t & 1) .. + 3 of the sub-tile
+      const int row = t >> 1, hf = t & 1;
+      const long long R = r0 + row, gc4 = (c0 >> 4) + 4 * hf;
+      if (R < a.rows && gc4 < ntc) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(s_rsc + row * 8 + 4 * hf);
+        if (rsc_word && gc4 + 4 <= ntc) {
+          *reinterpret_cast<uint32_t*>(a.row.scales + scale_off<SWZ>(a.row, b, R, gc4)) = v;
+        } else {
+          for (int q = 0; q < 4 && gc4 + q < ntc; ++q)
+            a.row.scales[scale_off<SWZ>(a.row, b, R, gc4 + q)] = (uint8_t)(v >> (8 * q));
+        }
       }
     }
     // rowwise copy: one bit per tile in the tile row-major order of x, so a
@@ -501,11 +529,32 @@ __global__ void __launch_bounds__(kThreads, SR ? 2 : FOS_2D_MIN_BLOCKS) k_2d16x1
       }
     }
   }
+  if (COL) {
+    __syncthreads();
+    // the strip's transposed-copy scales: column col holds tile rows tr0 ..
+    // tr0 + 4 nk - 1, one word per sub-tile; consecutive threads take
+    // consecutive words of a column
+    const long long left = (a.rows - rs0 + kSubRows - 1) / kSubRows;   // sub-tiles left from rs0
+    const int nk = left < nsub ? (int)left : nsub;
+    const long long tr0 = rs0 >> 4;   // a multiple of 4
+    for (int idx = t; idx < kSubCols * nk; idx += kThreads) {
+      const int col = idx / nk, w = idx - col * nk;
+      const long long c = c0 + col, trw = tr0 + 4 * w;
+      if (c < a.cols && trw < ntr) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(s_csc + col * 32 + 4 * w);
+        if (csc_word && trw + 4 <= ntr) {
+          *reinterpret_cast<uint32_t*>(a.col.scales + scale_off<SWZ>(a.col, b, c, trw)) = v;
+        } else {
+          for (int q = 0; q < 4 && trw + q < ntr; ++q)
+            a.col.scales[scale_off<SWZ>(a.col, b, c, trw + q)] = (uint8_t)(v >> (8 * q));
+        }
+      }
+    }
+  }
   // transposed copy: one bit per tile in the tile row-major order of x^T
   // ([cols][rows]), so source tile (gtr, gtc) is bit (b*ntc + gtc)*ntr + gtr
   // and the strip's 32 tile rows of one tile column are 32 consecutive bits
   if (COL && F46 && a.col.choice) {
-    __syncthreads();
     if (t < kSubCols / 16) {
       const long long gtc = (c0 >> 4) + t;
       if (gtc < ntc) {
