@@ -35,6 +35,22 @@ fos_status fos_testing_quantize_stalled(const void* x, int64_t batch, int64_t ro
                                         size_t workspace_bytes, uint32_t* status,
                                         int32_t stall_entry, uint32_t spin_limit, void* stream);
 
+/*
+ * fos_testing_quantize_2d_strip -- fos_quantize with the 16x16 2D kernel's
+ * strip length forced to `nsub` sub-tiles of 64 rows (1..8) instead of the
+ * length the library picks per launch to fill the GPU's resident CTA slots.
+ * Tests use it to reach every strip length, and the transposed copy's
+ * whole-word choice-bitmap stores that only strips of 8 take.  Arguments and
+ * outputs are those of fos_quantize: the results do not depend on the strip
+ * length.  opt->blk must be FOS_BLOCK_16X16 (FOS_ERR_UNSUPPORTED otherwise);
+ * nsub outside 1..8 gives FOS_ERR_ARG.
+ */
+fos_status fos_testing_quantize_2d_strip(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                                         int64_t ld, const fos_options* opt, const float* amax_in,
+                                         const fos_qtensor* rowwise, const fos_qtensor* colwise,
+                                         void* workspace, size_t workspace_bytes, uint32_t* status,
+                                         int32_t nsub, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -4,6 +4,7 @@
 
 #include "fos.h"
 #include "fos_internal.h"
+#include "fos_testing.h"
 
 namespace fos {
 
@@ -69,10 +70,13 @@ OutDesc make_out(const fos_qtensor* q, int64_t R, int64_t C, int64_t bs, uint32_
 
 size_t choice_bytes(int64_t nblocks) { return (size_t)(8 * ((nblocks + 63) / 64)); }
 
-// Test hooks of the fused kernel's bounded waits (fos_testing_quantize_stalled).
+// Test hooks: the fused kernel's bounded waits (fos_testing_quantize_stalled)
+// and the 2D kernel's strip length (fos_testing_quantize_2d_strip; 0 = the
+// per-launch choice).
 struct WaitHooks {
   uint32_t spin_limit = 1u << 21;
   int stall_entry = -1;
+  int strip_2d = 0;
 };
 
 fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
@@ -138,6 +142,20 @@ fos_status fos_testing_quantize_stalled(const void* x, int64_t batch, int64_t ro
   h.spin_limit = spin_limit;
   h.stall_entry = stall_entry;
   return quantize_impl(x, batch, rows, cols, ld, opt, nullptr, rowwise, nullptr, workspace,
+                       workspace_bytes, status, stream, h);
+}
+
+fos_status fos_testing_quantize_2d_strip(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                                         int64_t ld, const fos_options* opt, const float* amax_in,
+                                         const fos_qtensor* rowwise, const fos_qtensor* colwise,
+                                         void* workspace, size_t workspace_bytes, uint32_t* status,
+                                         int32_t nsub, void* stream) {
+  if (!opt) return FOS_ERR_NULL;
+  if (opt->blk != FOS_BLOCK_16X16) return FOS_ERR_UNSUPPORTED;
+  if (nsub < 1 || nsub > 8) return FOS_ERR_ARG;
+  WaitHooks h;
+  h.strip_2d = nsub;
+  return quantize_impl(x, batch, rows, cols, ld, opt, amax_in, rowwise, colwise, workspace,
                        workspace_bytes, status, stream, h);
 }
 
@@ -234,7 +252,9 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
     // rowwise: a CTA writes whole bytes (8 tile columns of one tile row);
     // transposed copy: whole 32-bit words (32 tile rows of one tile column)
     // when its strips are 8 sub-tiles long
-    nsub = q16x16_strip(rows, cols, batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr);
+    nsub = hooks.strip_2d > 0
+               ? hooks.strip_2d
+               : q16x16_strip(rows, cols, batch, opt->fmt, sr, swz, rowwise != nullptr, colwise != nullptr);
     a.row.choice_aligned = (cols / 16) % 8 == 0;
     a.col.choice_aligned = (rows / 16) % 32 == 0 && nsub == 8;
   } else if (colwise) {

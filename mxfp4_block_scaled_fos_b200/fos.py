@@ -37,7 +37,8 @@ ERRORS = {
 # every symbol include/fos.h declares
 EXPORTS = ("fos_quantize", "fos_amax", "fos_dequantize", "fos_workspace_size",
            "fos_scales_size", "fos_status_string", "fos_version", "fos_quantize_static",
-           "fos_testing_quantize_stalled", "fos_fake_quantize", "fos_gemm_nvfp4")
+           "fos_testing_quantize_stalled", "fos_testing_quantize_2d_strip", "fos_fake_quantize",
+           "fos_gemm_nvfp4")
 
 
 class Options(ctypes.Structure):
@@ -82,6 +83,10 @@ def lib(path: str = LIB_PATH):
     L.fos_testing_quantize_stalled.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options),
                                                ctypes.POINTER(QTensorC), P, ctypes.c_size_t, P,
                                                i32, u32, P]
+    L.fos_testing_quantize_2d_strip.restype = i32
+    L.fos_testing_quantize_2d_strip.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P,
+                                                ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), P,
+                                                ctypes.c_size_t, P, i32, P]
     L.fos_fake_quantize.restype = i32
     L.fos_fake_quantize.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P, P, i64, P,
                                     ctypes.c_size_t, P, P]

@@ -60,11 +60,29 @@ def zeroed_out(batch, R, C, fmt, block, flags, device, nblocks, choice=True):
     return F.QTensor(codes, scales, ts, ch, batch, R, C, fmt, block, flags)
 
 
+def quantize_2d_strip(x3, opts, amax, orow, ocol, status, nsub):
+    """fos_testing_quantize_2d_strip (include/fos_testing.h): fos_quantize
+    with the 2D kernel's strip length forced to nsub sub-tiles."""
+    import ctypes
+    batch, R, C = x3.shape
+    ws = torch.zeros(F.workspace_size(batch, R, C), dtype=torch.uint8, device=x3.device)
+    rc = orow.c_struct() if orow is not None else None
+    cc = ocol.c_struct() if ocol is not None else None
+    st = F.lib().fos_testing_quantize_2d_strip(
+        ctypes.c_void_p(x3.data_ptr()), batch, R, C, x3.stride(1), ctypes.byref(opts),
+        ctypes.c_void_p(amax.data_ptr()) if amax is not None else None,
+        ctypes.byref(rc) if rc is not None else None, ctypes.byref(cc) if cc is not None else None,
+        ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.c_void_p(status.data_ptr()), nsub,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, F.ERRORS.get(st, st)
+
+
 def check_quantize(x: torch.Tensor, fmt="nvfp4_46", block=None, rounding="rne", rht=False,
                    swizzle=False, seed=0, elem_offset=0, rowwise=True, colwise=False,
-                   amax=None, x_bits=None, rht_col=False):
+                   amax=None, x_bits=None, rht_col=False, strip_2d=None):
     """Quantize x on the GPU and with the oracle; assert bit equality of
-    codes, scales, tensor scales and choice bits.  Returns the GPU outputs."""
+    codes, scales, tensor scales and choice bits.  Returns the GPU outputs.
+    strip_2d: run the 16x16 kernel with that many sub-tiles per strip."""
     block = block or ("1x32" if fmt == "mxfp4" else "1x16")
     x3 = x if x.dim() == 3 else x.unsqueeze(0)
     batch, R, C = x3.shape
@@ -76,9 +94,14 @@ def check_quantize(x: torch.Tensor, fmt="nvfp4_46", block=None, rounding="rne", 
                       n_blocks(batch, C, R, "1x16") if block == "1x16" else n_blocks(batch, R, C, block)) \
         if colwise else None
     status = torch.zeros(1, dtype=torch.int32, device=x.device)
-    F.quantize(x3, fmt=fmt, block=block, rounding=rounding, rht=rht, swizzle=swizzle, seed=seed,
-               elem_offset=elem_offset, rowwise=rowwise, colwise=colwise, amax=amax,
-               status=status, out_row=orow, out_col=ocol, rht_col=rht_col)
+    if strip_2d is None:
+        F.quantize(x3, fmt=fmt, block=block, rounding=rounding, rht=rht, swizzle=swizzle, seed=seed,
+                   elem_offset=elem_offset, rowwise=rowwise, colwise=colwise, amax=amax,
+                   status=status, out_row=orow, out_col=ocol, rht_col=rht_col)
+    else:
+        from mxfp4_block_scaled_fos_b200.fos import BLK, FMT, RND, Options
+        opts = Options(FMT[fmt], BLK[block], RND[rounding], flags, seed, elem_offset)
+        quantize_2d_strip(x3, opts, amax, orow, ocol, status, strip_2d)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     xb = x_bits if x_bits is not None else np_bits(x3.contiguous() if x3.stride(1) != C else x3)

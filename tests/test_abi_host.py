@@ -95,6 +95,23 @@ def test_argument_errors(L):
     assert _call(L, rows=-1) == 3
 
 
+def test_strip_hook_argument_errors(L):
+    """fos_testing_quantize_2d_strip checks its own arguments before any
+    device work: 16x16 blocks only, 1..8 sub-tiles per strip."""
+    q = QTensorC(64, 128, 256, None, 16, 2)
+
+    def call(blk, nsub):
+        o = Options(0, blk, 0, 0, 0, 0)
+        return L.fos_testing_quantize_2d_strip(ctypes.c_void_p(16), 1, 32, 32, 32, ctypes.byref(o), None,
+                                               ctypes.byref(q), None, ctypes.c_void_p(16), 1 << 16, None,
+                                               nsub, None)
+    assert call(0, 4) == 4      # 1x16
+    assert call(1, 0) == 7
+    assert call(1, 9) == 7
+    assert L.fos_testing_quantize_2d_strip(ctypes.c_void_p(16), 1, 32, 32, 32, None, None, ctypes.byref(q),
+                                           None, None, 0, None, 4, None) == 1
+
+
 def test_library_has_no_oracle_dependency():
     """The product library must not link or name the CPU oracle."""
     src_dir = os.path.join(ROOT, "mxfp4_block_scaled_fos_b200")

@@ -91,6 +91,22 @@ def test_2d_16x16(shape, rounding, fmt):
     check_quantize(x, fmt=fmt, block="16x16", rounding=rounding, seed=5, rowwise=True, colwise=True)
 
 
+@pytest.mark.parametrize("nsub", range(1, 9))
+def test_2d_every_strip_length(nsub):
+    """The 2D kernel's results do not depend on how many 64-row sub-tiles a
+    CTA strip holds (the library picks it per launch).  1040 rows end strips
+    of every length early; 2048 rows make the transposed bitmap's 32-bit
+    words whole, which strips of 8 store directly."""
+    dev = require_gpu()
+    for shape, seed in (((2, 1040, 400), 3), ((1, 2048, 384), 4)):
+        x = _rand(shape, seed, dev, "scaled")
+        check_quantize(x, block="16x16", rowwise=True, colwise=True, strip_2d=nsub)
+        check_quantize(x, block="16x16", rowwise=True, colwise=True, swizzle=True, rounding="sr", seed=9,
+                       strip_2d=nsub)
+    x = _rand((1, 528, 272), 5, dev, "scaled")
+    check_quantize(x, fmt="nvfp4_6", block="16x16", rowwise=False, colwise=True, strip_2d=nsub)
+
+
 @pytest.mark.parametrize("row,col", [(True, False), (False, True)])
 def test_2d_one_orientation_and_swizzle(row, col):
     dev = require_gpu()
