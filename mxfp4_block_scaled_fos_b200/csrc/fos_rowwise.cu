@@ -508,6 +508,34 @@ __device__ __forceinline__ uint32_t slice_amax_bits(const QuantArgs& a, int b, u
   return m;
 }
 
+// K0 on rows stored contiguously (ld == cols, 32-byte aligned entries): the
+// blocks of an entry are one array, read 256 bits at a time with several
+// loads in flight (the fused kernel's amax loop), marked evict-last so that
+// the quantizer that follows finds part of them in L2.  grid (chunks, batch),
+// units_per_cta blocks per CTA.
+template <bool RHT>
+__global__ void __launch_bounds__(kThreads) k_amax_dense(const QuantArgs a, uint32_t* amax_ws) {
+  const int b = blockIdx.y;
+  const uint32_t lo = blockIdx.x * a.units_per_cta, hi = min(lo + a.units_per_cta, a.nblk);
+  const uint32_t mask16 = RHT ? rht_sign_mask(a.seed) : 0u;
+  uint32_t m = slice_amax_bits<RHT, true>(a, b, lo, hi, mask16, l2_policy_evict_last(), threadIdx.x);
+  m = __reduce_max_sync(0xffffffffu, m);
+  __shared__ uint32_t s_m[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) s_m[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t v = threadIdx.x < kThreads / 32 ? s_m[threadIdx.x] : 0u;
+    v = __reduce_max_sync(0xffffffffu, v);
+    if (threadIdx.x == 0) {
+      if (v >= 0x7f800000u) {
+        if (a.status) atomicOr(a.status, FOS_STATUS_NONFINITE);
+      } else if (v) {
+        atomicMax(amax_ws + b, v);
+      }
+    }
+  }
+}
+
 // The item sequence of one launch (computed on the host).
 struct FusedPlan {
   uint32_t na, nq;         // amax and quantize items per entry
@@ -790,15 +818,6 @@ static dim3 grid_for(uint32_t units, uint32_t per_cta, int batch) {
   return dim3((units + per_cta - 1) / per_cta, (unsigned)batch, 1);
 }
 
-cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_ws,
-                        cudaStream_t st) {
-  const uint32_t nunit = (a.nblk + 1) / 2;
-  const dim3 g = grid_for(nunit, a.units_per_cta, batch);
-  if (rht) k_amax<true><<<g, kThreads, 0, st>>>(a, amax_ws);
-  else     k_amax<false><<<g, kThreads, 0, st>>>(a, amax_ws);
-  return cudaGetLastError();
-}
-
 // Blocks per CTA for `nblk` blocks in each of `batch` entries on `slots`
 // resident CTAs: at most max_units, a multiple of 32 (whole choice words),
 // and spread so that the last wave of CTAs is about as full as the others
@@ -811,6 +830,40 @@ static uint32_t balanced_units(uint32_t nblk, int batch, uint32_t max_units, int
   unsigned long long u = (total + waves * slots - 1) / (waves * slots);
   u = (u + 31) / 32 * 32;
   return (uint32_t)(u < 32 ? 32 : (u > max_units ? max_units : u));
+}
+
+// The dense amax kernel with 2 * units_per_cta blocks per CTA at most,
+// spread over whole waves of its resident slots (looked up once per device).
+template <bool RHT>
+static cudaError_t launch_amax_dense(const QuantArgs& a, int batch, uint32_t* amax_ws, cudaStream_t st) {
+  static std::atomic<int> slots_of[kMaxDevices];
+  auto kern = k_amax_dense<RHT>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
+  int slots = slots_of[dev].load(std::memory_order_relaxed);
+  if (slots == 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess)
+      return cudaErrorNotSupported;
+    slots = sms * (per_sm > 0 ? per_sm : 1);
+    slots_of[dev].store(slots, std::memory_order_relaxed);
+  }
+  QuantArgs b = a;
+  b.units_per_cta = balanced_units(a.nblk, batch, 2 * a.units_per_cta, slots);
+  kern<<<grid_for(a.nblk, b.units_per_cta, batch), kThreads, 0, st>>>(b, amax_ws);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax(const QuantArgs& a, int batch, bool rht, uint32_t* amax_ws,
+                        cudaStream_t st) {
+  if (a.ld == a.cols && (reinterpret_cast<uintptr_t>(a.x) & 31) == 0 && (a.x_bs & 15) == 0)
+    return rht ? launch_amax_dense<true>(a, batch, amax_ws, st) : launch_amax_dense<false>(a, batch, amax_ws, st);
+  const uint32_t nunit = (a.nblk + 1) / 2;
+  const dim3 g = grid_for(nunit, a.units_per_cta, batch);
+  if (rht) k_amax<true><<<g, kThreads, 0, st>>>(a, amax_ws);
+  else     k_amax<false><<<g, kThreads, 0, st>>>(a, amax_ws);
+  return cudaGetLastError();
 }
 
 // One k_q1x16 variant, with the work per CTA balanced over the resident
