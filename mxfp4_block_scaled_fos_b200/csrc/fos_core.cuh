@@ -24,6 +24,42 @@ __device__ __forceinline__ uint32_t rht_word_mask(uint32_t mask16, int k) {
   return (((mask16 >> (2 * k)) & 1u) << 15) | (((mask16 >> (2 * k + 1)) & 1u) << 31);
 }
 
+// The sign flips of a whole block (8 words of bf16 pairs).  One 64-bit
+// spread s of the 16 sign bits holds bit 2k at bit 15 + 2k and bit 2k + 1 at
+// bit 31 + 2k, so word k's mask is (s >> 2k) & 0x80008000.
+__device__ __forceinline__ void rht_flip_signs(uint4 (&w)[2], uint32_t mask16) {
+  const unsigned long long s = ((unsigned long long)mask16 << 15) | ((unsigned long long)mask16 << 30);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    (&w[0].x)[k] ^= (uint32_t)(s >> (2 * k)) & 0x80008000u;
+    (&w[1].x)[k] ^= (uint32_t)(s >> (2 * k + 8)) & 0x80008000u;
+  }
+}
+
+// max(|a|, |b|, |c|) in binary32, NaN when any input is NaN.
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float d;
+  asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// max |v| of 16 binary32 values as bits (the same bits as the largest
+// |v| bit pattern; >= 0x7f800000 when one is infinite or NaN).
+__device__ __forceinline__ uint32_t amax_bits16(float v0, float v1, float v2, float v3, float v4, float v5,
+                                                float v6, float v7, float v8, float v9, float v10, float v11,
+                                                float v12, float v13, float v14, float v15) {
+  const float a = max3_abs(v0, v1, v2), b = max3_abs(v3, v4, v5), c = max3_abs(v6, v7, v8);
+  const float d = max3_abs(v9, v10, v11), e = max3_abs(v12, v13, v14);
+  const float m = max3_abs(max3_abs(a, b, c), max3_abs(d, e, v15), 0.0f);
+  return __float_as_uint(m) & 0x7fffffffu;
+}
+
+// max |P[k].x|, |P[k].y| of a block in split form (16 values).
+__device__ __forceinline__ uint32_t amax_bits_split(const float2 (&P)[8]) {
+  return amax_bits16(P[0].x, P[0].y, P[1].x, P[1].y, P[2].x, P[2].y, P[3].x, P[3].y, P[4].x, P[4].y, P[5].x,
+                     P[5].y, P[6].x, P[6].y, P[7].x, P[7].y);
+}
+
 // In-place 16-point fast Walsh-Hadamard transform of the packed pairs with
 // butterflies (a, b) -> (a + b, a - b) at strides 1, 2, 4, 8, then * 0.25.
 __device__ __forceinline__ void fwht16_pairs(float2 (&P)[16]) {
@@ -78,13 +114,10 @@ __device__ __forceinline__ uint32_t amax_bits_bf16(const uint4 (&w)[2]) {
 
 // max |P[i].x| and max |P[i].y| as binary32 bits.
 __device__ __forceinline__ void amax_bits_pairs(const float2 (&P)[16], uint32_t& ma, uint32_t& mb) {
-  ma = 0;
-  mb = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    ma = max(ma, __float_as_uint(P[i].x) & 0x7fffffffu);
-    mb = max(mb, __float_as_uint(P[i].y) & 0x7fffffffu);
-  }
+  ma = amax_bits16(P[0].x, P[1].x, P[2].x, P[3].x, P[4].x, P[5].x, P[6].x, P[7].x, P[8].x, P[9].x, P[10].x,
+                   P[11].x, P[12].x, P[13].x, P[14].x, P[15].x);
+  mb = amax_bits16(P[0].y, P[1].y, P[2].y, P[3].y, P[4].y, P[5].y, P[6].y, P[7].y, P[8].y, P[9].y, P[10].y,
+                   P[11].y, P[12].y, P[13].y, P[14].y, P[15].y);
 }
 
 // The per-tensor scale with what the block-scale step needs of it.
@@ -363,20 +396,12 @@ __device__ __forceinline__ void store_block(const OutDesc& o, int b, uint32_t j,
 
 // max |y| of the 16-wide RHT y of one block (as binary32 bits).
 __device__ __forceinline__ uint32_t rht_block_amax(uint4 (&w)[2], uint32_t mask16) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    (&w[0].x)[k] ^= rht_word_mask(mask16, k);
-    (&w[1].x)[k] ^= rht_word_mask(mask16, k + 4);
-  }
+  rht_flip_signs(w, mask16);
   const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
   float2 P[8];
   unpack_split(W, P);
   fwht16_split(P);
-  uint32_t m = 0;
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
-  return m;
+  return amax_bits_split(P);
 }
 
 // candidate1 with the scale as a table entry t = (inv, inv, -E, -E): both

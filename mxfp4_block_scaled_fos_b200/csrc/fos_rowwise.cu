@@ -63,12 +63,8 @@ __global__ void __launch_bounds__(kThreads) k_amax(const QuantArgs a, uint32_t* 
     if (has1) load_block(a, b, j0 + 1, wb);
     else      { wb[0] = wa[0]; wb[1] = wa[1]; }
     if (RHT) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t xa = rht_word_mask(mask16, k), xb = rht_word_mask(mask16, k + 4);
-        (&wa[0].x)[k] ^= xa; (&wb[0].x)[k] ^= xa;
-        (&wa[1].x)[k] ^= xb; (&wb[1].x)[k] ^= xb;
-      }
+      rht_flip_signs(wa, mask16);
+      rht_flip_signs(wb, mask16);
       float2 P[16];
       unpack_pairs(wa, wb, P);
       fwht16_pairs(P);
@@ -160,11 +156,7 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float4* s_tab
                                               long long e0, uint32_t& bad, uint32_t (&codes)[2],
                                               uint32_t& sc, bool& pick) {
   if (RHT) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      (&w[0].x)[k] ^= rht_word_mask(mask16, k);
-      (&w[1].x)[k] ^= rht_word_mask(mask16, k + 4);
-    }
+    rht_flip_signs(w, mask16);
   }
   const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
   float2 P[8];
@@ -172,10 +164,7 @@ __device__ __forceinline__ void rowwise_block(uint4 (&w)[2], const float4* s_tab
   uint32_t m;
   if (RHT) {
     fwht16_split(P);
-    m = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
+    m = amax_bits_split(P);
   } else {
     m = amax_bits_bf16(w);
   }
@@ -296,11 +285,7 @@ __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_
     uint32_t pick = 0;
     {  // computed for every lane (a missing block reads as zeros); only stores are predicated
       if (RHT) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          (&w[0].x)[k] ^= rht_word_mask(mask16, k);
-          (&w[1].x)[k] ^= rht_word_mask(mask16, k + 4);
-        }
+        rht_flip_signs(w, mask16);
       }
       const uint32_t W[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
       float2 P[8];
@@ -308,10 +293,7 @@ __device__ __forceinline__ void rowwise_range(const QuantArgs& a, int b, uint32_
       uint32_t m;
       if (RHT) {
         fwht16_split(P);
-        m = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
+        m = amax_bits_split(P);
       } else {
         m = amax_bits_bf16(w);
       }
@@ -487,19 +469,13 @@ __device__ __forceinline__ uint32_t slice_amax_bits(const QuantArgs& a, int b, u
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (RHT) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          (&w[u][0].x)[k] ^= rht_word_mask(mask16, k);
-          (&w[u][1].x)[k] ^= rht_word_mask(mask16, k + 4);
-        }
+        rht_flip_signs(w[u], mask16);
         const uint32_t W[8] = {w[u][0].x, w[u][0].y, w[u][0].z, w[u][0].w,
                                w[u][1].x, w[u][1].y, w[u][1].z, w[u][1].w};
         float2 P[8];
         unpack_split(W, P);
         fwht16_split(P);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          m = max(m, max(__float_as_uint(P[k].x) & 0x7fffffffu, __float_as_uint(P[k].y) & 0x7fffffffu));
+        m = max(m, amax_bits_split(P));
       } else {
         m = max(m, amax_bits_bf16(w[u]));
       }

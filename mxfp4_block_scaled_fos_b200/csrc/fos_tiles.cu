@@ -171,9 +171,9 @@ __global__ void __launch_bounds__(kThreads) k_amax_cols_rht(const QuantArgs a, u
       T[r] = make_float2(bf_lo(w), bf_hi(w));
     }
     fwht16_pairs(T);
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-      m = max(m, max(__float_as_uint(T[r].x) & 0x7fffffffu, __float_as_uint(T[r].y) & 0x7fffffffu));
+    uint32_t ma, mb;
+    amax_bits_pairs(T, ma, mb);
+    m = max(m, max(ma, mb));
   }
   m = __reduce_max_sync(0xffffffffu, m);
   if ((threadIdx.x & 31) == 0) {
@@ -265,12 +265,7 @@ __global__ void __launch_bounds__(kThreads, RHTC ? 2 : (SR ? FOS_DUALW_MIN_BLOCK
           T[r] = make_float2(bf_lo(wr), bf_hi(wr));
         }
         fwht16_pairs(T);
-        mc[0] = mc[1] = 0;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          mc[0] = max(mc[0], __float_as_uint(T[r].x) & 0x7fffffffu);
-          mc[1] = max(mc[1], __float_as_uint(T[r].y) & 0x7fffffffu);
-        }
+        amax_bits_pairs(T, mc[0], mc[1]);
       } else {
         uint32_t h[8];
 #pragma unroll
