@@ -227,7 +227,7 @@ fos_status fos_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int64_t M,
  * capture (cudaMalloc cannot be captured), serving paths that must not
  * allocate because an allocation can synchronize the device, and hosts or
  * plugins whose memory is owned by another allocator that hands out no
- * scratch buffers.  The paper has no counterpart; this is a deployment aid.
+ * scratch buffers.  The method itself has no such call; this is a deployment aid.
  *
  * Arguments, outputs and errors are those of fos_quantize.  The scratch
  * memory (per-batch-entry amax words and counters) lives in a fixed array in the

@@ -69,7 +69,7 @@ def test_swizzled_scales_drive_cublas_block_scaled_gemm(fmt):
     try:
         out = torch._scaled_mm(A, B.t(), qa.scales.view(-1).view(sdt), qb.scales.view(-1).view(sdt),
                                out_dtype=torch.float32)
-    except (RuntimeError, NotImplementedError) as e:   # no block-scaled FP4 GEMM in this build
+    except (RuntimeError, NotImplementedError) as e:   # this torch has no block-scaled FP4 GEMM
         pytest.skip("cuBLAS block-scaled FP4 GEMM unavailable: %s" % str(e).splitlines()[0])
     torch.cuda.synchronize()
     got = out.double().cpu().numpy() * (sta * stb)
