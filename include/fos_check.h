@@ -45,6 +45,12 @@ int fosck_div_tscale_bf16(float divisor, unsigned long long* counts, void* strea
 int fosck_div_tscale_random(unsigned long long seed, unsigned long long n,
                             unsigned long long* counts, void* stream);
 
+/* n seeded random (counter, key) pairs through the kernels' Philox4x32-10
+ * (Salmon et al., SC'11; the SR bytes and the RHT signs) and through
+ * cuRAND's curand_Philox4x32_10.  counts[0] += output words that differ. */
+int fosck_philox_vs_curand(unsigned long long seed, unsigned long long n, unsigned long long* counts,
+                           void* stream);
+
 /* Every binary32 v in [0, 16] and +inf with every byte 0..255: the E2M1 code
  * of the integer form and of the pair (ceiling) form of the
  * stochastic-rounding rule against the float form.  counts[0] += mismatching

@@ -25,6 +25,8 @@
 // bounded output arrays.
 #include <stdint.h>
 
+#include <curand_kernel.h>  // curand_Philox4x32_10: cuRAND's Philox4x32-10, called as a reference
+
 #include "fos_check.h"
 #include "fos_core.cuh"
 
@@ -139,6 +141,23 @@ __global__ void k_div_tscale_random(unsigned long long seed, unsigned long long 
   }
   if (bad_code) atomicAdd(counts + 0, bad_code);
   if (bad_bits) atomicAdd(counts + 1, bad_bits);
+}
+
+// ------------------------------------------------------------ Philox
+// n seeded random (counter, key) pairs: the kernels' Philox4x32-10 against
+// cuRAND's; counts[0] += output words that differ.
+__global__ void k_philox_vs_curand(unsigned long long seed, unsigned long long n, unsigned long long* counts) {
+  unsigned long long bad = 0;
+  for (unsigned long long u = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x; u < n;
+       u += (unsigned long long)gridDim.x * blockDim.x) {
+    const unsigned long long h = seed * 0x9E3779B97F4A7C15ull + 8 * u;
+    const uint4 c = make_uint4(mix32(h), mix32(h + 1), mix32(h + 2), mix32(h + 3));
+    const uint2 k = make_uint2(mix32(h + 4), mix32(h + 5));
+    const uint4 a = philox4x32_10(c, k);
+    const uint4 r = curand_Philox4x32_10(c, k);
+    bad += (a.x != r.x) + (a.y != r.y) + (a.z != r.z) + (a.w != r.w);
+  }
+  if (bad) atomicAdd(counts, bad);
 }
 
 // ------------------------------------------------------------ SR
@@ -293,6 +312,12 @@ int fosck_div_tscale_bf16(float divisor, unsigned long long* counts, void* strea
 int fosck_div_tscale_random(unsigned long long seed, unsigned long long n, unsigned long long* counts,
                             void* stream) {
   k_div_tscale_random<<<kGrid, kThreads, 0, (cudaStream_t)stream>>>(seed, n, counts);
+  return launched(cudaSuccess);
+}
+
+int fosck_philox_vs_curand(unsigned long long seed, unsigned long long n, unsigned long long* counts,
+                           void* stream) {
+  k_philox_vs_curand<<<kGrid, kThreads, 0, (cudaStream_t)stream>>>(seed, n, counts);
   return launched(cudaSuccess);
 }
 

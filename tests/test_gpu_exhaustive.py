@@ -42,6 +42,7 @@ def _lib():
             "fosck_div_tscale_bf16": [f32, P, P],
             "fosck_div_tscale_random": [u64, u64, P, P],
             "fosck_sr_forms": [P, P],
+            "fosck_philox_vs_curand": [u64, u64, P, P],
             "fosck_sr_codes": [P, P, i64, i32, P, P],
             "fosck_transitions": [i32, P, u32, P, P],
             "fosck_codes_at": [P, i64, i32, P, P],
@@ -92,6 +93,14 @@ def test_div_tscale_random_binary32_pairs():
     c = _counts()
     _run("fosck_div_tscale_random", 12345, 1 << 30, _p(c))
     assert c.tolist() == [0, 0], "a/S_t shortcut: %d code mismatches, %d quotient mismatches" % tuple(c.tolist())
+
+
+def test_philox_equals_curand():
+    """The device Philox4x32-10 behind the SR bytes and the RHT signs equals
+    cuRAND's curand_Philox4x32_10 on 2^24 random (counter, key) pairs."""
+    c = _counts(1)
+    _run("fosck_philox_vs_curand", 2024, 1 << 24, _p(c))
+    assert c.item() == 0, "Philox differs from cuRAND in %d words" % c.item()
 
 
 def test_sr_integer_and_pair_forms_equal_float_form_everywhere():
