@@ -164,6 +164,54 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
                         void* workspace, size_t workspace_bytes, uint32_t* status,
                         void* stream);
 
+/*
+ * fos_quantize_host -- fos_quantize of a batch held in HOST memory, with the
+ * rowwise outputs returned to HOST memory, pipelined in chunks of `chunk`
+ * batch entries on three caller streams: the host-to-device copy of chunk
+ * k + 1 (stream_h2d), the quantization of chunk k (stream_compute, one
+ * fos_quantize per chunk) and the device-to-host copy of chunk k - 1
+ * (stream_d2h) overlap.  Each batch entry has its own S_t and the
+ * stochastic-rounding counters follow the global element index, so the
+ * results equal one fos_quantize over the whole batch.  (The copies are
+ * data movement around the method; the quantization is the method's.)
+ *
+ *   x_host        bf16 [batch][rows][cols], dense, in pinned host memory
+ *                 (pageable memory works, without overlap).
+ *   opt, amax_in  as fos_quantize; rowwise 1x16 (NVFP4) or 1x32 (MXFP4)
+ *                 blocks only, linear scale layout (no FOS_FLAG_SCALE_SWIZZLED,
+ *                 no RHT16_COL); amax_in: DEVICE [batch] or NULL.
+ *   out_host      HOST codes, scales and (NVFP4) tensor_scale with their row
+ *                 strides; choice_bits must be NULL.
+ *   x_dev         DEVICE staging input, bf16 [batch][rows][cols], 32-byte
+ *                 aligned (rows of every chunk stay 16-byte aligned).
+ *   out_dev       DEVICE outputs in the same layout as out_host (the same
+ *                 codes_ld and scales_ld); choice_bits must be NULL.
+ *   workspace     DEVICE, fos_workspace_size(chunk, rows, cols, opt) bytes;
+ *                 the chunks use it one after another on stream_compute.
+ *   status        DEVICE word or NULL, as fos_quantize.
+ *   chunk         batch entries per pipeline stage, >= 1.
+ *   streams       cudaStream_t stream_h2d, stream_compute, stream_d2h; the
+ *                 call orders the chunks between them with `events`.
+ *   events        2 * ceil(batch / chunk) cudaEvent_t created by the caller
+ *                 (cudaEventDisableTiming is enough), recorded by this call.
+ *
+ * Ownership: every buffer, stream and event belongs to the caller; nothing
+ * is allocated.  The call only enqueues work and returns: the first copy
+ * waits for nothing the caller does not order (make the three streams wait
+ * on earlier work first), and the outputs are in host memory once
+ * stream_d2h reaches the point where the call returned.  Errors:
+ * FOS_ERR_NULL, FOS_ERR_ARG (chunk < 1), FOS_ERR_UNSUPPORTED (colwise-only
+ * options, 2D blocks, swizzled scales, choice bits), then fos_quantize's own
+ * codes for the shape and options, all returned before anything is
+ * enqueued; FOS_ERR_CUDA when a copy, record or launch fails (earlier chunks
+ * may already be enqueued).
+ */
+fos_status fos_quantize_host(const void* x_host, int64_t batch, int64_t rows, int64_t cols,
+                             const fos_options* opt, const float* amax_in, const fos_qtensor* out_host,
+                             void* x_dev, const fos_qtensor* out_dev, void* workspace,
+                             size_t workspace_bytes, uint32_t* status, int64_t chunk, void* stream_h2d,
+                             void* stream_compute, void* stream_d2h, void* const* events);
+
 /* fos_amax -- per-batch-entry amax of |x| (of the 16-wide RHT of x when
  * opt->flags has FOS_FLAG_RHT16) into amax_out (device float [batch]).
  * NaN/Inf input sets FOS_STATUS_NONFINITE in *status.  Only opt->flags and

@@ -70,6 +70,13 @@ OutDesc make_out(const fos_qtensor* q, int64_t R, int64_t C, int64_t bs, uint32_
 
 size_t choice_bytes(int64_t nblocks) { return (size_t)(8 * ((nblocks + 63) / 64)); }
 
+// nr rows of `width` bytes, `ld` apart on both sides, device to host: one
+// plain copy when the rows are packed, else a pitched one.
+cudaError_t rows_d2h(void* dst, const void* src, int64_t ld, int64_t width, int64_t nr, cudaStream_t st) {
+  if (ld == width) return cudaMemcpyAsync(dst, src, (size_t)(width * nr), cudaMemcpyDeviceToHost, st);
+  return cudaMemcpy2DAsync(dst, (size_t)ld, src, (size_t)ld, (size_t)width, (size_t)nr, cudaMemcpyDeviceToHost, st);
+}
+
 // Test hooks: the fused kernel's bounded waits (fos_testing_quantize_stalled)
 // and the 2D kernel's strip length (fos_testing_quantize_2d_strip; 0 = the
 // per-launch choice).
@@ -77,6 +84,7 @@ struct WaitHooks {
   uint32_t spin_limit = 1u << 21;
   int stall_entry = -1;
   int strip_2d = 0;
+  bool validate_only = false;   // check the arguments, enqueue nothing
 };
 
 fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int64_t ld,
@@ -128,6 +136,77 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
                         void* stream) {
   return quantize_impl(x, batch, rows, cols, ld, opt, amax_in, rowwise, colwise, workspace,
                        workspace_bytes, status, stream, WaitHooks());
+}
+
+fos_status fos_quantize_host(const void* x_host, int64_t batch, int64_t rows, int64_t cols,
+                             const fos_options* opt, const float* amax_in, const fos_qtensor* out_host,
+                             void* x_dev, const fos_qtensor* out_dev, void* workspace,
+                             size_t workspace_bytes, uint32_t* status, int64_t chunk, void* stream_h2d,
+                             void* stream_compute, void* stream_d2h, void* const* events) {
+  if (!x_host || !opt || !out_host || !x_dev || !out_dev || !events) return FOS_ERR_NULL;
+  if (chunk < 1) return FOS_ERR_ARG;
+  if (opt->blk == FOS_BLOCK_16X16 || (opt->flags & (FOS_FLAG_SCALE_SWIZZLED | FOS_FLAG_RHT16_COL)) ||
+      out_host->choice_bits || out_dev->choice_bits)
+    return FOS_ERR_UNSUPPORTED;
+  const bool mx = opt->fmt == FOS_FMT_MXFP4;
+  if (!out_host->codes || !out_host->scales || (!mx && !out_host->tensor_scale)) return FOS_ERR_NULL;
+  if (out_host->codes_ld != out_dev->codes_ld || out_host->scales_ld != out_dev->scales_ld) return FOS_ERR_ARG;
+  if (!aligned(x_dev, 32)) return FOS_ERR_ALIGN;
+  // every chunk has the shape and options of the first (the last may hold
+  // fewer entries, which needs no more workspace): check them all up front
+  WaitHooks check;
+  check.validate_only = true;
+  fos_status e = quantize_impl(x_dev, batch < chunk ? batch : chunk, rows, cols, cols, opt, amax_in, out_dev,
+                               nullptr, workspace, workspace_bytes, status, stream_compute, check);
+  if (e != FOS_OK) return e;
+  cudaStream_t s_in = (cudaStream_t)stream_h2d, s_q = (cudaStream_t)stream_compute, s_out = (cudaStream_t)stream_d2h;
+  if (batch == 0) return FOS_OK;
+  if (rows == 0 || cols == 0) {   // empty entries: only S_t = 0 to deliver
+    for (int64_t c0 = 0; c0 < batch; c0 += chunk) {
+      const int64_t nb = batch - c0 < chunk ? batch - c0 : chunk;
+      fos_qtensor q = *out_dev;
+      if (!mx) q.tensor_scale += c0;
+      e = quantize_impl(x_dev, nb, rows, cols, cols, opt, nullptr, &q, nullptr, workspace, workspace_bytes,
+                        status, s_q, WaitHooks());
+      if (e != FOS_OK) return e;
+    }
+    if (!mx && (cudaEventRecord((cudaEvent_t)events[1], s_q) != cudaSuccess ||
+                cudaStreamWaitEvent(s_out, (cudaEvent_t)events[1], 0) != cudaSuccess ||
+                cudaMemcpyAsync(out_host->tensor_scale, out_dev->tensor_scale, 4 * batch, cudaMemcpyDeviceToHost,
+                                s_out) != cudaSuccess))
+      return FOS_ERR_CUDA;
+    return FOS_OK;
+  }
+  const int64_t per_entry = rows * cols;   // elements
+  const int64_t code_w = cols / 2, scale_w = cols / (mx ? 32 : 16);
+  for (int64_t c0 = 0, k = 0; c0 < batch; c0 += chunk, ++k) {
+    const int64_t nb = batch - c0 < chunk ? batch - c0 : chunk;
+    cudaEvent_t ev_in = (cudaEvent_t)events[2 * k], ev_q = (cudaEvent_t)events[2 * k + 1];
+    const size_t xoff = (size_t)(c0 * per_entry) * 2;
+    if (cudaMemcpyAsync((char*)x_dev + xoff, (const char*)x_host + xoff, (size_t)(nb * per_entry) * 2,
+                        cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(s_q, ev_in, 0) != cudaSuccess)
+      return FOS_ERR_CUDA;
+    fos_options o = *opt;
+    o.elem_offset = opt->elem_offset + c0 * per_entry;
+    fos_qtensor q = *out_dev;
+    q.codes += c0 * rows * q.codes_ld;
+    q.scales += c0 * rows * q.scales_ld;
+    if (!mx) q.tensor_scale += c0;
+    e = quantize_impl((char*)x_dev + xoff, nb, rows, cols, cols, &o, amax_in ? amax_in + c0 : nullptr, &q,
+                      nullptr, workspace, workspace_bytes, status, s_q, WaitHooks());
+    if (e != FOS_OK) return e;
+    if (cudaEventRecord(ev_q, s_q) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_q, 0) != cudaSuccess)
+      return FOS_ERR_CUDA;
+    const int64_t r0 = c0 * rows, nr = nb * rows;
+    if (rows_d2h(out_host->codes + r0 * out_host->codes_ld, q.codes, q.codes_ld, code_w, nr, s_out) != cudaSuccess ||
+        rows_d2h(out_host->scales + r0 * out_host->scales_ld, q.scales, q.scales_ld, scale_w, nr, s_out) !=
+            cudaSuccess ||
+        (!mx && cudaMemcpyAsync(out_host->tensor_scale + c0, q.tensor_scale, 4 * nb, cudaMemcpyDeviceToHost,
+                                s_out) != cudaSuccess))
+      return FOS_ERR_CUDA;
+  }
+  return FOS_OK;
 }
 
 fos_status fos_testing_quantize_stalled(const void* x, int64_t batch, int64_t rows, int64_t cols,
@@ -203,6 +282,7 @@ fos_status quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t col
     if (!aligned(workspace, 16)) return FOS_ERR_ALIGN;
   }
   if (amax_in && !aligned(amax_in, 4)) return FOS_ERR_ALIGN;
+  if (hooks.validate_only) return FOS_OK;
 
   cudaStream_t st = (cudaStream_t)stream;
   if (batch == 0) return FOS_OK;

@@ -35,7 +35,7 @@ ERRORS = {
 }
 
 # every symbol include/fos.h declares
-EXPORTS = ("fos_quantize", "fos_amax", "fos_dequantize", "fos_workspace_size",
+EXPORTS = ("fos_quantize", "fos_quantize_host", "fos_amax", "fos_dequantize", "fos_workspace_size",
            "fos_scales_size", "fos_status_string", "fos_version", "fos_quantize_static",
            "fos_testing_quantize_stalled", "fos_testing_quantize_2d_strip", "fos_fake_quantize",
            "fos_gemm_nvfp4")
@@ -76,6 +76,10 @@ def lib(path: str = LIB_PATH):
     L.fos_quantize.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P,
                                ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), P,
                                ctypes.c_size_t, P, P]
+    L.fos_quantize_host.restype = i32
+    L.fos_quantize_host.argtypes = [P, i64, i64, i64, ctypes.POINTER(Options), P, ctypes.POINTER(QTensorC), P,
+                                    ctypes.POINTER(QTensorC), P, ctypes.c_size_t, P, i64, P, P, P,
+                                    ctypes.POINTER(ctypes.c_void_p)]
     L.fos_quantize_static.restype = i32
     L.fos_quantize_static.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P,
                                       ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), P, P]

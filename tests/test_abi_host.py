@@ -112,6 +112,30 @@ def test_strip_hook_argument_errors(L):
                                            None, None, 0, None, 4, None) == 1
 
 
+def test_host_pipeline_argument_errors(L):
+    """fos_quantize_host checks its arguments before enqueueing anything."""
+    q = QTensorC(64, 128, 256, None, 16, 2)
+    ev = (ctypes.c_void_p * 2)(16, 32)
+
+    def call(x=16, opts=None, out_host=True, x_dev=32, chunk=1, events=True, qh=None):
+        o = opts or Options(0, 0, 0, 0, 0, 0)
+        return L.fos_quantize_host(ctypes.c_void_p(x) if x else None, 1, 16, 32, ctypes.byref(o), None,
+                                   ctypes.byref(qh or q) if out_host else None,
+                                   ctypes.c_void_p(x_dev) if x_dev else None, ctypes.byref(q),
+                                   ctypes.c_void_p(16), 1 << 16, None, chunk, None, None, None,
+                                   ev if events else None)
+    assert call(x=0) == 1
+    assert call(out_host=False) == 1
+    assert call(events=False) == 1
+    assert call(chunk=0) == 7
+    assert call(opts=Options(0, 1, 0, 0, 0, 0)) == 4                        # 16x16
+    assert call(opts=Options(0, 0, 0, 2, 0, 0)) == 4                        # swizzled scales
+    assert call(qh=QTensorC(64, 128, 256, 512, 16, 2)) == 4                 # choice bits
+    assert call(qh=QTensorC(64, 128, 256, None, 32, 2)) == 7                # host and device strides differ
+    assert call(x_dev=48) == 2                                              # staging not 32-byte aligned
+    assert call(opts=Options(3, 0, 0, 0, 0, 0)) == 7                        # bad format (fos_quantize's check)
+
+
 def test_library_has_no_oracle_dependency():
     """The product library must not link or name the CPU oracle."""
     src_dir = os.path.join(ROOT, "mxfp4_block_scaled_fos_b200")
