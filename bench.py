@@ -589,11 +589,11 @@ def run_rows(args, world, rank):
 
 
 def measure_e2e(args, world, x, row, ws, status, stream):
-    """Same metric through the public API with pinned host buffers: every
-    step copies the input in, quantizes it (per-expert amax + 4/6) and copies
-    codes, scales and S_t back, in chunks of 4 experts pipelined over three
-    streams (mxfp4_block_scaled_fos_b200.host.HostQuantizer), so that the
-    copies in both directions and the kernels overlap."""
+    """Same metric through the C-ABI call with pinned host buffers
+    (fos_quantize_host, bound as host.HostQuantizer): every step copies the
+    input in, quantizes it (per-expert amax + 4/6) and copies codes, scales
+    and S_t back, in chunks of 4 experts pipelined over three streams, so
+    that the copies in both directions and the kernels overlap."""
     from mxfp4_block_scaled_fos_b200.host import HostQuantizer
     batch, rows, cols = x.shape
     hq = HostQuantizer(batch, rows, cols, chunk=4, device=x.device)
