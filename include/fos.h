@@ -185,7 +185,9 @@ fos_status fos_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols
  *   x_dev         DEVICE staging input, bf16 [batch][rows][cols], 32-byte
  *                 aligned (rows of every chunk stay 16-byte aligned).
  *   out_dev       DEVICE outputs in the same layout as out_host (the same
- *                 codes_ld and scales_ld); choice_bits must be NULL.
+ *                 codes_ld and scales_ld); choice_bits must be NULL.  Each
+ *                 chunk's codes start chunk * rows * codes_ld bytes on and
+ *                 must stay 16-byte aligned (FOS_ERR_ALIGN otherwise).
  *   workspace     DEVICE, fos_workspace_size(chunk, rows, cols, opt) bytes;
  *                 the chunks use it one after another on stream_compute.
  *   status        DEVICE word or NULL, as fos_quantize.

@@ -152,6 +152,8 @@ fos_status fos_quantize_host(const void* x_host, int64_t batch, int64_t rows, in
   if (!out_host->codes || !out_host->scales || (!mx && !out_host->tensor_scale)) return FOS_ERR_NULL;
   if (out_host->codes_ld != out_dev->codes_ld || out_host->scales_ld != out_dev->scales_ld) return FOS_ERR_ARG;
   if (!aligned(x_dev, 32)) return FOS_ERR_ALIGN;
+  // later chunks start chunk * rows rows further: their codes stay 16-byte aligned
+  if (batch > chunk && (chunk * rows * out_dev->codes_ld) % 16 != 0) return FOS_ERR_ALIGN;
   // every chunk has the shape and options of the first (the last may hold
   // fewer entries, which needs no more workspace): check them all up front
   WaitHooks check;

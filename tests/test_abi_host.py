@@ -134,6 +134,12 @@ def test_host_pipeline_argument_errors(L):
     assert call(qh=QTensorC(64, 128, 256, None, 32, 2)) == 7                # host and device strides differ
     assert call(x_dev=48) == 2                                              # staging not 32-byte aligned
     assert call(opts=Options(3, 0, 0, 0, 0, 0)) == 7                        # bad format (fos_quantize's check)
+    # 3 rows of 8 code bytes per entry: the second chunk's codes would be 8-byte aligned
+    qo = QTensorC(64, 128, 256, None, 8, 1)
+    o = Options(0, 0, 0, 0, 0, 0)
+    assert L.fos_quantize_host(ctypes.c_void_p(16), 2, 3, 16, ctypes.byref(o), None, ctypes.byref(qo),
+                               ctypes.c_void_p(32), ctypes.byref(qo), ctypes.c_void_p(16), 1 << 16, None, 1,
+                               None, None, None, (ctypes.c_void_p * 4)(16, 32, 48, 64)) == 2
 
 
 def test_library_has_no_oracle_dependency():
