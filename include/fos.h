@@ -272,6 +272,23 @@ fos_status fos_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int64_t M,
                           void* d, int64_t ldd, int32_t out_dtype, uint32_t* status, void* stream);
 
 /*
+ * fos_gemm_nvfp4_ws -- fos_gemm_nvfp4 with a device workspace of
+ * fos_gemm_workspace_size(M, N, K) bytes (16-byte aligned; NULL gives
+ * fos_gemm_nvfp4).  The call first rewrites a's and b's swizzled scales into
+ * the workspace as copy sources of the tensor core's 128 x 256-bit scale
+ * copy (each 16-byte atom row four times; 4x the scale bytes), then runs the
+ * product with 6 scale copies per 256-wide K step instead of 12 (4 instead
+ * of 8 for 128 x 128 tiles).  Same result as fos_gemm_nvfp4, bit for bit; the
+ * workspace is only read by this call's kernels and may be reused once the
+ * stream has passed them.  Errors: those of fos_gemm_nvfp4, and
+ * FOS_ERR_WORKSPACE / FOS_ERR_ALIGN for a small or misaligned workspace.
+ */
+size_t fos_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+fos_status fos_gemm_nvfp4_ws(const fos_qtensor* a, const fos_qtensor* b, int64_t M, int64_t N, int64_t K,
+                             void* d, int64_t ldd, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                             uint32_t* status, void* stream);
+
+/*
  * fos_quantize_static -- fos_quantize without a workspace argument, for
  * callers that cannot allocate device memory: code that runs inside a stream
  * capture (cudaMalloc cannot be captured), serving paths that must not

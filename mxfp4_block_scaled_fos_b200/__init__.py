@@ -7,7 +7,8 @@ ctypes binding that passes torch device buffers and the current stream to it;
 """
 from .fos import (  # noqa: F401
     FLAG_RHT16, FLAG_RHT16_COL, FLAG_SCALE_SWIZZLED, STATUS_NONFINITE, STATUS_TIMEOUT, FosError, Options,
-    QTensor, amax, dequantize, fake_quantize, gemm_nvfp4, lib, quantize, scales_size, status_string, version,
+    QTensor, amax, dequantize, fake_quantize, gemm_nvfp4, gemm_workspace_size, lib, quantize, scales_size,
+    status_string, version,
     workspace_size,
 )
 from .host import HostQuantizer  # noqa: F401

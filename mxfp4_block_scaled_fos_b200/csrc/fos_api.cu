@@ -481,6 +481,17 @@ fos_status fos_fake_quantize(const void* x, int64_t batch, int64_t rows, int64_t
 
 fos_status fos_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int64_t M, int64_t N, int64_t K,
                           void* d, int64_t ldd, int32_t out_dtype, uint32_t* status, void* stream) {
+  return fos_gemm_nvfp4_ws(a, b, M, N, K, d, ldd, out_dtype, nullptr, 0, status, stream);
+}
+
+size_t fos_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return gemm_workspace_bytes(M, N, K);
+}
+
+fos_status fos_gemm_nvfp4_ws(const fos_qtensor* a, const fos_qtensor* b, int64_t M, int64_t N, int64_t K,
+                             void* d, int64_t ldd, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                             uint32_t* status, void* stream) {
   if (!a || !b || !d) return FOS_ERR_NULL;
   if (!a->codes || !a->scales || !a->tensor_scale || !b->codes || !b->scales || !b->tensor_scale)
     return FOS_ERR_NULL;
@@ -494,6 +505,10 @@ fos_status fos_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int64_t M,
     return FOS_ERR_ALIGN;
   if (a->codes_ld < K / 2 || b->codes_ld < K / 2) return FOS_ERR_SHAPE;
   if (a->codes_ld % 16 || b->codes_ld % 16 || ldd % (out_dtype ? 4 : 8)) return FOS_ERR_ALIGN;
+  if (workspace) {
+    if (workspace_bytes < gemm_workspace_bytes(M, N, K)) return FOS_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return FOS_ERR_ALIGN;
+  }
   if (M == 0 || N == 0) return FOS_OK;
   if (K == 0) {
     const size_t es = out_dtype ? 4 : 2;
@@ -501,7 +516,7 @@ fos_status fos_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int64_t M,
                ? FOS_OK : FOS_ERR_CUDA;
   }
   const cudaError_t e = launch_gemm_nvfp4(a, b, (int)M, (int)N, (int)K, d, ldd, out_dtype, status,
-                                          (cudaStream_t)stream);
+                                          (cudaStream_t)stream, workspace);
   if (e == cudaErrorNotSupported) return FOS_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FOS_OK : FOS_ERR_CUDA;
 }

@@ -51,6 +51,7 @@ namespace {
 constexpr int BM = 128, BK = 256;                // BK in FP4 elements (128 bytes)
 constexpr int kTileA = BM * BK / 2;              // 16384 bytes
 constexpr int kSFRowTile = 2048;                 // one 128-row tile's 4 scale atoms per K step
+constexpr int kSFImage = 4096;                   // one 128 x 256-bit scale copy source (wide layout)
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kGroupM = 8;                       // tile rows per group of the tile order
@@ -61,12 +62,17 @@ constexpr uint32_t kWaitLimit = 1u << 22;        // polls of one mbarrier wait
 // (measured: an N = 256 MMA takes as long as an N = 128 one here), at the
 // price of one accumulator buffer instead of two: 256 tensor-memory columns
 // of accumulator leave room only for the scale buffers.
-template <int BN>
+//
+// WIDE: the scales come as copy-source images of the 128 x 256-bit
+// tensor-memory copy (k_expand_sf): 6 copies per K step at BN = 256 instead
+// of 12 of 32 x 128 bits, for 4 times the scale bytes in shared memory.
+template <int BN, bool WIDE = false>
 struct Cfg {
-  static constexpr int kStages = BN == 128 ? 6 : 4;
+  static constexpr int kStages = WIDE ? (BN == 128 ? 4 : 3) : (BN == 128 ? 6 : 4);
   static constexpr int kTileB = BN * BK / 2;
-  static constexpr int kSFB = (BN / 128) * kSFRowTile;   // B scales per stage
-  static constexpr uint32_t kStageTx = kTileA + kTileB + kSFRowTile + kSFB;
+  static constexpr int kSFA = WIDE ? 2 * kSFImage : kSFRowTile;                    // A scales per stage
+  static constexpr int kSFB = (BN / 128) * (WIDE ? 2 * kSFImage : kSFRowTile);     // B scales per stage
+  static constexpr uint32_t kStageTx = kTileA + kTileB + kSFA + kSFB;
   static constexpr int kAcc = BN == 128 ? 2 : 1;         // accumulator buffers (kAcc * BN <= 256 columns)
   // tensor memory: accumulators from column 0; A scales 256 + 16 * (k step &
   // 1) (4 columns per K-64 group); B scales 288 + (BN / 8) * (k step & 1)
@@ -77,7 +83,7 @@ struct Cfg {
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kTileA;
   static constexpr int kOffSFA = kOffB + kStages * kTileB;
-  static constexpr int kOffSFB = kOffSFA + kStages * kSFRowTile;
+  static constexpr int kOffSFB = kOffSFA + kStages * kSFA;
   static constexpr int kOffBar = kOffSFB + kStages * kSFB;  // full[S], empty[S], acc_full[2], acc_empty[2]
   static constexpr int kOffTmem = kOffBar + (2 * kStages + 4) * 8;
   static constexpr int kOffFlag = kOffTmem + 8;
@@ -134,6 +140,14 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// Descriptor of one 4 KB wide copy source (128 rows of 32 bytes, no
+// swizzle): the two 16-byte core-matrix columns of an 8-row group 128 bytes
+// apart, 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf_wide(uint32_t addr) {
+  return (uint64_t)((addr & 0x3FFFF) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(256 >> 4) << 32) |
+         ((uint64_t)1 << 46);
+}
+
 // Descriptor of one 512-byte scale atom (32 rows of 16 bytes, no swizzle,
 // 8-row groups 128 bytes apart) as the source of tcgen05.cp.
 __device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
@@ -152,6 +166,11 @@ __device__ __forceinline__ void umma(uint32_t tmem_c, uint64_t da, uint64_t db, 
 
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+
+// 128 lanes x 32 bytes from a wide copy source: lane l gets its row l.
+__device__ __forceinline__ void tmem_cp_sf_wide(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
@@ -183,11 +202,11 @@ __device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int& tm, in
   tn = r / gm;
 }
 
-template <int BN>
+template <int BN, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_nvfp4(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const GemmArgs g) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, WIDE>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -236,13 +255,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(fb, C::kStageTx);
           tma_load_2d(sbase + C::kOffA + s * kTileA, &map_a, kt * (BK / 2), tm * BM, fb);
           tma_load_2d(sbase + C::kOffB + s * C::kTileB, &map_b, kt * (BK / 2), tn * BN, fb);
-          // the 4 scale atoms of each 128-row tile, scale columns [16 kt, +16)
-          bulk_load(sbase + C::kOffSFA + s * kSFRowTile, g.sfa + ((long long)tm * g.sf_col_tiles + 4 * kt) * 512,
-                    kSFRowTile, fb);
+          if (WIDE) {
+            // the K step's copy sources: A's of tile row tm, B's of tile column tn
+            bulk_load(sbase + C::kOffSFA + s * C::kSFA, g.sfa + ((long long)tm * ksteps + kt) * C::kSFA, C::kSFA,
+                      fb);
+            bulk_load(sbase + C::kOffSFB + s * C::kSFB, g.sfb + ((long long)tn * ksteps + kt) * C::kSFB, C::kSFB,
+                      fb);
+          } else {
+            // the 4 scale atoms of each 128-row tile, scale columns [16 kt, +16)
+            bulk_load(sbase + C::kOffSFA + s * kSFRowTile, g.sfa + ((long long)tm * g.sf_col_tiles + 4 * kt) * 512,
+                      kSFRowTile, fb);
 #pragma unroll
-          for (int h = 0; h < BN / 128; ++h)
-            bulk_load(sbase + C::kOffSFB + s * C::kSFB + h * kSFRowTile,
-                      g.sfb + ((long long)(tn * (BN / 128) + h) * g.sf_col_tiles + 4 * kt) * 512, kSFRowTile, fb);
+            for (int h = 0; h < BN / 128; ++h)
+              bulk_load(sbase + C::kOffSFB + s * C::kSFB + h * kSFRowTile,
+                        g.sfb + ((long long)(tn * (BN / 128) + h) * g.sf_col_tiles + 4 * kt) * 512, kSFRowTile,
+                        fb);
+          }
         }
       }
       // before leaving, every copy this thread started must have landed
@@ -264,15 +292,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
           const uint32_t sfa = tmem + C::kColSFA + 16u * (it & 1);
           const uint32_t sfb = tmem + C::kColSFB + 4u * C::kSFBGroup * (it & 1);
-          // scale atom j of each 128-row tile h -> 4 columns (K-64 group j);
-          // B's groups hold BN / 32 columns, its row tiles 4 columns apart
+          if (WIDE) {
+            // a source holds two atoms side by side -> 8 columns: A's K-64
+            // groups (0, 1) and (2, 3); B likewise at BN = 128, and at
+            // BN = 256 group j of both 128-row tiles (columns 8 j .. 8 j + 7)
+            const uint32_t src_a = sbase + C::kOffSFA + s * C::kSFA, src_b = sbase + C::kOffSFB + s * C::kSFB;
+            tmem_cp_sf_wide(sfa, desc_sf_wide(src_a));
+            tmem_cp_sf_wide(sfa + 8, desc_sf_wide(src_a + kSFImage));
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_sf(sfa + 4 * j, desc_sf(sbase + C::kOffSFA + s * kSFRowTile + 512 * j));
+            for (int c = 0; c < C::kSFB / kSFImage; ++c)
+              tmem_cp_sf_wide(sfb + 8 * c, desc_sf_wide(src_b + c * kSFImage));
+          } else {
+            // scale atom j of each 128-row tile h -> 4 columns (K-64 group j);
+            // B's groups hold BN / 32 columns, its row tiles 4 columns apart
 #pragma unroll
-            for (int h = 0; h < BN / 128; ++h)
-              tmem_cp_sf(sfb + C::kSFBGroup * j + 4 * h,
-                         desc_sf(sbase + C::kOffSFB + s * C::kSFB + h * kSFRowTile + 512 * j));
+            for (int j = 0; j < 4; ++j) {
+              tmem_cp_sf(sfa + 4 * j, desc_sf(sbase + C::kOffSFA + s * kSFRowTile + 512 * j));
+#pragma unroll
+              for (int h = 0; h < BN / 128; ++h)
+                tmem_cp_sf(sfb + C::kSFBGroup * j + 4 * h,
+                           desc_sf(sbase + C::kOffSFB + s * C::kSFB + h * kSFRowTile + 512 * j));
+            }
           }
           const uint64_t da = desc_sw128(sbase + C::kOffA + s * kTileA);
           const uint64_t db = desc_sw128(sbase + C::kOffB + s * C::kTileB);
@@ -353,6 +393,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *fail && g.status) atomicOr(g.status, FOS_STATUS_TIMEOUT);
 }
 
+// The wide layout's copy sources from the swizzled scales (512-byte atoms
+// of 128 rows x 4 scales, atom (t, c) at (t * col_tiles + c) * 512; row r of
+// an atom holds the scales of rows r, r + 32, r + 64, r + 96).  A source is
+// 4 KB: row l (32 bytes at (l >> 3) * 256 + (l & 7) * 16, second half 128
+// bytes on) is row l % 32 of two atoms.  pair_tiles = 0: source (t, kt, s)
+// pairs atoms (t, 4 kt + 2 s) and (t, 4 kt + 2 s + 1); pair_tiles = 1:
+// source (p, kt, j) pairs atoms (2 p, 4 kt + j) and (2 p + 1, 4 kt + j).
+// One thread per 16 bytes of the output, in output order.
+__global__ void __launch_bounds__(256) k_expand_sf(const uint8_t* src, long long col_tiles, long long ksteps,
+                                                   unsigned long long nimages, int pair_tiles, uint8_t* dst) {
+  const unsigned long long nchunks = nimages * 256ull;
+  for (unsigned long long q = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x; q < nchunks;
+       q += (unsigned long long)gridDim.x * blockDim.x) {
+    const unsigned long long img = q >> 8;
+    const int w = (int)(q & 255);
+    const int half = (w >> 3) & 1, l = ((w >> 4) << 3) | (w & 7);
+    long long tile, ctile;
+    if (!pair_tiles) {
+      const long long r = (long long)(img >> 1), kt = r % ksteps;
+      tile = r / ksteps;
+      ctile = 4 * kt + 2 * (long long)(img & 1) + half;
+    } else {
+      const long long r = (long long)(img >> 2), kt = r % ksteps;
+      tile = 2 * (r / ksteps) + half;
+      ctile = 4 * kt + (long long)(img & 3);
+    }
+    *reinterpret_cast<uint4*>(dst + q * 16) =
+        *reinterpret_cast<const uint4*>(src + (tile * col_tiles + ctile) * 512 + (l & 31) * 16);
+  }
+}
+
 // ---------------------------------------------------------------- host
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -386,7 +457,7 @@ bool make_code_map(CUtensorMap* m, const void* codes, long long rows, long long 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN>
+template <int BN, bool WIDE = false>
 cudaError_t launch_bn(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, const GemmArgs& g,
                       cudaStream_t st) {
   CUtensorMap ma, mb;
@@ -396,8 +467,8 @@ cudaError_t launch_bn(const fos_qtensor* a, const fos_qtensor* b, int M, int N, 
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(k_gemm_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    Cfg<BN>::kSmemBytes);
+    attr_err = cudaFuncSetAttribute(k_gemm_nvfp4<BN, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg<BN, WIDE>::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   int dev = 0, sms = 0;
@@ -405,15 +476,29 @@ cudaError_t launch_bn(const fos_qtensor* a, const fos_qtensor* b, int M, int N, 
       cudaSuccess)
     return cudaErrorNotSupported;
   const int ntiles = (M / BM) * (N / BN);
-  k_gemm_nvfp4<BN><<<dim3(ntiles < sms ? ntiles : sms), kThreads, Cfg<BN>::kSmemBytes, st>>>(ma, mb, g);
+  k_gemm_nvfp4<BN, WIDE><<<dim3(ntiles < sms ? ntiles : sms), kThreads, Cfg<BN, WIDE>::kSmemBytes, st>>>(ma, mb, g);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t gemm_workspace_bytes(long long M, long long N, long long K) {
+  return (size_t)4 * 512 * (size_t)((M / 128) * (K / 64) + (N / 128) * (K / 64));
+}
+
+static cudaError_t expand_sf(const uint8_t* src, long long rows, int K, int pair_tiles, uint8_t* dst,
+                             cudaStream_t st) {
+  const long long col_tiles = K / 64, ksteps = K / 256;
+  const unsigned long long nimages = (unsigned long long)(rows / 128) * ksteps * 2;
+  const unsigned long long blocks = (nimages * 256 + 255) / 256;
+  k_expand_sf<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(src, col_tiles, ksteps, nimages,
+                                                                               pair_tiles, dst);
+  return cudaGetLastError();
+}
+
 // 128 x 256 tiles when N allows them, else 128 x 128.
 cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, void* d,
-                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st) {
+                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st, void* workspace) {
   GemmArgs g;
   g.sfa = a->scales;
   g.sfb = b->scales;
@@ -427,7 +512,18 @@ cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M,
   g.f32_out = f32_out;
   g.sf_col_tiles = K / 64;
   g.status = status;
-  return N % 256 == 0 ? launch_bn<256>(a, b, M, N, K, g, st) : launch_bn<128>(a, b, M, N, K, g, st);
+  const bool bn256 = N % 256 == 0;
+  if (workspace) {  // the wide layout: expand both operands' scales, then 6 or 4 copies per K step
+    uint8_t* ea = static_cast<uint8_t*>(workspace);
+    uint8_t* eb = ea + gemm_workspace_bytes(M, 0, K);
+    cudaError_t e = expand_sf(a->scales, M, K, 0, ea, st);
+    if (e == cudaSuccess) e = expand_sf(b->scales, N, K, bn256 ? 1 : 0, eb, st);
+    if (e != cudaSuccess) return e;
+    g.sfa = ea;
+    g.sfb = eb;
+    return bn256 ? launch_bn<256, true>(a, b, M, N, K, g, st) : launch_bn<128, true>(a, b, M, N, K, g, st);
+  }
+  return bn256 ? launch_bn<256>(a, b, M, N, K, g, st) : launch_bn<128>(a, b, M, N, K, g, st);
 }
 
 }  // namespace fos

@@ -76,8 +76,12 @@ cudaError_t launch_fake_mx(const QuantArgs& a, int batch, cudaStream_t st);
 
 // NVFP4 block-scaled GEMM on the tensor cores (fos_gemm.cu); shapes checked
 // by the caller (M, N multiples of 128, K of 256).
+// workspace (nullable): gemm_workspace_bytes(M, N, K) bytes for the wide
+// scale layout (expanded from a's and b's swizzled scales in the call)
 cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M, int N, int K, void* d,
-                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st);
+                              long long ldd, int f32_out, uint32_t* status, cudaStream_t st,
+                              void* workspace = nullptr);
+size_t gemm_workspace_bytes(long long M, long long N, long long K);
 
 // Workspace bytes of fos_quantize for `batch` entries: per-entry amax words,
 // per-entry completion counters and the fused kernel's queue counter.

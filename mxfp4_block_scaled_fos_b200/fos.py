@@ -38,7 +38,7 @@ ERRORS = {
 EXPORTS = ("fos_quantize", "fos_quantize_host", "fos_amax", "fos_dequantize", "fos_workspace_size",
            "fos_scales_size", "fos_status_string", "fos_version", "fos_quantize_static",
            "fos_testing_quantize_stalled", "fos_testing_quantize_2d_strip", "fos_fake_quantize",
-           "fos_gemm_nvfp4")
+           "fos_gemm_nvfp4", "fos_gemm_nvfp4_ws", "fos_gemm_workspace_size")
 
 
 class Options(ctypes.Structure):
@@ -94,6 +94,11 @@ def lib(path: str = LIB_PATH):
     L.fos_fake_quantize.restype = i32
     L.fos_fake_quantize.argtypes = [P, i64, i64, i64, i64, ctypes.POINTER(Options), P, P, i64, P,
                                     ctypes.c_size_t, P, P]
+    L.fos_gemm_nvfp4_ws.restype = i32
+    L.fos_gemm_nvfp4_ws.argtypes = [ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), i64, i64, i64, P, i64,
+                                    i32, P, ctypes.c_size_t, P, P]
+    L.fos_gemm_workspace_size.restype = ctypes.c_size_t
+    L.fos_gemm_workspace_size.argtypes = [i64, i64, i64]
     L.fos_gemm_nvfp4.restype = i32
     L.fos_gemm_nvfp4.argtypes = [ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), i64, i64, i64, P, i64,
                                  i32, P, P]
@@ -285,9 +290,13 @@ def dequantize(q: QTensor, out: Optional[torch.Tensor] = None, stream=None) -> t
 
 
 def gemm_nvfp4(a: QTensor, b: QTensor, out: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16,
-               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+               status: Optional[torch.Tensor] = None, stream=None, wide: bool = True,
+               workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """D = (S_tA * S_tB) * A @ B^T on the tensor cores, for rowwise NVFP4
-    quantizations A [M, K] and B [N, K] with swizzled scales (batch 1)."""
+    quantizations A [M, K] and B [N, K] with swizzled scales (batch 1).
+    wide: the scales are first rewritten into `workspace` (allocated here when
+    None) for the wider tensor-memory scale copy (fos_gemm_nvfp4_ws); False
+    runs fos_gemm_nvfp4 without a workspace.  Same result either way."""
     if not (a.flags & FLAG_SCALE_SWIZZLED and b.flags & FLAG_SCALE_SWIZZLED):
         raise ValueError("gemm_nvfp4 needs scales in the swizzled tensor-core layout")
     if a.fmt == "mxfp4" or b.fmt == "mxfp4" or a.batch != 1 or b.batch != 1 or a.cols != b.cols:
@@ -298,12 +307,22 @@ def gemm_nvfp4(a: QTensor, b: QTensor, out: Optional[torch.Tensor] = None, out_d
     if out.dtype not in (torch.bfloat16, torch.float32) or out.stride(-1) != 1:
         raise ValueError("out must be a row-contiguous bf16 or f32 tensor")
     ac, bc = a.c_struct(), b.c_struct()
-    st = lib().fos_gemm_nvfp4(ctypes.byref(ac), ctypes.byref(bc), M, N, K, ctypes.c_void_p(out.data_ptr()),
-                              out.stride(0), 1 if out.dtype == torch.float32 else 0, _ptr(status),
-                              _stream(stream))
+    if wide and workspace is None:
+        workspace = torch.empty(gemm_workspace_size(M, N, K), dtype=torch.uint8, device=a.codes.device)
+    if not wide:
+        workspace = None
+    st = lib().fos_gemm_nvfp4_ws(ctypes.byref(ac), ctypes.byref(bc), M, N, K, ctypes.c_void_p(out.data_ptr()),
+                                 out.stride(0), 1 if out.dtype == torch.float32 else 0, _ptr(workspace),
+                                 workspace.numel() if workspace is not None else 0, _ptr(status),
+                                 _stream(stream))
     if st != 0:
-        raise FosError(st, "fos_gemm_nvfp4")
+        raise FosError(st, "fos_gemm_nvfp4_ws" if wide else "fos_gemm_nvfp4")
     return out
+
+
+def gemm_workspace_size(M: int, N: int, K: int) -> int:
+    """Bytes of workspace gemm_nvfp4(wide=True) needs."""
+    return int(lib().fos_gemm_workspace_size(M, N, K))
 
 
 def status_string(code: int) -> str:

@@ -49,12 +49,13 @@ def _operand(rows, K, seed, dev, fmt):
 @pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 512), (384, 256, 1024), (128, 512, 2304)])
 @pytest.mark.parametrize("fmt", ["nvfp4_46", "nvfp4_6"])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_gemm_matches_fp64_reference(M, N, K, fmt, out_dtype):
+@pytest.mark.parametrize("wide", [True, False])
+def test_gemm_matches_fp64_reference(M, N, K, fmt, out_dtype, wide):
     dev = require_gpu()
     xa, qa = _operand(M, K, M + 3 * K, dev, fmt)
     xb, qb = _operand(N, K, N + 7 * K + 1, dev, fmt)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    d = F.gemm_nvfp4(qa, qb, out_dtype=out_dtype, status=status)
+    d = F.gemm_nvfp4(qa, qb, out_dtype=out_dtype, status=status, wide=wide)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     fo = oracle.FMT_NVFP4_46 if fmt == "nvfp4_46" else oracle.FMT_NVFP4_6
@@ -71,6 +72,24 @@ def test_gemm_matches_fp64_reference(M, N, K, fmt, out_dtype):
     bad = np.argwhere(err > bound)
     assert bad.size == 0, "GEMM differs at %s: got %r ref %r bound %r" % (
         bad[:3].tolist(), got[tuple(bad[0])], ref[tuple(bad[0])], bound[tuple(bad[0])])
+
+
+@pytest.mark.parametrize("M,N,K", [(1024, 1024, 2048), (512, 896, 1280)])
+def test_wide_scale_layout_gives_the_same_bits(M, N, K):
+    """The workspace path (scales rewritten for the 128 x 256-bit tensor-memory
+    copy) feeds the same scales to the same MMAs in the same order as the
+    plain path: the outputs are equal bit for bit, on 128 x 256 tiles
+    (N % 256 == 0) and on 128 x 128 tiles."""
+    dev = require_gpu()
+    _, qa = _operand(M, K, 5, dev, "nvfp4_46")
+    _, qb = _operand(N, K, 6, dev, "nvfp4_46")
+    d_wide = F.gemm_nvfp4(qa, qb, out_dtype=torch.float32, wide=True)
+    d_plain = F.gemm_nvfp4(qa, qb, out_dtype=torch.float32, wide=False)
+    torch.cuda.synchronize()
+    assert torch.equal(d_wide.view(torch.int32), d_plain.view(torch.int32))
+    ws = torch.empty(F.gemm_workspace_size(M, N, K) - 16, dtype=torch.uint8, device=dev)
+    with pytest.raises(F.FosError):
+        F.gemm_nvfp4(qa, qb, workspace=ws)   # one 16-byte chunk short
 
 
 def test_gemm_rejects_bad_shapes():
