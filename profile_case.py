@@ -93,7 +93,8 @@ def main():
         qa = F.quantize(xa, swizzle=True, choice=False)[0]
         qb = F.quantize(xb, swizzle=True, choice=False)[0]
         d = torch.empty(n, n, dtype=torch.bfloat16, device=dev)
-        fn = lambda: F.gemm_nvfp4(qa, qb, out=d)
+        ws = torch.empty(F.gemm_workspace_size(n, n, n), dtype=torch.uint8, device=dev)
+        fn = lambda: F.gemm_nvfp4(qa, qb, out=d, workspace=ws)
     else:
         raise SystemExit("unknown case " + c)
     fn()
