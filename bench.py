@@ -532,8 +532,8 @@ def measure_modes(args, world, x, dev, stream, peak):
         qw = F.quantize_weight(wl)
 
         def layer_step():
-            F.linear_forward(xl, qw)
-            F.linear_backward(dyl, xl, qw, seed=7)
+            _, qx_t = F.linear_forward(xl, qw, save_colwise=True, seed=7)
+            F.linear_backward(dyl, None, qw, seed=7, qx_t=qx_t)
 
         ms = time_loop(layer_step, n, 3, world, stream) / n
         tf = 3 * 2.0 * M_ * N_ * K_ / (ms * 1e-3) / 1e12
@@ -541,8 +541,8 @@ def measure_modes(args, world, x, dev, stream, peak):
                                        "frac": round(tf / peak_tf, 4), "peak_TFLOP_s": peak_tf,
                                        "peak_source": peak_src, "shape": [M_, N_, K_],
                                        "note": "3 GEMMs (forward, dgrad, wgrad) + the quantization of "
-                                               "x (both orientations) and dy (SR, both orientations) per "
-                                               "step; f32 gradients, bf16 y"}
+                                               "x (both orientations, from one read in the forward) and dy "
+                                               "(SR, both orientations) per step; f32 gradients, bf16 y"}
         del xl, wl, dyl, qw
     except Exception as e:
         res["linear_error"] = repr(e)

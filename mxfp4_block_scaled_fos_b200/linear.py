@@ -69,31 +69,51 @@ def quantize_weight(w: torch.Tensor, fmt: str = "nvfp4_46", stream=None) -> Quan
 
 
 def linear_forward(x: torch.Tensor, qw: QuantizedWeight, fmt: str = "nvfp4_46",
-                   out: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
-    """y [M, N] = x [M, K] @ W^T with x quantized 1x16 along K (RNE)."""
+                   out: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16, save_colwise: bool = False,
+                   rht: bool = False, seed: int = 0, stream=None):
+    """y [M, N] = x [M, K] @ W^T with x quantized 1x16 along K (RNE).
+
+    save_colwise: also quantize x^T along M (the wgrad operand) from the same
+    read of x, and return (y, qx_t) for linear_backward(..., qx_t=qx_t); with
+    rht the colwise copy is transformed along M with the signs of `seed` (pass
+    the backward's seed).  The rowwise copy is the same either way."""
     if x.dim() != 2 or x.shape[1] != qw.shape[1]:
         raise ValueError("x must be [M, K] with the weight's K")
     _check("M", x.shape[0], 256)
+    if save_colwise:
+        qx, qx_t = fos.quantize(x, fmt=fmt, swizzle=True, colwise=True, choice=False, rht_col=rht, seed=seed,
+                                stream=stream)
+        return fos.gemm_nvfp4(qx, qw.row, out=out, out_dtype=out_dtype, stream=stream), qx_t
     qx = fos.quantize(x, fmt=fmt, swizzle=True, choice=False, stream=stream)[0]
     return fos.gemm_nvfp4(qx, qw.row, out=out, out_dtype=out_dtype, stream=stream)
 
 
-def linear_backward(dy: torch.Tensor, x: torch.Tensor, qw: QuantizedWeight, seed: int = 0,
+def linear_backward(dy: torch.Tensor, x: Optional[torch.Tensor], qw: QuantizedWeight, seed: int = 0,
                     elem_offset: int = 0, fmt: str = "nvfp4_46", out_dtype=torch.float32,
-                    rht: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                    rht: bool = False, qx_t: Optional[fos.QTensor] = None,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """(dx [M, K], dW [N, K]) from dy [M, N], the forward input x [M, K] and
     the quantized weight.  dy is quantized once, in both orientations, with
     stochastic rounding keyed on (seed, elem_offset + element index).  rht:
     the wgrad operands (dy^T, x^T) are transformed along M with the signs of
-    the same key (seed), each with its own S_t."""
+    the same key (seed), each with its own S_t.  qx_t: x^T as saved by
+    linear_forward(save_colwise=True) with the same rht and seed; x is then
+    not read (and may be None)."""
     N, K = qw.shape
-    if dy.dim() != 2 or x.dim() != 2 or dy.shape[1] != N or x.shape[1] != K or dy.shape[0] != x.shape[0]:
-        raise ValueError("dy must be [M, N] and x [M, K] for a weight [N, K]")
-    _check("M", dy.shape[0], 256)
+    M = dy.shape[0] if dy.dim() == 2 else -1
+    if dy.dim() != 2 or dy.shape[1] != N:
+        raise ValueError("dy must be [M, N] for a weight [N, K]")
+    if qx_t is None:
+        if x is None or x.dim() != 2 or x.shape[1] != K or x.shape[0] != M:
+            raise ValueError("x must be [M, K] for dy [M, N] and a weight [N, K]")
+    elif qx_t.rows != K or qx_t.cols != M or qx_t.batch != 1:
+        raise ValueError("qx_t must be the colwise copy of an [M, K] input")
+    _check("M", M, 256)
     qdy, qdy_t = fos.quantize(dy, fmt=fmt, rounding="sr", seed=seed, elem_offset=elem_offset, swizzle=True,
                               colwise=True, choice=False, rht_col=rht, stream=stream)
-    qx_t = fos.quantize(x, fmt=fmt, swizzle=True, rowwise=False, colwise=True, choice=False, rht_col=rht,
-                        seed=seed, stream=stream)[1]
+    if qx_t is None:
+        qx_t = fos.quantize(x, fmt=fmt, swizzle=True, rowwise=False, colwise=True, choice=False, rht_col=rht,
+                            seed=seed, stream=stream)[1]
     dx = fos.gemm_nvfp4(qdy, qw.col, out_dtype=out_dtype, stream=stream)
     dw = fos.gemm_nvfp4(qdy_t, qx_t, out_dtype=out_dtype, stream=stream)
     return dx, dw

@@ -93,6 +93,27 @@ def test_linear_forward_and_backward_match_oracle_operands(M, N, K, rht):
     _check(dw, *_ref(gt_v, st_gt, xt_v, st_xt), "wgrad dW")
 
 
+@pytest.mark.parametrize("rht", [False, True])
+def test_saved_colwise_copy_gives_the_same_layer(rht):
+    """linear_forward(save_colwise=True) makes x^T's copy from the forward's
+    read of x (the two-orientation kernel); the forward output and the
+    backward's dx and dW equal those of the path that quantizes x again in
+    the backward, bit for bit."""
+    dev = require_gpu()
+    M, N, K, seed = 512, 256, 768, 77
+    x, w, dy = _inputs(M, N, K, dev, 9)
+    qw = F.quantize_weight(w)
+    y0 = F.linear_forward(x, qw, out_dtype=torch.float32)
+    dx0, dw0 = F.linear_backward(dy, x, qw, seed=seed, rht=rht)
+    y1, qx_t = F.linear_forward(x, qw, out_dtype=torch.float32, save_colwise=True, rht=rht, seed=seed)
+    dx1, dw1 = F.linear_backward(dy, None, qw, seed=seed, rht=rht, qx_t=qx_t)
+    torch.cuda.synchronize()
+    for a, b in ((y0, y1), (dx0, dx1), (dw0, dw1)):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    with pytest.raises(ValueError):
+        F.linear_backward(dy[:256].contiguous(), None, qw, seed=seed, qx_t=qx_t)   # M differs
+
+
 def test_linear_shape_errors():
     dev = require_gpu()
     x, w, dy = _inputs(256, 256, 256, dev, 5)
