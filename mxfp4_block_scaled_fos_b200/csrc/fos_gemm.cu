@@ -173,6 +173,13 @@ __device__ __forceinline__ void tmem_cp_sf_wide(uint32_t taddr, uint64_t sdesc) 
   asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
 }
 
+// 32 bytes to global memory in one store; p 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t a4, uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               :: "l"(p), "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7) : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
 }
@@ -186,6 +193,7 @@ struct GemmArgs {
   long long ldd;       // elements
   int M, N, K;
   int f32_out;
+  int wide_st;         // rows of d 32-byte aligned: 256-bit stores
   long long sf_col_tiles;  // K / 64 (4-scale column tiles per 128-row tile)
   uint32_t* status;
 };
@@ -359,7 +367,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar_acce + 8 * acc) : "memory");
         }
         const long long col = (long long)tn * BN + c0;
-        if (g.f32_out) {
+        if (g.f32_out && g.wide_st) {
+          // each lane's 128 bytes of its row in 4 stores of full 32-byte sectors
+          float* dp = static_cast<float*>(g.d) + row * g.ldd + col;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint32_t o[8];
+#pragma unroll
+            for (int h = 0; h < 8; ++h) o[h] = __float_as_uint(__fmul_rn(__uint_as_float(r[8 * k + h]), alpha));
+            st_global_v8(dp + 8 * k, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+          }
+        } else if (g.f32_out) {
           float4* dp = reinterpret_cast<float4*>(static_cast<float*>(g.d) + row * g.ldd + col);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
@@ -367,6 +385,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 __fmul_rn(__uint_as_float(r[4 * k + 1]), alpha),
                                 __fmul_rn(__uint_as_float(r[4 * k + 2]), alpha),
                                 __fmul_rn(__uint_as_float(r[4 * k + 3]), alpha));
+        } else if (g.wide_st) {
+          uint16_t* dp = static_cast<uint16_t*>(g.d) + row * g.ldd + col;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            uint32_t o[8];
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[16 * k + 2 * h]), alpha),
+                                                              __fmul_rn(__uint_as_float(r[16 * k + 2 * h + 1]), alpha));
+              o[h] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            st_global_v8(dp + 16 * k, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+          }
         } else {
           uint4* dp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.d) + row * g.ldd + col);
 #pragma unroll
@@ -510,6 +541,7 @@ cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M,
   g.N = N;
   g.K = K;
   g.f32_out = f32_out;
+  g.wide_st = (reinterpret_cast<uintptr_t>(d) % 32 == 0) && (ldd * (f32_out ? 4 : 2)) % 32 == 0;
   g.sf_col_tiles = K / 64;
   g.status = status;
   const bool bn256 = N % 256 == 0;
