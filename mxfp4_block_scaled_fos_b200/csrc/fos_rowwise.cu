@@ -33,8 +33,9 @@ constexpr int kThreads = 256;
 #ifndef FOS_K1_PREFETCH
 #define FOS_K1_PREFETCH 1
 #endif
-// the fused amax + quantize kernel: 5 CTAs per SM, no prefetch (its amax
-// items want the CTAs; 0.729 ms against 0.747 ms with 4 CTAs and prefetch)
+// the fused amax + quantize kernel: the threads of 5 such CTAs per SM, no
+// prefetch (its amax items want the CTAs; 0.729 ms against 0.747 ms with 4
+// CTAs and prefetch)
 #ifndef FOS_FUSED_MIN_BLOCKS
 #define FOS_FUSED_MIN_BLOCKS 5
 #endif
@@ -377,10 +378,9 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 // chunks run side by side on every SM, and with the L + 1 entries in flight
 // smaller than L2 (and the amax reads marked evict-last) the quantize reads
 // hit L2, so HBM sees the input about once.
-// Lag in entries between an entry's amax and its quantize items, and the item
-// sizes in blocks: measured on the 128 x 2880 x 2880 expert batch (lag 2,
-// claims at item end: 0.738 ms for 4/6 against 0.781 ms for lag 3 with
-// claim-ahead; 2048-block quantize items 0.729 ms).
+// Lag in entries between an entry's amax and its quantize items: measured on
+// the 128 x 2880 x 2880 expert batch (lag 2, claims at item end: 0.738 ms for
+// 4/6 against 0.781 ms for lag 3 with claim-ahead).
 #ifndef FOS_FUSED_LAG_46
 #define FOS_FUSED_LAG_46 2
 #endif
@@ -389,6 +389,29 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 #endif
 #ifndef FOS_FUSED_AMAX_UNROLL
 #define FOS_FUSED_AMAX_UNROLL 4
+#endif
+// 1: a CTA claims its next item when it starts an item (the claim's latency
+// hides behind the item, but twice as many items are in flight, so an entry's
+// quantize items reach the queue head while its amax items are still being
+// reduced unless the lag grows); 0: when it ends one
+#ifndef FOS_FUSED_CLAIM_AHEAD
+#define FOS_FUSED_CLAIM_AHEAD 0
+#endif
+// Threads per CTA and item sizes in blocks (amax, quantize) per variant.  The
+// plain 4/6 kernel (round to nearest, codes out), bound by instruction issue,
+// runs 128-thread CTAs so that the barrier at each item end waits on 4 warps,
+// not 8: 0.722 ms against 0.729 ms (256 threads, items of 4096 / 2048 blocks)
+// on the expert batch.  The others keep 256 threads: the 6-only kernel, bound
+// by memory (0.472 ms against 0.481 ms with 128), and the fake-quantizing and
+// Hadamard 4/6 kernels (0.872 against 0.907 ms, 0.048 against 0.052 ms).
+#ifndef FOS_FUSED_SMALL_THREADS
+#define FOS_FUSED_SMALL_THREADS 128
+#endif
+#ifndef FOS_FUSED_SMALL_ACHUNK
+#define FOS_FUSED_SMALL_ACHUNK 2048
+#endif
+#ifndef FOS_FUSED_SMALL_QCHUNK
+#define FOS_FUSED_SMALL_QCHUNK 1024
 #endif
 #ifndef FOS_FUSED_ACHUNK
 #define FOS_FUSED_ACHUNK 4096
@@ -399,18 +422,18 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 #ifndef FOS_FUSED_QCHUNK_6
 #define FOS_FUSED_QCHUNK_6 1536
 #endif
-// 1: a CTA claims its next item when it starts an item (the claim's latency
-// hides behind the item, but twice as many items are in flight, so an entry's
-// quantize items reach the queue head while its amax items are still being
-// reduced unless the lag grows); 0: when it ends one
-#ifndef FOS_FUSED_CLAIM_AHEAD
-#define FOS_FUSED_CLAIM_AHEAD 0
-#endif
-constexpr uint32_t kAChunk = FOS_FUSED_ACHUNK;  // blocks per amax item
-// blocks per quantize item
-template <bool F46>
-constexpr uint32_t qchunk() { return F46 ? FOS_FUSED_QCHUNK_46 : FOS_FUSED_QCHUNK_6; }
-static_assert(qchunk<true>() % 32 == 0 && qchunk<false>() % 32 == 0, "quantize items hold whole choice words");
+template <bool F46, bool SR, bool RHT, bool FAKE>
+struct FusedCfg {
+  static constexpr bool small = F46 && !SR && !RHT && !FAKE;
+  static constexpr int threads = small ? FOS_FUSED_SMALL_THREADS : kThreads;
+  static constexpr uint32_t achunk = small ? FOS_FUSED_SMALL_ACHUNK : FOS_FUSED_ACHUNK;
+  static constexpr uint32_t qchunk = small ? FOS_FUSED_SMALL_QCHUNK : F46 ? FOS_FUSED_QCHUNK_46 : FOS_FUSED_QCHUNK_6;
+  // resident CTAs per SM: the threads of FOS_FUSED_MIN_BLOCKS 256-thread CTAs
+  // (FOS_K1_MIN_BLOCKS_HEAVY with SR or the transform)
+  static constexpr int min_blocks = (SR || RHT ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_FUSED_MIN_BLOCKS) * kThreads / threads;
+  static_assert(threads % 32 == 0 && kThreads % threads == 0, "whole warps, a divisor of 256");
+  static_assert(qchunk % 32 == 0, "quantize items hold whole choice words");
+};
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
@@ -560,11 +583,13 @@ __device__ __forceinline__ void amax_count_in(const QuantArgs& a, uint32_t* amax
 }
 
 template <bool F46, bool SR, bool RHT, bool SWZ, bool DENSE, bool FAKE>
-__global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAVY : FOS_FUSED_MIN_BLOCKS)
+__global__ void __launch_bounds__((FusedCfg<F46, SR, RHT, FAKE>::threads), (FusedCfg<F46, SR, RHT, FAKE>::min_blocks))
     k_q1x16_fused(const QuantArgs a, int batch, const FusedPlan p, uint32_t* amax_ws, uint32_t* done_a,
                   uint32_t* queue) {
   __shared__ float4 s_tab[128];
-  __shared__ uint32_t s_red[kThreads / 32];
+  using Cfg = FusedCfg<F46, SR, RHT, FAKE>;
+  constexpr int NT = Cfg::threads;
+  __shared__ uint32_t s_red[NT / 32];
   __shared__ float s_St;
   __shared__ uint32_t s_item[2];
   const uint32_t mask16 = RHT ? rht_sign_mask(a.seed) : 0u;
@@ -584,15 +609,15 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
 #endif
     const FusedItem it = fused_item(i, batch, p);
     if (it.amax) {
-      const uint32_t lo = it.chunk * kAChunk, hi = min(lo + kAChunk, a.nblk);
-      uint32_t m = slice_amax_bits<RHT, DENSE>(a, it.entry, lo, hi, mask16, pol_keep, threadIdx.x);
+      const uint32_t lo = it.chunk * Cfg::achunk, hi = min(lo + Cfg::achunk, a.nblk);
+      uint32_t m = slice_amax_bits<RHT, DENSE, NT>(a, it.entry, lo, hi, mask16, pol_keep, threadIdx.x);
       m = __reduce_max_sync(0xffffffffu, m);
       if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
       __syncthreads();
       if (threadIdx.x == 0) {
         uint32_t v = 0;
 #pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) v = max(v, s_red[w]);
+        for (int w = 0; w < NT / 32; ++w) v = max(v, s_red[w]);
         amax_count_in(a, amax_ws, done_a, it.entry, v);
       }
     } else {
@@ -609,9 +634,8 @@ __global__ void __launch_bounds__(kThreads, (SR || RHT) ? FOS_K1_MIN_BLOCKS_HEAV
         tab_entry = it.entry;
       }
       if (it.chunk == 0 && threadIdx.x == 0 && a.row.tensor_scale) a.row.tensor_scale[it.entry] = ts.St;
-      const uint32_t lo = it.chunk * qchunk<F46>(), hi = min(lo + qchunk<F46>(), a.nblk);
-      rowwise_range<F46, SR, RHT, SWZ, DENSE, kThreads, FAKE>(a, it.entry, lo, hi, s_tab, ts, mask16, bad,
-                                                              pol_done);
+      const uint32_t lo = it.chunk * Cfg::qchunk, hi = min(lo + Cfg::qchunk, a.nblk);
+      rowwise_range<F46, SR, RHT, SWZ, DENSE, NT, FAKE>(a, it.entry, lo, hi, s_tab, ts, mask16, bad, pol_done);
     }
 #if !FOS_FUSED_CLAIM_AHEAD
     if (threadIdx.x == 0) s_item[k ^ 1] = atomicAdd(queue, 1u);
@@ -924,7 +948,8 @@ static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_
   static std::atomic<int> grid_of[kMaxDevices];
   auto kern = k_q1x16_fused<F46, SR, RHT, SWZ, DENSE, FAKE>;
   FusedPlan plan;
-  if (!make_plan(plan, a.nblk, batch, kAChunk, qchunk<F46>(), F46 ? FOS_FUSED_LAG_46 : FOS_FUSED_LAG_6))
+  using Cfg = FusedCfg<F46, SR, RHT, FAKE>;
+  if (!make_plan(plan, a.nblk, batch, Cfg::achunk, Cfg::qchunk, F46 ? FOS_FUSED_LAG_46 : FOS_FUSED_LAG_6))
     return cudaErrorNotSupported;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
@@ -932,13 +957,13 @@ static cudaError_t launch_fused_t(const QuantArgs& a, int batch, uint32_t* amax_
   if (grid == 0) {
     int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess)
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::threads, 0) != cudaSuccess)
       return cudaErrorNotSupported;
     grid = per_sm >= 1 ? sms * per_sm : -1;
     grid_of[dev].store(grid, std::memory_order_relaxed);
   }
   if (grid < 1) return cudaErrorNotSupported;
-  kern<<<grid, kThreads, 0, st>>>(a, batch, plan, amax_ws, done_a, queue);
+  kern<<<grid, Cfg::threads, 0, st>>>(a, batch, plan, amax_ws, done_a, queue);
   return cudaGetLastError();
 }
 
