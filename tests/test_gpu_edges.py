@@ -1,8 +1,9 @@
 """GPU edge cases through the C ABI: empty tensors, one block, many tiny
 batch entries (the fused amax + quantize queue with one item of each kind
-per entry), and the largest block counts a 16-bit batch index allows with
-small entries.  Checked bit for bit against the oracle where there is
-output."""
+per entry), a few entries with several ragged items each in dense,
+strided and swizzled layouts, and the largest block counts a 16-bit batch
+index allows with small entries.  Checked bit for bit against the oracle
+where there is output."""
 import ctypes
 
 import numpy as np
@@ -12,7 +13,7 @@ import torch
 import mxfp4_block_scaled_fos_b200 as F
 from mxfp4_block_scaled_fos_b200.fos import Options
 
-from helpers import check_quantize, require_gpu, zeroed_out
+from helpers import check_quantize, np_bits, require_gpu, zeroed_out
 
 pytestmark = pytest.mark.gpu
 
@@ -73,3 +74,27 @@ def test_entries_with_all_zero_and_all_tiny_values_in_one_batch():
     x[0] = 0.0
     x[1] *= 1e-39
     check_quantize(x.to(torch.bfloat16).cuda())
+
+
+@pytest.mark.parametrize("layout", ["dense", "ragged_words", "strided", "swizzled"])
+@pytest.mark.parametrize("fmt", ["nvfp4_46", "nvfp4_6"])
+def test_fused_queue_several_items_per_entry(layout, fmt):
+    """Three entries with several amax and quantize items each and a ragged
+    last item, so that with a lag of two entries the middle entry's items
+    interleave with both neighbours' in the queue.  dense: 72 x 1024 (4608
+    blocks, whole choice words per entry: the dense loop); ragged_words:
+    70 x 1040 (4550 blocks, choice words that straddle entries); strided:
+    the same rows read with ld = 1104; swizzled: swizzled scales.  The
+    per-entry scales differ by up to 2^12."""
+    require_gpu()
+    g = torch.Generator().manual_seed(8)
+    rows, cols = (72, 1024) if layout == "dense" else (70, 1040)
+    big = torch.randn(3, rows, 1104, generator=g)
+    big *= torch.exp2(torch.randint(-6, 7, (3, 1, 1), generator=g).float())
+    big = big.to(torch.bfloat16).cuda()
+    if layout == "strided":
+        x = big[:, :, :cols]
+        assert x.stride(1) == 1104
+        check_quantize(x, fmt=fmt, x_bits=np_bits(x.contiguous()))
+    else:
+        check_quantize(big[:, :, :cols].contiguous(), fmt=fmt, swizzle=layout == "swizzled")
