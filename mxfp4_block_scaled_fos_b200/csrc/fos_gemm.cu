@@ -431,27 +431,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 // bytes on) is row l % 32 of two atoms.  pair_tiles = 0: source (t, kt, s)
 // pairs atoms (t, 4 kt + 2 s) and (t, 4 kt + 2 s + 1); pair_tiles = 1:
 // source (p, kt, j) pairs atoms (2 p, 4 kt + j) and (2 p + 1, 4 kt + j).
-// One thread per 16 bytes of the output, in output order.
-__global__ void __launch_bounds__(256) k_expand_sf(const uint8_t* src, long long col_tiles, long long ksteps,
-                                                   unsigned long long nimages, int pair_tiles, uint8_t* dst) {
-  const unsigned long long nchunks = nimages * 256ull;
-  for (unsigned long long q = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x; q < nchunks;
+// One thread per 16 bytes of the output, in output order; both operands'
+// expansions in one launch (A's chunks first, then B's).
+struct ExpandJob {
+  const uint8_t* src;
+  uint8_t* dst;
+  long long col_tiles, ksteps;
+  unsigned long long nchunks;   // 16-byte chunks of dst: images * 256
+  int pair_tiles;
+};
+
+__device__ __forceinline__ void expand_chunk(const ExpandJob& j, unsigned long long q) {
+  const unsigned long long img = q >> 8;
+  const int w = (int)(q & 255);
+  const int half = (w >> 3) & 1, l = ((w >> 4) << 3) | (w & 7);
+  long long tile, ctile;
+  if (!j.pair_tiles) {
+    const long long r = (long long)(img >> 1), kt = r % j.ksteps;
+    tile = r / j.ksteps;
+    ctile = 4 * kt + 2 * (long long)(img & 1) + half;
+  } else {
+    const long long r = (long long)(img >> 2), kt = r % j.ksteps;
+    tile = 2 * (r / j.ksteps) + half;
+    ctile = 4 * kt + (long long)(img & 3);
+  }
+  *reinterpret_cast<uint4*>(j.dst + q * 16) =
+      *reinterpret_cast<const uint4*>(j.src + (tile * j.col_tiles + ctile) * 512 + (l & 31) * 16);
+}
+
+__global__ void __launch_bounds__(256) k_expand_sf(const ExpandJob ja, const ExpandJob jb) {
+  const unsigned long long n = ja.nchunks + jb.nchunks;
+  for (unsigned long long q = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x; q < n;
        q += (unsigned long long)gridDim.x * blockDim.x) {
-    const unsigned long long img = q >> 8;
-    const int w = (int)(q & 255);
-    const int half = (w >> 3) & 1, l = ((w >> 4) << 3) | (w & 7);
-    long long tile, ctile;
-    if (!pair_tiles) {
-      const long long r = (long long)(img >> 1), kt = r % ksteps;
-      tile = r / ksteps;
-      ctile = 4 * kt + 2 * (long long)(img & 1) + half;
-    } else {
-      const long long r = (long long)(img >> 2), kt = r % ksteps;
-      tile = 2 * (r / ksteps) + half;
-      ctile = 4 * kt + (long long)(img & 3);
-    }
-    *reinterpret_cast<uint4*>(dst + q * 16) =
-        *reinterpret_cast<const uint4*>(src + (tile * col_tiles + ctile) * 512 + (l & 31) * 16);
+    if (q < ja.nchunks) expand_chunk(ja, q);
+    else                expand_chunk(jb, q - ja.nchunks);
   }
 }
 
@@ -517,13 +530,20 @@ size_t gemm_workspace_bytes(long long M, long long N, long long K) {
   return (size_t)4 * 512 * (size_t)((M / 128) * (K / 64) + (N / 128) * (K / 64));
 }
 
-static cudaError_t expand_sf(const uint8_t* src, long long rows, int K, int pair_tiles, uint8_t* dst,
-                             cudaStream_t st) {
-  const long long col_tiles = K / 64, ksteps = K / 256;
-  const unsigned long long nimages = (unsigned long long)(rows / 128) * ksteps * 2;
-  const unsigned long long blocks = (nimages * 256 + 255) / 256;
-  k_expand_sf<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(src, col_tiles, ksteps, nimages,
-                                                                               pair_tiles, dst);
+static ExpandJob expand_job(const uint8_t* src, long long rows, int K, int pair_tiles, uint8_t* dst) {
+  ExpandJob j;
+  j.src = src;
+  j.dst = dst;
+  j.col_tiles = K / 64;
+  j.ksteps = K / 256;
+  j.nchunks = (unsigned long long)(rows / 128) * j.ksteps * 2 * 256;
+  j.pair_tiles = pair_tiles;
+  return j;
+}
+
+static cudaError_t expand_sf(const ExpandJob& ja, const ExpandJob& jb, cudaStream_t st) {
+  const unsigned long long blocks = (ja.nchunks + jb.nchunks + 255) / 256;
+  k_expand_sf<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(ja, jb);
   return cudaGetLastError();
 }
 
@@ -548,8 +568,8 @@ cudaError_t launch_gemm_nvfp4(const fos_qtensor* a, const fos_qtensor* b, int M,
   if (workspace) {  // the wide layout: expand both operands' scales, then 6 or 4 copies per K step
     uint8_t* ea = static_cast<uint8_t*>(workspace);
     uint8_t* eb = ea + gemm_workspace_bytes(M, 0, K);
-    cudaError_t e = expand_sf(a->scales, M, K, 0, ea, st);
-    if (e == cudaSuccess) e = expand_sf(b->scales, N, K, bn256 ? 1 : 0, eb, st);
+    const cudaError_t e = expand_sf(expand_job(a->scales, M, K, 0, ea), expand_job(b->scales, N, K, bn256 ? 1 : 0, eb),
+                                    st);
     if (e != cudaSuccess) return e;
     g.sfa = ea;
     g.sfb = eb;
