@@ -162,9 +162,13 @@ def _alloc_qtensor(batch, R, C, fmt, block, flags, device, with_choice, nblocks)
     bs = 32 if fmt == "mxfp4" else 16
     codes = torch.empty(batch, R, C // 2, dtype=torch.uint8, device=device)
     if flags & FLAG_SCALE_SWIZZLED:
-        # zeroed: the library leaves the layout's padding unwritten, and a
-        # tensor-core GEMM reads the padded scales of partial tiles
-        scales = torch.zeros(batch, scales_size(R, C // bs, flags), dtype=torch.uint8, device=device)
+        # zeroed where the layout has padding (rows not a multiple of 128 or
+        # scale columns not a multiple of 4): the library leaves the padding
+        # unwritten, and a tensor-core GEMM reads the padded scales of
+        # partial tiles; without padding the quantizer writes every byte
+        padded = R % 128 != 0 or (C // bs) % 4 != 0
+        alloc = torch.zeros if padded else torch.empty
+        scales = alloc(batch, scales_size(R, C // bs, flags), dtype=torch.uint8, device=device)
     else:
         scales = torch.empty(batch, R, C // bs, dtype=torch.uint8, device=device)
     ts = torch.empty(batch, dtype=torch.float32, device=device) if fmt != "mxfp4" else None

@@ -17,6 +17,8 @@ a reduced batch so a capture stays small), runs one untimed call, then
   weight_2d 4/6 16x16 2D with the transposed copy on 0.02-normal weights (rows x 4096)
   moe_fake  4/6 fake quantization (quantize + dequantize, bf16 out), amax in the call
   gemm      NVFP4 block-scaled GEMM, rows x rows x rows (rows a multiple of 256)
+  linear    one step of the quantized Linear layer, 8192 x 4096 -> 4096: forward,
+            dgrad and wgrad with x and dy quantized in the step (several kernels)
 """
 from __future__ import annotations
 
@@ -95,6 +97,17 @@ def main():
         d = torch.empty(n, n, dtype=torch.bfloat16, device=dev)
         ws = torch.empty(F.gemm_workspace_size(n, n, n), dtype=torch.uint8, device=dev)
         fn = lambda: F.gemm_nvfp4(qa, qb, out=d, workspace=ws)
+    elif c == "linear":
+        # the bench's Linear step: 8192 tokens x 4096 -> 4096, forward, dgrad
+        # and wgrad with x and dy quantized inside the step
+        xl = workloads.activation_outliers(8192, 4096, device=dev)[0]
+        wl = workloads.weight_normal(4096, 4096, device=dev)[0]
+        dyl = workloads.gradient_student_t(8192, 4096, device=dev)[0]
+        qw = F.quantize_weight(wl)
+
+        def fn():
+            _, qx_t = F.linear_forward(xl, qw, save_colwise=True, seed=7)
+            F.linear_backward(dyl, None, qw, seed=7, qx_t=qx_t)
     else:
         raise SystemExit("unknown case " + c)
     fn()
